@@ -1,0 +1,125 @@
+/*
+ * Format B oracle: the 243-word ternary code book, unpacking and the fp64
+ * reference matmul (test infrastructure only; see oref.h).
+ *
+ * Follows "A Discrete Weight Language for Large Language Models"
+ * (alphaneural.io):
+ *   - section 3.2: a weight is the word c = (c_1..c_5) in {-1,0,+1}^5 and
+ *     decodes to alpha * sum_i c_i s_i; the 243 words are enumerated once per
+ *     layer, multiplied by alpha and stored as a 243-entry table; the weight
+ *     matrix is then the matrix of codes in 0..242 (base-3 encoding of the
+ *     word);
+ *   - section 3.3: with a per-row scale rho_n (fp16), W_hat = rho_n LUT[code];
+ *   - section 4.1: one uint8 code per weight (8 bits of storage);
+ *   - section 4.2: rho is applied to the output accumulator.
+ *
+ * Readings where the page leaves a step open:
+ *   B1 the digit order of the code is the one of the five-trits-per-byte
+ *      layout: code = sum_i (c_i + 1) 3^(i-1), c_1 least significant;
+ *   B2 the table is LUT[b] = fp32(alpha * S_b), S_b = sum_{i=1..5} c_i a_i in
+ *      fp64 over ascending i, the ladder a_i and alpha given as fp32;
+ *      entries 243..255 of the padded 256-entry table are NaN;
+ *   B3 rho is optional; row n uses rho[n / rows_per_scale] (per row when
+ *      rows_per_scale = 1, per attention head when it is the head size);
+ *   B4 unpack yields bf16(fp32(rho * LUT[code])), or bf16(LUT[code]) without
+ *      rho; codes >= 243 are OREF_ERR_BAD_CODE;
+ *   B5 the matmul uses the exact weight rho * LUT[code] (fp64).
+ */
+#include <math.h>
+#include <stdlib.h>
+
+#include "oref.h"
+
+int oref_build_lut(float alpha, const float ladder[5], float lut[256]) {
+  if (!ladder || !lut) return OREF_ERR_INVALID_ARG;
+  for (int b = 0; b < 243; ++b) {
+    double sum = 0.0;
+    int rest = b;
+    for (int i = 0; i < 5; ++i) { /* i = 0 is c_1, the least significant */
+      int c = rest % 3 - 1;
+      rest /= 3;
+      sum += (double)c * (double)ladder[i];
+    }
+    lut[b] = oref_f64_to_f32((double)alpha * sum);
+  }
+  for (int b = 243; b < 256; ++b) lut[b] = NAN;
+  return OREF_OK;
+}
+
+static int check_B(const uint8_t *codes, int64_t n, int64_t k,
+                   const float *lut, const uint16_t *rho, int32_t rps) {
+  if (!codes || !lut || n < 0 || k < 0) return OREF_ERR_INVALID_ARG;
+  if (rps < 0) return OREF_ERR_INVALID_ARG;
+  if (rps > 0 && !rho) return OREF_ERR_INVALID_ARG;
+  return OREF_OK;
+}
+
+int oref_unpack_B(const uint8_t *codes, int64_t n, int64_t k, const float *lut,
+                  const uint16_t *rho, int32_t rps, uint16_t *W_out) {
+  int st = check_B(codes, n, k, lut, rho, rps);
+  if (st != OREF_OK) return st;
+  if (!W_out) return OREF_ERR_INVALID_ARG;
+  int status = OREF_OK;
+  for (int64_t r = 0; r < n; ++r) {
+    double scale = (rps > 0) ? oref_f16_to_f64(rho[r / rps]) : 1.0;
+    for (int64_t j = 0; j < k; ++j) {
+      uint8_t c = codes[r * k + j];
+      if (c >= 243 && status == OREF_OK) status = OREF_ERR_BAD_CODE;
+      double v = (double)lut[c];
+      /* rho * LUT: fp16 x fp32 is exact in fp64, then rounded to fp32 */
+      float f = (rps > 0) ? oref_f64_to_f32(scale * v) : (float)v;
+      W_out[r * k + j] = oref_f32_to_bf16(f);
+    }
+  }
+  return status;
+}
+
+int oref_weights_B(const uint8_t *codes, int64_t n, int64_t k, const float *lut,
+                   const uint16_t *rho, int32_t rps, const int64_t *rows,
+                   int64_t nrows, double *w_out) {
+  int st = check_B(codes, n, k, lut, rho, rps);
+  if (st != OREF_OK) return st;
+  if (!w_out) return OREF_ERR_INVALID_ARG;
+  if (!rows) nrows = n;
+  int status = OREF_OK;
+  for (int64_t i = 0; i < nrows; ++i) {
+    int64_t r = rows ? rows[i] : i;
+    if (r < 0 || r >= n) return OREF_ERR_INVALID_ARG;
+    double scale = (rps > 0) ? oref_f16_to_f64(rho[r / rps]) : 1.0;
+    for (int64_t j = 0; j < k; ++j) {
+      uint8_t c = codes[r * k + j];
+      if (c >= 243 && status == OREF_OK) status = OREF_ERR_BAD_CODE;
+      w_out[i * k + j] = scale * (double)lut[c]; /* exact (B5) */
+    }
+  }
+  return status;
+}
+
+int oref_linear_B(const uint8_t *codes, int64_t n, int64_t k, const float *lut,
+                  const uint16_t *rho, int32_t rps, const int64_t *rows,
+                  int64_t nrows, const uint16_t *x, int64_t batch, int64_t ldx,
+                  double *y) {
+  int st = check_B(codes, n, k, lut, rho, rps);
+  if (st != OREF_OK) return st;
+  if (!x || !y || batch < 0 || ldx < k) return OREF_ERR_INVALID_ARG;
+  if (!rows) nrows = n;
+  double *w = (double *)malloc(sizeof(double) * (size_t)(k > 0 ? k : 1));
+  int status = OREF_OK;
+  for (int64_t i = 0; i < nrows; ++i) {
+    int64_t r = rows ? rows[i] : i;
+    if (r < 0 || r >= n) {
+      status = OREF_ERR_INVALID_ARG;
+      break;
+    }
+    int s = oref_weights_B(codes, n, k, lut, rho, rps, &r, 1, w);
+    if (s != OREF_OK && status == OREF_OK) status = s;
+    for (int64_t b = 0; b < batch; ++b) {
+      const uint16_t *xb = x + b * ldx;
+      double acc = 0.0;
+      for (int64_t j = 0; j < k; ++j) acc += w[j] * oref_bf16_to_f64(xb[j]);
+      y[b * nrows + i] = acc;
+    }
+  }
+  free(w);
+  return status;
+}
