@@ -1,0 +1,173 @@
+// C ABI of the tq library: argument validation, the host-side code book
+// builder and dispatch to the kernels. Every check here happens before any
+// launch; kernels report data errors through the caller's status word.
+#include <math.h>
+#include <string.h>
+
+#include "tq_common.cuh"
+
+namespace {
+
+bool aligned(const void *p, uintptr_t a) {
+  return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
+}
+
+tq_status from_cuda(cudaError_t e) {
+  return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
+}
+
+// Validate a weight descriptor; fills `v` on success.
+tq_status check_weights(const tq_weights *w, tq::WeightsView *v) {
+  if (w == nullptr) return TQ_ERR_INVALID_ARG;
+  if (w->n_rows < 0 || w->k_cols < 0) return TQ_ERR_INVALID_ARG;
+  if (w->codes == nullptr) return TQ_ERR_INVALID_ARG;
+  v->format = w->format;
+  v->n = w->n_rows;
+  v->k = w->k_cols;
+  v->codes = w->codes;
+  v->scales = w->scales;
+  v->lut = w->lut;
+  v->group = w->group;
+  v->planes = w->planes;
+  v->rps = w->rows_per_scale;
+  v->codes_plane_stride = 0;
+  v->scales_plane_stride = 0;
+  if (w->format == TQ_FMT_A) {
+    if (w->scales == nullptr) return TQ_ERR_INVALID_ARG;
+    if (w->planes < 1 || w->planes > 2) return TQ_ERR_INVALID_ARG;
+    if (w->group != 64 && w->group != 128) return TQ_ERR_UNSUPPORTED;
+    if (w->k_cols % w->group != 0) return TQ_ERR_SHAPE;
+    const int64_t groups = w->n_rows * (w->k_cols / w->group);
+    const int64_t nb = tq::bytes_per_group(w->group);
+    v->codes_plane_stride =
+        w->codes_plane_stride ? w->codes_plane_stride : groups * nb;
+    v->scales_plane_stride =
+        w->scales_plane_stride ? w->scales_plane_stride : groups;
+    if (w->planes == 2 && (v->codes_plane_stride < groups * nb ||
+                           v->scales_plane_stride < groups))
+      return TQ_ERR_SHAPE;
+    if (w->codes_plane_stride < 0 || w->scales_plane_stride < 0)
+      return TQ_ERR_INVALID_ARG;
+    if (!aligned(w->codes, 16) || !aligned(w->scales, 2))
+      return TQ_ERR_ALIGNMENT;
+  } else if (w->format == TQ_FMT_B) {
+    if (w->planes != 1) return TQ_ERR_INVALID_ARG;
+    if (w->lut == nullptr) return TQ_ERR_INVALID_ARG;
+    if (w->rows_per_scale < 0) return TQ_ERR_INVALID_ARG;
+    if (w->rows_per_scale > 0 && w->scales == nullptr)
+      return TQ_ERR_INVALID_ARG;
+    if (w->k_cols % 16 != 0) return TQ_ERR_SHAPE;
+    if (!aligned(w->codes, 16) || !aligned(w->lut, 16)) return TQ_ERR_ALIGNMENT;
+    if (w->scales != nullptr && !aligned(w->scales, 2)) return TQ_ERR_ALIGNMENT;
+    v->group = 0;
+    if (w->rows_per_scale == 0) v->scales = nullptr;
+  } else {
+    return TQ_ERR_INVALID_ARG;
+  }
+  return TQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t tq_packed_bytes(int32_t format, int64_t n, int64_t k, int32_t group,
+                       int32_t planes) {
+  if (n < 0 || k < 0) return 0;
+  if (format == TQ_FMT_A) {
+    if (group <= 0 || k % group != 0 || planes < 1 || planes > 2) return 0;
+    const size_t groups = (size_t)n * (size_t)(k / group);
+    return (size_t)planes * groups * ((size_t)tq::bytes_per_group(group) + 2);
+  }
+  if (format == TQ_FMT_B) return (size_t)n * (size_t)k + 243u * 4u;
+  return 0;
+}
+
+tq_status tq_build_lut(float alpha, const float ladder[5], float lut_out[256]) {
+  if (ladder == nullptr || lut_out == nullptr) return TQ_ERR_INVALID_ARG;
+  for (int code = 0; code < 243; ++code) {
+    // c_1 is the least significant base-3 digit of the code.
+    double acc = 0.0;
+    int digits = code;
+    for (int i = 0; i < 5; ++i) {
+      const int c = digits % 3 - 1;
+      digits /= 3;
+      acc += (double)c * (double)ladder[i];
+    }
+    lut_out[code] = (float)((double)alpha * acc);
+  }
+  for (int code = 243; code < 256; ++code) lut_out[code] = nanf("");
+  return TQ_OK;
+}
+
+tq_status tq_quantize_pack(const void *W_bf16, int64_t n, int64_t k,
+                           int32_t group, int32_t planes, uint8_t *codes_out,
+                           uint16_t *scales_out, int32_t *dev_status,
+                           void *cuda_stream) {
+  if (W_bf16 == nullptr || codes_out == nullptr || scales_out == nullptr)
+    return TQ_ERR_INVALID_ARG;
+  if (n < 0 || k < 0 || planes < 1 || planes > 2) return TQ_ERR_INVALID_ARG;
+  if (group != 64 && group != 128) return TQ_ERR_UNSUPPORTED;
+  if (k % group != 0) return TQ_ERR_SHAPE;
+  if (!aligned(W_bf16, 16) || !aligned(codes_out, 16) ||
+      !aligned(scales_out, 4))
+    return TQ_ERR_ALIGNMENT;
+  if (dev_status != nullptr && !aligned(dev_status, 4)) return TQ_ERR_ALIGNMENT;
+  if (n == 0 || k == 0) return TQ_OK;
+  return from_cuda(tq::launch_quantize_pack(
+      static_cast<const uint16_t *>(W_bf16), n, k, group, planes, codes_out,
+      scales_out, dev_status, static_cast<cudaStream_t>(cuda_stream)));
+}
+
+tq_status tq_unpack(const tq_weights *w, void *W_bf16_out, int32_t *dev_status,
+                    void *cuda_stream) {
+  tq::WeightsView v;
+  const tq_status st = check_weights(w, &v);
+  if (st != TQ_OK) return st;
+  if (W_bf16_out == nullptr) return TQ_ERR_INVALID_ARG;
+  if (!aligned(W_bf16_out, 16)) return TQ_ERR_ALIGNMENT;
+  if (dev_status != nullptr && !aligned(dev_status, 4)) return TQ_ERR_ALIGNMENT;
+  if (v.n == 0 || v.k == 0) return TQ_OK;
+  return from_cuda(tq::launch_unpack(v, static_cast<uint16_t *>(W_bf16_out),
+                                     dev_status,
+                                     static_cast<cudaStream_t>(cuda_stream)));
+}
+
+tq_status tq_linear(const tq_weights *w, const void *x_bf16, int64_t batch,
+                    int64_t ldx, float *y, int64_t ldy, void *cuda_stream) {
+  tq::WeightsView v;
+  const tq_status st = check_weights(w, &v);
+  if (st != TQ_OK) return st;
+  if (x_bf16 == nullptr || y == nullptr || batch < 1) return TQ_ERR_INVALID_ARG;
+  if (ldx < v.k || ldy < v.n) return TQ_ERR_SHAPE;
+  if (!aligned(x_bf16, 16) || ldx % 8 != 0) return TQ_ERR_ALIGNMENT;
+  if (!aligned(y, 16) || ldy % 4 != 0) return TQ_ERR_ALIGNMENT;
+  if (v.n == 0) return TQ_OK;
+  cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+  if (v.k == 0) {  // empty sum: y = 0
+    return from_cuda(cudaMemset2DAsync(y, (size_t)ldy * sizeof(float), 0,
+                                       (size_t)v.n * sizeof(float),
+                                       (size_t)batch, stream));
+  }
+  return from_cuda(tq::launch_linear(
+      v, static_cast<const __nv_bfloat16 *>(x_bf16), batch, ldx, y, ldy,
+      stream));
+}
+
+const char *tq_status_string(tq_status status) {
+  switch (status) {
+    case TQ_OK: return "TQ_OK";
+    case TQ_ERR_INVALID_ARG: return "TQ_ERR_INVALID_ARG: invalid argument";
+    case TQ_ERR_SHAPE: return "TQ_ERR_SHAPE: inconsistent shape or stride";
+    case TQ_ERR_ALIGNMENT: return "TQ_ERR_ALIGNMENT: misaligned pointer or stride";
+    case TQ_ERR_UNSUPPORTED: return "TQ_ERR_UNSUPPORTED: unsupported parameter";
+    case TQ_ERR_BAD_CODE: return "TQ_ERR_BAD_CODE: invalid code byte";
+    case TQ_ERR_NONFINITE: return "TQ_ERR_NONFINITE: NaN or Inf weight";
+    case TQ_ERR_RANGE: return "TQ_ERR_RANGE: group scale overflows fp16";
+    case TQ_ERR_TIMEOUT: return "TQ_ERR_TIMEOUT: in-kernel wait timed out";
+    case TQ_ERR_CUDA: return "TQ_ERR_CUDA: CUDA error";
+  }
+  return "unknown tq_status";
+}
+
+}  // extern "C"

@@ -1,0 +1,47 @@
+// Shared declarations of the tq CUDA library (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "tq.h"
+
+namespace tq {
+
+constexpr int kLutEntries = 256;  // 243 words + NaN padding
+
+__host__ __device__ constexpr int bytes_per_group(int G) { return (G + 4) / 5; }
+
+// First error wins: the status word moves away from TQ_OK only once.
+__device__ __forceinline__ void report(int32_t *status, int code) {
+  if (status != nullptr) atomicCAS(status, (int32_t)TQ_OK, (int32_t)code);
+}
+
+// Validated, flattened view of a tq_weights descriptor.
+struct WeightsView {
+  int format;
+  int group;
+  int planes;
+  int rps;
+  int64_t n, k;
+  const uint8_t *codes;
+  const uint16_t *scales;  // A: group scales; B: rho or nullptr
+  const float *lut;
+  int64_t codes_plane_stride;   // bytes
+  int64_t scales_plane_stride;  // elements
+};
+
+// ---- launchers (each enqueues on `stream`, returns the launch error) ----
+cudaError_t launch_quantize_pack(const uint16_t *W, int64_t n, int64_t k,
+                                 int G, int planes, uint8_t *codes,
+                                 uint16_t *scales, int32_t *status,
+                                 cudaStream_t stream);
+cudaError_t launch_unpack(const WeightsView &w, uint16_t *out,
+                          int32_t *status, cudaStream_t stream);
+cudaError_t launch_linear(const WeightsView &w, const __nv_bfloat16 *x,
+                          int64_t batch, int64_t ldx, float *y, int64_t ldy,
+                          cudaStream_t stream);
+
+}  // namespace tq

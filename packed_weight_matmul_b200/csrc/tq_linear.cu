@@ -1,0 +1,12 @@
+// Dispatch of tq_linear to the fused matmul kernels.
+#include "tq_linear.cuh"
+
+namespace tq {
+
+cudaError_t launch_linear(const WeightsView &w, const __nv_bfloat16 *x,
+                          int64_t batch, int64_t ldx, float *y, int64_t ldy,
+                          cudaStream_t stream) {
+  return linear_simple(w, x, batch, ldx, y, ldy, stream);
+}
+
+}  // namespace tq

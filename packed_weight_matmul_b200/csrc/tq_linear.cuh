@@ -1,0 +1,13 @@
+// Internal interface of the fused matmul kernels and their dispatcher.
+#pragma once
+
+#include "tq_common.cuh"
+
+namespace tq {
+
+// One warp per row; any shape the boundary accepts.
+cudaError_t linear_simple(const WeightsView &w, const __nv_bfloat16 *x,
+                          int64_t batch, int64_t ldx, float *y, int64_t ldy,
+                          cudaStream_t stream);
+
+}  // namespace tq

@@ -1,0 +1,189 @@
+"""Thin ctypes binding of libtq.so (include/tq.h), for torch tensors.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+library. The names follow the C entry points. Importing this module loads
+libtq.so and raises TqError if it has not been built: there is no fallback.
+
+Device tensors are passed by pointer; the CUDA stream defaults to torch's
+current stream. A non-TQ_OK status raises TqError (status in `.status`).
+"""
+import ctypes as C
+import os
+
+import numpy as np
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                        "libtq.so")
+
+TQ_OK, TQ_ERR_INVALID_ARG, TQ_ERR_SHAPE, TQ_ERR_ALIGNMENT = 0, 1, 2, 3
+TQ_ERR_UNSUPPORTED, TQ_ERR_BAD_CODE, TQ_ERR_NONFINITE = 4, 5, 6
+TQ_ERR_RANGE, TQ_ERR_TIMEOUT, TQ_ERR_CUDA = 7, 8, 9
+TQ_FMT_A, TQ_FMT_B = 1, 2
+
+# Every entry point declared in include/tq.h.
+ENTRY_POINTS = ("tq_packed_bytes", "tq_build_lut", "tq_quantize_pack",
+                "tq_unpack", "tq_linear", "tq_status_string")
+
+
+class TqError(RuntimeError):
+    def __init__(self, status, what=""):
+        msg = _lib.tq_status_string(status).decode() if _lib else str(status)
+        super().__init__(f"{what}: {msg}" if what else msg)
+        self.status = status
+
+
+class tq_weights(C.Structure):
+    _fields_ = [("format", C.c_int32), ("group", C.c_int32),
+                ("planes", C.c_int32), ("rows_per_scale", C.c_int32),
+                ("n_rows", C.c_int64), ("k_cols", C.c_int64),
+                ("codes", C.c_void_p), ("scales", C.c_void_p),
+                ("lut", C.c_void_p), ("codes_plane_stride", C.c_int64),
+                ("scales_plane_stride", C.c_int64)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            f"{LIB_PATH} is missing: build it with "
+            "`python -m packed_weight_matmul_b200.build`")
+    L = C.CDLL(LIB_PATH)
+    i32, i64, P = C.c_int32, C.c_int64, C.c_void_p
+    L.tq_packed_bytes.restype = C.c_size_t
+    L.tq_packed_bytes.argtypes = [i32, i64, i64, i32, i32]
+    L.tq_build_lut.restype = C.c_int
+    L.tq_build_lut.argtypes = [C.c_float, P, P]
+    L.tq_quantize_pack.restype = C.c_int
+    L.tq_quantize_pack.argtypes = [P, i64, i64, i32, i32, P, P, P, P]
+    L.tq_unpack.restype = C.c_int
+    L.tq_unpack.argtypes = [C.POINTER(tq_weights), P, P, P]
+    L.tq_linear.restype = C.c_int
+    L.tq_linear.argtypes = [C.POINTER(tq_weights), P, i64, i64, P, i64, P]
+    L.tq_status_string.restype = C.c_char_p
+    L.tq_status_string.argtypes = [C.c_int]
+    return L
+
+
+_lib = None
+_lib = _load()
+
+
+def lib():
+    return _lib
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return stream
+
+
+def _check(status, what):
+    if status != TQ_OK:
+        raise TqError(status, what)
+
+
+# ---- host entry points --------------------------------------------------------
+
+def tq_packed_bytes(fmt: int, n: int, k: int, group: int = 64,
+                    planes: int = 1) -> int:
+    return _lib.tq_packed_bytes(fmt, n, k, group, planes)
+
+
+def tq_build_lut(alpha: float, ladder) -> np.ndarray:
+    lad = np.ascontiguousarray(np.asarray(ladder, np.float32))
+    assert lad.shape == (5,)
+    out = np.zeros(256, np.float32)
+    _check(_lib.tq_build_lut(C.c_float(alpha),
+                             lad.ctypes.data_as(C.c_void_p),
+                             out.ctypes.data_as(C.c_void_p)), "tq_build_lut")
+    return out
+
+
+def tq_status_string(status: int) -> str:
+    return _lib.tq_status_string(status).decode()
+
+
+# ---- weight descriptors --------------------------------------------------------
+
+class Weights:
+    """A tq_weights descriptor that keeps its tensors alive."""
+
+    def __init__(self, desc: tq_weights, keep):
+        self.desc = desc
+        self._keep = keep
+
+    @property
+    def n(self):
+        return self.desc.n_rows
+
+    @property
+    def k(self):
+        return self.desc.k_cols
+
+
+def weights_a(codes, scales, n, k, group=64, planes=1, codes_plane_stride=0,
+              scales_plane_stride=0) -> Weights:
+    d = tq_weights(format=TQ_FMT_A, group=group, planes=planes,
+                   rows_per_scale=0, n_rows=n, k_cols=k, codes=_ptr(codes),
+                   scales=_ptr(scales), lut=None,
+                   codes_plane_stride=codes_plane_stride,
+                   scales_plane_stride=scales_plane_stride)
+    return Weights(d, (codes, scales))
+
+
+def weights_b(codes, lut, rho=None, rows_per_scale=0, n=None, k=None) -> Weights:
+    if n is None:
+        n, k = codes.shape
+    d = tq_weights(format=TQ_FMT_B, group=0, planes=1,
+                   rows_per_scale=rows_per_scale if rho is not None else 0,
+                   n_rows=n, k_cols=k, codes=_ptr(codes), scales=_ptr(rho),
+                   lut=_ptr(lut), codes_plane_stride=0, scales_plane_stride=0)
+    return Weights(d, (codes, lut, rho))
+
+
+# ---- GPU entry points -----------------------------------------------------------
+
+def tq_quantize_pack(W, group, planes, codes_out, scales_out, dev_status=None,
+                     stream=None, n=None, k=None, check=True):
+    if n is None:
+        n, k = W.shape
+    st = _lib.tq_quantize_pack(_ptr(W), n, k, group, planes, _ptr(codes_out),
+                               _ptr(scales_out), _ptr(dev_status),
+                               _stream(stream))
+    if check:
+        _check(st, "tq_quantize_pack")
+    return st
+
+
+def tq_unpack(w: Weights, out, dev_status=None, stream=None, check=True):
+    st = _lib.tq_unpack(C.byref(w.desc), _ptr(out), _ptr(dev_status),
+                        _stream(stream))
+    if check:
+        _check(st, "tq_unpack")
+    return st
+
+
+def tq_linear(w: Weights, x, y, batch=None, ldx=None, ldy=None, stream=None,
+              check=True):
+    if batch is None:
+        batch = x.shape[0]
+    if ldx is None:
+        ldx = x.stride(0) if x.dim() == 2 else w.k
+    if ldy is None:
+        ldy = y.stride(0) if y.dim() == 2 else w.n
+    st = _lib.tq_linear(C.byref(w.desc), _ptr(x), batch, ldx, _ptr(y), ldy,
+                        _stream(stream))
+    if check:
+        _check(st, "tq_linear")
+    return st
