@@ -144,7 +144,7 @@ tq_status tq_unpack(const tq_weights *w, void *W_bf16_out, int32_t *dev_status,
  *   A: y[b][n] = sum_p sum_g s_p[n][g] sum_{j in g} t_p[n][j] x[b][j]
  *   B: y[b][n] = rho[n / rows_per_scale] * sum_k LUT[code[n][k]] x[b][k]
  *   x     device, bf16 [batch][ldx], 16-byte aligned, ldx >= k, ldx % 8 == 0.
- *   y     device, fp32 [batch][ldy], 16-byte aligned, ldy >= n, ldy % 4 == 0.
+ *   y     device, fp32 [batch][ldy], 4-byte aligned, ldy >= n.
  *         Overwritten. fp32 accumulation.
  *   batch >= 1 (1..64 per pass; larger batches run in passes of 64).
  * Codes are not validated here (tq_unpack does that): a Format B code >= 243

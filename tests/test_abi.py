@@ -111,8 +111,7 @@ def test_validation_before_launch(tq):
     assert _linear(tq, _wa(tq), ldy=2) == E.TQ_ERR_SHAPE
     assert _linear(tq, _wa(tq), x=0x40002) == E.TQ_ERR_ALIGNMENT
     assert _linear(tq, _wa(tq), ldx=132) == E.TQ_ERR_ALIGNMENT
-    assert _linear(tq, _wa(tq), y=0x50004) == E.TQ_ERR_ALIGNMENT
-    assert _linear(tq, _wa(tq), ldy=6) == E.TQ_ERR_ALIGNMENT
+    assert _linear(tq, _wa(tq), y=0x50002) == E.TQ_ERR_ALIGNMENT
     assert _linear(tq, _wa(tq, planes=2, codes_plane_stride=10)) == \
         E.TQ_ERR_SHAPE
     assert _linear(tq, _wb(tq, lut=None)) == E.TQ_ERR_INVALID_ARG
