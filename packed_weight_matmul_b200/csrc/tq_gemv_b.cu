@@ -8,14 +8,17 @@
 //   - Inside a CTA every warp sees every row of the CTA but only its own
 //     k-chunks (chunk = 32 lanes x KPL codes): the chunk count is chosen per
 //     shape so that it divides evenly among the warps.
+//   - Codes stream through a per-warp ring of shared-memory stages filled by
+//     cp.async (16 B per lane and row, L2 only), several row groups ahead of
+//     the math and continuously across chunks. Each lane reads back exactly
+//     the bytes its own copies wrote.
 //   - x for the warp's chunk is converted once to fp32 and kept in registers
-//     while the warp walks the CTA's rows, R rows at a time, with the next
-//     group's code loads in flight (128-bit coalesced loads, streamed).
-//   - The 243-entry code book is replicated once per lane in shared memory:
-//     entry e of lane l's copy sits at byte e*256 + 4*l (all 256 byte
-//     values, so an invalid code reads its NaN entry), so a warp's 32
-//     random lookups hit 32 distinct banks, and one byte-permute builds the
-//     address from the code byte.
+//     while the warp walks the CTA's rows, R rows at a time; the next chunk's
+//     x is fetched one row group early.
+//   - The code book is replicated once per lane in shared memory: entry e of
+//     lane l's copy sits at byte e*128 + 4*l (all 256 byte values, so an
+//     invalid code reads its NaN entry): a warp's 32 random lookups hit 32
+//     distinct banks.
 //   - Products accumulate in fp32 with packed FFMA2 over k pairs; per row
 //     group the R*B partial sums are reduced across lanes with a transposing
 //     butterfly (about 2 shuffles per value instead of 5), summed over the
@@ -27,47 +30,40 @@
 namespace tq {
 namespace {
 
-constexpr int kLutStride = 256;                 // bytes per code-book entry
-constexpr int kLutBytes = 256 * kLutStride;     // all byte values: 64 KB
+constexpr int kLutStride = 128;              // bytes per code-book entry
+constexpr int kLutBytes = 256 * kLutStride;  // all byte values: 32 KB
 constexpr int kMaxWarps = 8;
 constexpr int kCtasPerSm = 2;
+constexpr int kStages = 4;                   // row groups in flight per warp
 
-__device__ __forceinline__ uint4 ld_stream16(const void *p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
 }
 
-__device__ __forceinline__ uint2 ld_stream8(const void *p) {
-  uint2 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
-               : "=r"(v.x), "=r"(v.y)
-               : "l"(p));
-  return v;
-}
-
-__device__ __forceinline__ uint32_t ld_stream4(const void *p) {
-  uint32_t v;
-  asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];"
-               : "=r"(v)
-               : "l"(p));
-  return v;
-}
-
-// Load KPL code bytes as KPL/4 words.
-template <int KPL>
-__device__ __forceinline__ void load_codes(const uint8_t *p, uint32_t *w) {
-  if constexpr (KPL == 16) {
-    const uint4 v = ld_stream16(p);
-    w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
-  } else if constexpr (KPL == 8) {
-    const uint2 v = ld_stream8(p);
-    w[0] = v.x; w[1] = v.y;
+// Asynchronous global -> shared copy of BYTES (16 or 8) bytes; src_size 0
+// writes zeros and reads nothing.
+template <int BYTES>
+__device__ __forceinline__ void cp_async(uint32_t dst, const void *src,
+                                         bool valid) {
+  const int n = valid ? BYTES : 0;
+  if constexpr (BYTES == 16) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst),
+                 "l"(src), "r"(n)
+                 : "memory");
   } else {
-    w[0] = ld_stream4(p);
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(dst),
+                 "l"(src), "r"(n)
+                 : "memory");
   }
+}
+
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 // bf16 pair (low half = lower k) -> float2.
@@ -75,12 +71,12 @@ __device__ __forceinline__ float2 bf16x2_to_float2(uint32_t u) {
   return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
 }
 
-// Code-book value of byte q of word w for this lane (lane4 = 4 * lane).
+// Code-book value of byte q of word w for this lane (lane8 = 8 * lane): the
+// byte permute yields code*256 + 8*lane, halved to code*128 + 4*lane.
 __device__ __forceinline__ float lut_at(const uint8_t *lut_smem, uint32_t w,
-                                        int q, uint32_t lane4) {
-  // result bytes: [0] = lane4, [1] = code byte q, [2], [3] = 0 (lane4 < 256)
-  const uint32_t addr = __byte_perm(w, lane4, 0x5504u | ((uint32_t)q << 4));
-  return *reinterpret_cast<const float *>(lut_smem + addr);
+                                        int q, uint32_t lane8) {
+  const uint32_t a2 = __byte_perm(w, lane8, 0x5504u | ((uint32_t)q << 4));
+  return *reinterpret_cast<const float *>(lut_smem + (a2 >> 1));
 }
 
 // Reduce M (power of two, <= 32) per-lane values across the warp. On return
@@ -107,16 +103,26 @@ __device__ __forceinline__ float butterfly_reduce(float *v, int lane) {
   return v[0];
 }
 
-template <int B>
-struct RowsPerGroup {
-  static constexpr int value = (B <= 2) ? 4 : ((B <= 4) ? 4 : 2);
-};
-
 constexpr int pow2_ceil(int v) {
   int p = 1;
   while (p < v) p *= 2;
   return p;
 }
+
+template <int B>
+struct Rows {  // rows per group
+  static constexpr int value = (B <= 2) ? 4 : 2;
+};
+
+template <int B, int KPL>
+struct GemvBShape {
+  static constexpr int R = Rows<B>::value;
+  static constexpr int M = pow2_ceil(R * B);  // values reduced per group
+  static constexpr int KC = 32 * KPL;         // k per warp chunk
+  static constexpr int NW = KPL / 4;          // code words per lane per row
+  static constexpr int SLOT = R * 32 * KPL;   // ring-slot bytes per warp
+  static constexpr int RING = kStages * SLOT; // ring bytes per warp
+};
 
 template <int B, int KPL>
 __global__ void __launch_bounds__(kMaxWarps * 32, kCtasPerSm)
@@ -125,115 +131,143 @@ __global__ void __launch_bounds__(kMaxWarps * 32, kCtasPerSm)
                   const uint16_t *__restrict__ rho, int rps,
                   const __nv_bfloat16 *__restrict__ x, int64_t ldx,
                   float *__restrict__ y, int64_t ldy, int rows_max) {
-  constexpr int R = RowsPerGroup<B>::value;
-  constexpr int M = pow2_ceil(R * B);  // values reduced per row group
-  constexpr int KC = 32 * KPL;         // k per warp chunk
-  constexpr int NW = KPL / 4;          // code words per lane per row
+  using S = GemvBShape<B, KPL>;
+  constexpr int R = S::R, M = S::M, KC = S::KC, NW = S::NW;
   extern __shared__ __align__(16) uint8_t smem[];
-  float *red = reinterpret_cast<float *>(smem + kLutBytes);  // [warps][rows_max][B]
-
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nwarps = blockDim.x >> 5;
+  uint8_t *ring = smem + kLutBytes + warp * S::RING;
+  float *red = reinterpret_cast<float *>(smem + kLutBytes + nwarps * S::RING);
+
   const int64_t row_lo = (int64_t)blockIdx.x * n / gridDim.x;
   const int rows = (int)((int64_t)(blockIdx.x + 1) * n / gridDim.x - row_lo);
   const uint8_t *crow = codes + row_lo * k;
+  const int64_t nchunks = (k + KC - 1) / KC;
+  const int nc_w = (int)((nchunks - warp + nwarps - 1) / nwarps);  // my chunks
+  const int ng = (rows + R - 1) / R;                               // row groups
+  const int total = nc_w * ng;
 
-  // Replicate the code book (all 256 entries, so an invalid code reads its
-  // NaN entry): word e*64 + l holds LUT[e] for lane l.
-  float *lut_words = reinterpret_cast<float *>(smem);
-  for (int i = threadIdx.x; i < 256 * 32; i += blockDim.x)
-    lut_words[(i >> 5) * 64 + (i & 31)] = __ldg(lut + (i >> 5));
+  // Issue the copies of item i (chunk i / ng, row group i % ng) into its slot.
+  auto issue = [&](int i) {
+    const int ci = i / ng, g = i % ng;
+    const int64_t kb = (warp + (int64_t)ci * nwarps) * KC + (int64_t)lane * KPL;
+    const bool lane_ok = kb < k;
+    const uint32_t dst = smem_addr(ring + (i % kStages) * S::SLOT) + lane * KPL;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int row = g * R + r;
+      const bool ok = lane_ok && row < rows;
+      cp_async<KPL>(dst + r * 32 * KPL, ok ? crow + (int64_t)row * k + kb : codes,
+                    ok);
+    }
+  };
+  // Raw bf16 words of x for chunk ci (this lane's KPL columns).
+  uint32_t xr[B][KPL / 2];
+  auto load_x = [&](int ci) {
+    const int64_t kb = (warp + (int64_t)ci * nwarps) * KC + (int64_t)lane * KPL;
+#pragma unroll
+    for (int b = 0; b < B; ++b) {
+#pragma unroll
+      for (int i = 0; i < KPL / 2; i += 4) {
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (ci < nc_w && kb < k)
+          v = *reinterpret_cast<const uint4 *>(x + b * ldx + kb + 2 * i);
+        xr[b][i] = v.x;
+        xr[b][i + 1] = v.y;
+        xr[b][i + 2] = v.z;
+        xr[b][i + 3] = v.w;
+      }
+    }
+  };
+
+  // Start the code stream and the first x before building the code book.
+#pragma unroll
+  for (int p = 0; p < kStages - 1; ++p) {
+    if (p < total) issue(p);
+    cp_async_commit();
+  }
+  load_x(0);
+
+  // Replicate the code book, coalesced loads and conflict-free 16 B stores:
+  // entry e's 32 lane copies are 8 float4 chunks, written in rotated order.
+  for (int e = threadIdx.x; e < 256; e += blockDim.x) {
+    const float v = __ldg(lut + e);
+    const float4 v4 = make_float4(v, v, v, v);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int jj = (j + e) & 7;
+      *reinterpret_cast<float4 *>(smem + e * kLutStride + jj * 16) = v4;
+    }
+  }
   for (int i = threadIdx.x; i < nwarps * rows_max * B; i += blockDim.x)
     red[i] = 0.0f;
   __syncthreads();
 
-  const uint32_t lane4 = (uint32_t)lane * 4u;
-  const int64_t nchunks = (k + KC - 1) / KC;
-  for (int64_t c = warp; c < nchunks; c += nwarps) {
-    const int64_t kb = c * KC + (int64_t)lane * KPL;
-    const bool valid = kb < k;  // k % 16 == 0: a lane is all in or all out
-    float2 xv[B][KPL / 2];
+  const uint32_t lane8 = (uint32_t)lane * 8u;
+  float2 xv[B][KPL / 2];
+  bool lane_ok = false;
+  for (int i = 0; i < total; ++i) {
+    if (i + kStages - 1 < total) issue(i + kStages - 1);
+    cp_async_commit();
+    cp_async_wait<kStages - 1>();  // item i's copies have landed
+    const int ci = i / ng, g = i % ng;
+    if (g == 0) {
+      const int64_t kb =
+          (warp + (int64_t)ci * nwarps) * KC + (int64_t)lane * KPL;
+      lane_ok = kb < k;
 #pragma unroll
-    for (int b = 0; b < B; ++b) {
-      if (valid) {
-        const __nv_bfloat16 *xp = x + b * ldx + kb;
-        uint32_t u[KPL / 2];
+      for (int b = 0; b < B; ++b)
+#pragma unroll
+        for (int q = 0; q < KPL / 2; ++q) xv[b][q] = bf16x2_to_float2(xr[b][q]);
+      load_x(ci + 1);  // next chunk's x, consumed ng groups later
+    }
+    float2 acc[R][B];
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int b = 0; b < B; ++b) acc[r][b] = make_float2(0.f, 0.f);
+    if (lane_ok) {
+      const uint8_t *slot = ring + (i % kStages) * S::SLOT + lane * KPL;
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        uint32_t cw[NW];
         if constexpr (KPL == 16) {
-          const uint4 a = *reinterpret_cast<const uint4 *>(xp);
-          const uint4 d = *reinterpret_cast<const uint4 *>(xp + 8);
-          u[0] = a.x; u[1] = a.y; u[2] = a.z; u[3] = a.w;
-          u[4] = d.x; u[5] = d.y; u[6] = d.z; u[7] = d.w;
-        } else if constexpr (KPL == 8) {
-          const uint4 a = *reinterpret_cast<const uint4 *>(xp);
-          u[0] = a.x; u[1] = a.y; u[2] = a.z; u[3] = a.w;
+          const uint4 v = *reinterpret_cast<const uint4 *>(slot + r * 32 * KPL);
+          cw[0] = v.x; cw[1] = v.y; cw[2] = v.z; cw[3] = v.w;
         } else {
-          const uint2 a = *reinterpret_cast<const uint2 *>(xp);
-          u[0] = a.x; u[1] = a.y;
+          const uint2 v = *reinterpret_cast<const uint2 *>(slot + r * 32 * KPL);
+          cw[0] = v.x; cw[1] = v.y;
         }
 #pragma unroll
-        for (int i = 0; i < KPL / 2; ++i) xv[b][i] = bf16x2_to_float2(u[i]);
-      } else {
-#pragma unroll
-        for (int i = 0; i < KPL / 2; ++i) xv[b][i] = make_float2(0.f, 0.f);
-      }
-    }
-
-    // software pipeline over row groups: codes of group g+1 load during g
-    uint32_t cw[R][NW], cn[R][NW];
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-#pragma unroll
-      for (int i = 0; i < NW; ++i) cw[r][i] = 0x79797979u;  // code 121 = 0
-      if (valid && r < rows) load_codes<KPL>(crow + (int64_t)r * k + kb, cw[r]);
-    }
-    for (int r0 = 0; r0 < rows; r0 += R) {
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-#pragma unroll
-        for (int i = 0; i < NW; ++i) cn[r][i] = 0x79797979u;
-        const int rn = r0 + R + r;
-        if (valid && rn < rows)
-          load_codes<KPL>(crow + (int64_t)rn * k + kb, cn[r]);
-      }
-      float2 acc[R][B];
-#pragma unroll
-      for (int r = 0; r < R; ++r)
-#pragma unroll
-        for (int b = 0; b < B; ++b) acc[r][b] = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-#pragma unroll
-        for (int i = 0; i < NW; ++i) {
+        for (int wi = 0; wi < NW; ++wi) {
 #pragma unroll
           for (int q = 0; q < 4; q += 2) {
-            const float2 wv = make_float2(lut_at(smem, cw[r][i], q, lane4),
-                                          lut_at(smem, cw[r][i], q + 1, lane4));
+            const float2 wv = make_float2(lut_at(smem, cw[wi], q, lane8),
+                                          lut_at(smem, cw[wi], q + 1, lane8));
 #pragma unroll
             for (int b = 0; b < B; ++b)
-              acc[r][b] = __ffma2_rn(wv, xv[b][i * 2 + q / 2], acc[r][b]);
+              acc[r][b] = __ffma2_rn(wv, xv[b][wi * 2 + q / 2], acc[r][b]);
           }
         }
       }
-      float v[M];
+    }
+    float v[M];
 #pragma unroll
-      for (int r = 0; r < R; ++r)
+    for (int r = 0; r < R; ++r)
 #pragma unroll
-        for (int b = 0; b < B; ++b) v[r * B + b] = acc[r][b].x + acc[r][b].y;
+      for (int b = 0; b < B; ++b) v[r * B + b] = acc[r][b].x + acc[r][b].y;
 #pragma unroll
-      for (int i = R * B; i < M; ++i) v[i] = 0.0f;
-      const float s = butterfly_reduce<M>(v, lane);
-      constexpr int kLowBits = 32 / M;  // lanes sharing one reduced value
-      const int idx = lane / kLowBits;
-      if ((lane % kLowBits) == 0 && idx < R * B) {
-        const int r = idx / B, b = idx % B;
-        if (r0 + r < rows) red[(warp * rows_max + r0 + r) * B + b] += s;
-      }
-#pragma unroll
-      for (int r = 0; r < R; ++r)
-#pragma unroll
-        for (int i = 0; i < NW; ++i) cw[r][i] = cn[r][i];
+    for (int q = R * B; q < M; ++q) v[q] = 0.0f;
+    const float s = butterfly_reduce<M>(v, lane);
+    constexpr int kLow = 32 / M;  // lanes holding the same reduced value
+    const int idx = lane / kLow;
+    if ((lane % kLow) == 0 && idx < R * B) {
+      const int r = idx / B, b = idx % B;
+      const int row = g * R + r;
+      if (row < rows) red[(warp * rows_max + row) * B + b] += s;
     }
   }
+  cp_async_wait<0>();
   __syncthreads();
   for (int i = threadIdx.x; i < rows * B; i += blockDim.x) {
     const int r = i / B, b = i % B;
@@ -253,16 +287,14 @@ struct ChunkPlan {
   int warps;
 };
 
-ChunkPlan plan_chunks(int64_t k, int kpl_max) {
-  ChunkPlan best{4, 1};
+ChunkPlan plan_chunks(int64_t k) {
+  ChunkPlan best{8, 1};
   double best_eff = -1.0;
-  for (int kpl = kpl_max; kpl >= 4; kpl /= 2) {
+  for (int kpl = 16; kpl >= 8; kpl /= 2) {
     const int64_t nchunks = (k + 32 * kpl - 1) / (32 * kpl);
     const int wmax = (int)(nchunks < kMaxWarps ? nchunks : kMaxWarps);
     for (int w = wmax; w >= 1 && w >= wmax - 4; --w) {
       const int64_t rounds = (nchunks + w - 1) / w;
-      // useful lane-chunks over issued lane-chunks (a partial last chunk
-      // counts by its valid lanes)
       const double useful = (double)k / (32.0 * kpl);
       const double eff = useful / (double)(rounds * w) * (w >= 4 ? 1.0 : 0.9);
       if (eff > best_eff + 1e-9) {
@@ -278,16 +310,18 @@ template <int B, int KPL>
 cudaError_t launch_kpl(const WeightsView &w, const __nv_bfloat16 *x,
                        int64_t ldx, float *y, int64_t ldy, int warps,
                        cudaStream_t stream) {
+  using S = GemvBShape<B, KPL>;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  constexpr int kMaxRedBytes = 96 * 1024;
+  constexpr int kMaxRedBytes = 16 * 1024;
   const int64_t rows_cap = kMaxRedBytes / (warps * B * 4);
   int64_t ctas = (int64_t)sms * kCtasPerSm;
   if ((w.n + ctas - 1) / ctas > rows_cap) ctas = (w.n + rows_cap - 1) / rows_cap;
   if (ctas > w.n) ctas = w.n;
   const int rows_max = (int)((w.n + ctas - 1) / ctas);
-  const size_t smem = kLutBytes + (size_t)warps * rows_max * B * sizeof(float);
+  const size_t smem = kLutBytes + (size_t)warps * S::RING +
+                      (size_t)warps * rows_max * B * sizeof(float);
   auto kern = gemv_b_kernel<B, KPL>;
   cudaError_t e = cudaFuncSetAttribute(
       kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -300,23 +334,15 @@ cudaError_t launch_kpl(const WeightsView &w, const __nv_bfloat16 *x,
 template <int B>
 cudaError_t launch_b(const WeightsView &w, const __nv_bfloat16 *x, int64_t ldx,
                      float *y, int64_t ldy, cudaStream_t stream) {
-  constexpr int kplMax = (B <= 2) ? 16 : ((B <= 4) ? 8 : 4);
-  const ChunkPlan p = plan_chunks(w.k, kplMax);
-  if (p.kpl == 16) {
-    if constexpr (kplMax >= 16)
-      return launch_kpl<B, 16>(w, x, ldx, y, ldy, p.warps, stream);
-  }
-  if (p.kpl >= 8) {
-    if constexpr (kplMax >= 8)
-      return launch_kpl<B, 8>(w, x, ldx, y, ldy, p.warps, stream);
-  }
-  return launch_kpl<B, 4>(w, x, ldx, y, ldy, p.warps, stream);
+  const ChunkPlan p = plan_chunks(w.k);
+  if (p.kpl == 16) return launch_kpl<B, 16>(w, x, ldx, y, ldy, p.warps, stream);
+  return launch_kpl<B, 8>(w, x, ldx, y, ldy, p.warps, stream);
 }
 
 }  // namespace
 
 bool gemv_b_supported(const WeightsView &w, int64_t batch) {
-  return w.format == TQ_FMT_B && batch >= 1 && batch <= 8;
+  return w.format == TQ_FMT_B && batch >= 1 && batch <= 4;
 }
 
 cudaError_t gemv_b(const WeightsView &w, const __nv_bfloat16 *x, int64_t batch,
@@ -325,11 +351,7 @@ cudaError_t gemv_b(const WeightsView &w, const __nv_bfloat16 *x, int64_t batch,
     case 1: return launch_b<1>(w, x, ldx, y, ldy, stream);
     case 2: return launch_b<2>(w, x, ldx, y, ldy, stream);
     case 3: return launch_b<3>(w, x, ldx, y, ldy, stream);
-    case 4: return launch_b<4>(w, x, ldx, y, ldy, stream);
-    case 5: return launch_b<5>(w, x, ldx, y, ldy, stream);
-    case 6: return launch_b<6>(w, x, ldx, y, ldy, stream);
-    case 7: return launch_b<7>(w, x, ldx, y, ldy, stream);
-    default: return launch_b<8>(w, x, ldx, y, ldy, stream);
+    default: return launch_b<4>(w, x, ldx, y, ldy, stream);
   }
 }
 

@@ -10,7 +10,7 @@ cudaError_t linear_simple(const WeightsView &w, const __nv_bfloat16 *x,
                           int64_t batch, int64_t ldx, float *y, int64_t ldy,
                           cudaStream_t stream);
 
-// Format B, batch 1..8: CUDA-core GEMV with a replicated code book.
+// Format B, batch 1..4: CUDA-core GEMV with a replicated code book.
 bool gemv_b_supported(const WeightsView &w, int64_t batch);
 cudaError_t gemv_b(const WeightsView &w, const __nv_bfloat16 *x, int64_t batch,
                    int64_t ldx, float *y, int64_t ldy, cudaStream_t stream);
