@@ -2,68 +2,50 @@
 // 3.3 and 4.2): y[b][n] = rho[n / rps] * sum_k LUT[code[n][k]] * x[b][k].
 //
 // HBM-bound: one code byte per weight is read once; everything else lives on
-// chip.
-//   - Grid: one CTA per resident slot (a multiple of the SM count); CTA i
-//     owns rows [i*n/P, (i+1)*n/P), an even share of the matrix.
-//   - Inside a CTA every warp sees every row of the CTA but only its own
-//     k-chunks (chunk = 32 lanes x KPL codes): the chunk count is chosen per
-//     shape so that it divides evenly among the warps.
-//   - Codes stream through a per-warp ring of shared-memory stages filled by
-//     cp.async (16 B per lane and row, L2 only), several row groups ahead of
-//     the math and continuously across chunks. Each lane reads back exactly
-//     the bytes its own copies wrote.
-//   - x for the warp's chunk is converted once to fp32 and kept in registers
-//     while the warp walks the CTA's rows, R rows at a time; the next chunk's
-//     x is fetched one row group early.
+// chip. The design keeps the per-weight instruction count near three (one
+// byte permute, one shared load, one FFMA) and the SM full of warps:
+//   - Grid: one CTA per SM; CTA i owns rows [i*n/P, (i+1)*n/P), an even share
+//     of the matrix. The CTA is large (up to 32 warps) so that many 16-byte
+//     code loads are in flight per SM while registers stay under 64.
+//   - Warps are arranged as WK x WR: the WK warps of a row slice split the
+//     k-chunks (chunk = 32 lanes x KPL codes; KPL and WK are chosen per shape
+//     so the chunks divide evenly), the WR slices split the CTA's rows.
+//   - x for the warp's chunk is converted to fp32 once and kept in registers
+//     while the warp walks its rows, R at a time; the next row group's codes
+//     (and, at a chunk's start, the next chunk's x) are loaded a step ahead,
+//     128-bit, streaming past L1.
 //   - The code book is replicated once per lane in shared memory: entry e of
-//     lane l's copy sits at byte e*128 + 4*l (all 256 byte values, so an
-//     invalid code reads its NaN entry): a warp's 32 random lookups hit 32
-//     distinct banks.
-//   - Products accumulate in fp32 with packed FFMA2 over k pairs; per row
-//     group the R*B partial sums are reduced across lanes with a transposing
-//     butterfly (about 2 shuffles per value instead of 5), summed over the
-//     warp's chunks in shared memory, then over warps in a fixed order:
-//     deterministic.
+//     lane l's copy sits at byte e*256 + 4*l, so a warp's 32 random lookups
+//     hit 32 distinct banks, and one byte permute of the code word with 4*l
+//     is the whole address. All 256 byte values are present, so an invalid
+//     code reads its NaN entry.
+//   - Per row group the R*B partial sums are reduced across lanes with a
+//     transposing butterfly (about 2 shuffles per value instead of 5), summed
+//     over the warp's chunks in shared memory and finally over the WK warps in
+//     a fixed order: deterministic.
 #include "tq_common.cuh"
 #include "tq_linear.cuh"
 
 namespace tq {
 namespace {
 
-constexpr int kLutStride = 128;              // bytes per code-book entry
-constexpr int kLutBytes = 256 * kLutStride;  // all byte values: 32 KB
-constexpr int kMaxWarps = 8;
-constexpr int kCtasPerSm = 2;
-constexpr int kStages = 4;                   // row groups in flight per warp
+constexpr int kLutStride = 256;              // bytes per code-book entry
+constexpr int kLutBytes = 256 * kLutStride;  // all byte values: 64 KB
 
-__device__ __forceinline__ uint32_t smem_addr(const void *p) {
-  return (uint32_t)__cvta_generic_to_shared(p);
+__device__ __forceinline__ uint4 ld_stream16(const void *p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
 }
 
-// Asynchronous global -> shared copy of BYTES (16 or 8) bytes; src_size 0
-// writes zeros and reads nothing.
-template <int BYTES>
-__device__ __forceinline__ void cp_async(uint32_t dst, const void *src,
-                                         bool valid) {
-  const int n = valid ? BYTES : 0;
-  if constexpr (BYTES == 16) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst),
-                 "l"(src), "r"(n)
-                 : "memory");
-  } else {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(dst),
-                 "l"(src), "r"(n)
-                 : "memory");
-  }
-}
-
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+__device__ __forceinline__ uint2 ld_stream8(const void *p) {
+  uint2 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
+               : "=r"(v.x), "=r"(v.y)
+               : "l"(p));
+  return v;
 }
 
 // bf16 pair (low half = lower k) -> float2.
@@ -71,12 +53,12 @@ __device__ __forceinline__ float2 bf16x2_to_float2(uint32_t u) {
   return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
 }
 
-// Code-book value of byte q of word w for this lane (lane8 = 8 * lane): the
-// byte permute yields code*256 + 8*lane, halved to code*128 + 4*lane.
+// Code-book value of byte q of word w for this lane (lane4 = 4 * lane): the
+// byte permute yields code*256 + 4*lane.
 __device__ __forceinline__ float lut_at(const uint8_t *lut_smem, uint32_t w,
-                                        int q, uint32_t lane8) {
-  const uint32_t a2 = __byte_perm(w, lane8, 0x5504u | ((uint32_t)q << 4));
-  return *reinterpret_cast<const float *>(lut_smem + (a2 >> 1));
+                                        int q, uint32_t lane4) {
+  const uint32_t a = __byte_perm(w, lane4, 0x5504u | ((uint32_t)q << 4));
+  return *reinterpret_cast<const float *>(lut_smem + a);
 }
 
 // Reduce M (power of two, <= 32) per-lane values across the warp. On return
@@ -110,84 +92,90 @@ constexpr int pow2_ceil(int v) {
 }
 
 template <int B>
-struct Rows {  // rows per group
-  static constexpr int value = (B <= 2) ? 4 : 2;
+struct GemvBCfg {
+  static constexpr int R = 2;                         // rows per group
+  static constexpr int kMaxThreads = (B == 1) ? 1024 : 512;
 };
 
-template <int B, int KPL>
-struct GemvBShape {
-  static constexpr int R = Rows<B>::value;
-  static constexpr int M = pow2_ceil(R * B);  // values reduced per group
-  static constexpr int KC = 32 * KPL;         // k per warp chunk
-  static constexpr int NW = KPL / 4;          // code words per lane per row
-  static constexpr int SLOT = R * 32 * KPL;   // ring-slot bytes per warp
-  static constexpr int RING = kStages * SLOT; // ring bytes per warp
-};
 
 template <int B, int KPL>
-__global__ void __launch_bounds__(kMaxWarps * 32, kCtasPerSm)
+__global__ void __launch_bounds__(GemvBCfg<B>::kMaxThreads, 1)
     gemv_b_kernel(const uint8_t *__restrict__ codes, int64_t n, int64_t k,
                   const float *__restrict__ lut,
                   const uint16_t *__restrict__ rho, int rps,
                   const __nv_bfloat16 *__restrict__ x, int64_t ldx,
-                  float *__restrict__ y, int64_t ldy, int rows_max) {
-  using S = GemvBShape<B, KPL>;
-  constexpr int R = S::R, M = S::M, KC = S::KC, NW = S::NW;
+                  float *__restrict__ y, int64_t ldy, int wk_count,
+                  int rows_max) {
+  constexpr int R = GemvBCfg<B>::R;
+  constexpr int M = pow2_ceil(R * B);  // values reduced per row group
+  constexpr int KC = 32 * KPL;         // k per warp chunk
+  constexpr int NW = KPL / 4;          // code words per lane per row
   extern __shared__ __align__(16) uint8_t smem[];
+  float *red = reinterpret_cast<float *>(smem + kLutBytes);  // [WK][rows][B]
+
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nwarps = blockDim.x >> 5;
-  uint8_t *ring = smem + kLutBytes + warp * S::RING;
-  float *red = reinterpret_cast<float *>(smem + kLutBytes + nwarps * S::RING);
-
+  const int wk = warp % wk_count, wr = warp / wk_count;
+  const int wr_count = nwarps / wk_count;
   const int64_t row_lo = (int64_t)blockIdx.x * n / gridDim.x;
   const int rows = (int)((int64_t)(blockIdx.x + 1) * n / gridDim.x - row_lo);
-  const uint8_t *crow = codes + row_lo * k;
+  const int r_begin = rows * wr / wr_count;
+  const int my_rows = rows * (wr + 1) / wr_count - r_begin;
+  const uint8_t *crow = codes + (row_lo + r_begin) * k;
   const int64_t nchunks = (k + KC - 1) / KC;
-  const int nc_w = (int)((nchunks - warp + nwarps - 1) / nwarps);  // my chunks
-  const int ng = (rows + R - 1) / R;                               // row groups
+  const int nc_w = (int)((nchunks - wk + wk_count - 1) / wk_count);
+  const int ng = (my_rows + R - 1) / R;
   const int total = nc_w * ng;
 
-  // Issue the copies of item i (chunk i / ng, row group i % ng) into its slot.
-  auto issue = [&](int i) {
-    const int ci = i / ng, g = i % ng;
-    const int64_t kb = (warp + (int64_t)ci * nwarps) * KC + (int64_t)lane * KPL;
-    const bool lane_ok = kb < k;
-    const uint32_t dst = smem_addr(ring + (i % kStages) * S::SLOT) + lane * KPL;
+  auto kb_of = [&](int ci) -> int64_t {
+    return (wk + (int64_t)ci * wk_count) * KC + (int64_t)lane * KPL;
+  };
+  // Codes of item i (chunk i / ng, row group i % ng); 121 (weight 0) where
+  // there is nothing to load.
+  auto load_group = [&](int i, uint32_t (&cw)[R][NW]) {
+    const int ci = ng ? i / ng : 0, g = ng ? i % ng : 0;
+    const int64_t kb = kb_of(ci);
+    const bool ok_i = i < total && kb < k;
 #pragma unroll
     for (int r = 0; r < R; ++r) {
+#pragma unroll
+      for (int q = 0; q < NW; ++q) cw[r][q] = 0x79797979u;
       const int row = g * R + r;
-      const bool ok = lane_ok && row < rows;
-      cp_async<KPL>(dst + r * 32 * KPL, ok ? crow + (int64_t)row * k + kb : codes,
-                    ok);
+      if (ok_i && row < my_rows) {
+        const uint8_t *p = crow + (int64_t)row * k + kb;
+        if constexpr (KPL == 16) {
+          const uint4 v = ld_stream16(p);
+          cw[r][0] = v.x; cw[r][1] = v.y; cw[r][2] = v.z; cw[r][3] = v.w;
+        } else {
+          const uint2 v = ld_stream8(p);
+          cw[r][0] = v.x; cw[r][1] = v.y;
+        }
+      }
     }
   };
   // Raw bf16 words of x for chunk ci (this lane's KPL columns).
   uint32_t xr[B][KPL / 2];
   auto load_x = [&](int ci) {
-    const int64_t kb = (warp + (int64_t)ci * nwarps) * KC + (int64_t)lane * KPL;
+    const int64_t kb = kb_of(ci);
+    const bool ok = ci < nc_w && kb < k;
 #pragma unroll
     for (int b = 0; b < B; ++b) {
 #pragma unroll
-      for (int i = 0; i < KPL / 2; i += 4) {
+      for (int q = 0; q < KPL / 2; q += 4) {
         uint4 v = make_uint4(0, 0, 0, 0);
-        if (ci < nc_w && kb < k)
-          v = *reinterpret_cast<const uint4 *>(x + b * ldx + kb + 2 * i);
-        xr[b][i] = v.x;
-        xr[b][i + 1] = v.y;
-        xr[b][i + 2] = v.z;
-        xr[b][i + 3] = v.w;
+        if (ok) v = *reinterpret_cast<const uint4 *>(x + b * ldx + kb + 2 * q);
+        xr[b][q] = v.x;
+        xr[b][q + 1] = v.y;
+        xr[b][q + 2] = v.z;
+        xr[b][q + 3] = v.w;
       }
     }
   };
 
-  // Start the code stream and the first x before building the code book.
-#pragma unroll
-  for (int p = 0; p < kStages - 1; ++p) {
-    if (p < total) issue(p);
-    cp_async_commit();
-  }
+  // Start the first loads, then build the code book while they fly.
+  uint32_t cw[R][NW], cn[R][NW];
+  load_group(0, cw);
   load_x(0);
-
   // Replicate the code book, coalesced loads and conflict-free 16 B stores:
   // entry e's 32 lane copies are 8 float4 chunks, written in rotated order.
   for (int e = threadIdx.x; e < 256; e += blockDim.x) {
@@ -199,63 +187,50 @@ __global__ void __launch_bounds__(kMaxWarps * 32, kCtasPerSm)
       *reinterpret_cast<float4 *>(smem + e * kLutStride + jj * 16) = v4;
     }
   }
-  for (int i = threadIdx.x; i < nwarps * rows_max * B; i += blockDim.x)
+  for (int i = threadIdx.x; i < wk_count * rows_max * B; i += blockDim.x)
     red[i] = 0.0f;
   __syncthreads();
 
-  const uint32_t lane8 = (uint32_t)lane * 8u;
-  float2 xv[B][KPL / 2];
+  const uint32_t lane4 = (uint32_t)lane * 4u;
+  float xv[B][KPL];
   bool lane_ok = false;
   for (int i = 0; i < total; ++i) {
-    if (i + kStages - 1 < total) issue(i + kStages - 1);
-    cp_async_commit();
-    cp_async_wait<kStages - 1>();  // item i's copies have landed
+    load_group(i + 1, cn);  // one row group ahead
     const int ci = i / ng, g = i % ng;
     if (g == 0) {
-      const int64_t kb =
-          (warp + (int64_t)ci * nwarps) * KC + (int64_t)lane * KPL;
-      lane_ok = kb < k;
+      lane_ok = kb_of(ci) < k;
 #pragma unroll
       for (int b = 0; b < B; ++b)
 #pragma unroll
-        for (int q = 0; q < KPL / 2; ++q) xv[b][q] = bf16x2_to_float2(xr[b][q]);
+        for (int q = 0; q < KPL / 2; ++q) {
+          xv[b][2 * q] = __uint_as_float(xr[b][q] << 16);
+          xv[b][2 * q + 1] = __uint_as_float(xr[b][q] & 0xFFFF0000u);
+        }
       load_x(ci + 1);  // next chunk's x, consumed ng groups later
     }
-    float2 acc[R][B];
+    float acc[R][B];
 #pragma unroll
     for (int r = 0; r < R; ++r)
 #pragma unroll
-      for (int b = 0; b < B; ++b) acc[r][b] = make_float2(0.f, 0.f);
+      for (int b = 0; b < B; ++b) acc[r][b] = 0.0f;
     if (lane_ok) {
-      const uint8_t *slot = ring + (i % kStages) * S::SLOT + lane * KPL;
 #pragma unroll
-      for (int r = 0; r < R; ++r) {
-        uint32_t cw[NW];
-        if constexpr (KPL == 16) {
-          const uint4 v = *reinterpret_cast<const uint4 *>(slot + r * 32 * KPL);
-          cw[0] = v.x; cw[1] = v.y; cw[2] = v.z; cw[3] = v.w;
-        } else {
-          const uint2 v = *reinterpret_cast<const uint2 *>(slot + r * 32 * KPL);
-          cw[0] = v.x; cw[1] = v.y;
-        }
+      for (int r = 0; r < R; ++r)
 #pragma unroll
-        for (int wi = 0; wi < NW; ++wi) {
+        for (int q = 0; q < NW; ++q)
 #pragma unroll
-          for (int q = 0; q < 4; q += 2) {
-            const float2 wv = make_float2(lut_at(smem, cw[wi], q, lane8),
-                                          lut_at(smem, cw[wi], q + 1, lane8));
+          for (int e = 0; e < 4; ++e) {
+            const float wv = lut_at(smem, cw[r][q], e, lane4);
 #pragma unroll
             for (int b = 0; b < B; ++b)
-              acc[r][b] = __ffma2_rn(wv, xv[b][wi * 2 + q / 2], acc[r][b]);
+              acc[r][b] = fmaf(wv, xv[b][q * 4 + e], acc[r][b]);
           }
-        }
-      }
     }
     float v[M];
 #pragma unroll
     for (int r = 0; r < R; ++r)
 #pragma unroll
-      for (int b = 0; b < B; ++b) v[r * B + b] = acc[r][b].x + acc[r][b].y;
+      for (int b = 0; b < B; ++b) v[r * B + b] = acc[r][b];
 #pragma unroll
     for (int q = R * B; q < M; ++q) v[q] = 0.0f;
     const float s = butterfly_reduce<M>(v, lane);
@@ -264,15 +239,19 @@ __global__ void __launch_bounds__(kMaxWarps * 32, kCtasPerSm)
     if ((lane % kLow) == 0 && idx < R * B) {
       const int r = idx / B, b = idx % B;
       const int row = g * R + r;
-      if (row < rows) red[(warp * rows_max + row) * B + b] += s;
+      if (row < my_rows)
+        red[(wk * rows_max + r_begin + row) * B + b] += s;
     }
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int q = 0; q < NW; ++q) cw[r][q] = cn[r][q];
   }
-  cp_async_wait<0>();
   __syncthreads();
   for (int i = threadIdx.x; i < rows * B; i += blockDim.x) {
     const int r = i / B, b = i % B;
     float s = 0.0f;
-    for (int w = 0; w < nwarps; ++w) s += red[(w * rows_max + r) * B + b];
+    for (int w = 0; w < wk_count; ++w) s += red[(w * rows_max + r) * B + b];
     const int64_t row = row_lo + r;
     const float scale =
         rho ? __half2float(__ushort_as_half(rho[row / rps])) : 1.0f;
@@ -280,26 +259,30 @@ __global__ void __launch_bounds__(kMaxWarps * 32, kCtasPerSm)
   }
 }
 
-// Pick the lane width KPL (codes per lane per chunk) and the warp count so
-// that the k-chunks divide evenly among the warps of a CTA.
-struct ChunkPlan {
+// Warp layout and lane width for one shape: the k-chunks split evenly over
+// WK warps, WR row slices fill the CTA.
+struct GemvPlan {
   int kpl;
-  int warps;
+  int wk;
+  int wr;
 };
 
-ChunkPlan plan_chunks(int64_t k) {
-  ChunkPlan best{8, 1};
-  double best_eff = -1.0;
+GemvPlan plan_gemv(int64_t k, int64_t rows_per_cta, int max_warps, int R) {
+  GemvPlan best{8, 1, 1};
+  double best_score = -1.0;
   for (int kpl = 16; kpl >= 8; kpl /= 2) {
     const int64_t nchunks = (k + 32 * kpl - 1) / (32 * kpl);
-    const int wmax = (int)(nchunks < kMaxWarps ? nchunks : kMaxWarps);
-    for (int w = wmax; w >= 1 && w >= wmax - 4; --w) {
-      const int64_t rounds = (nchunks + w - 1) / w;
-      const double useful = (double)k / (32.0 * kpl);
-      const double eff = useful / (double)(rounds * w) * (w >= 4 ? 1.0 : 0.9);
-      if (eff > best_eff + 1e-9) {
-        best_eff = eff;
-        best = ChunkPlan{kpl, w};
+    const double useful = (double)k / (32.0 * kpl);
+    for (int wk = 1; wk <= max_warps && wk <= nchunks; ++wk) {
+      const int64_t rounds = (nchunks + wk - 1) / wk;
+      const double eff = useful / (double)(rounds * wk);
+      int wr = max_warps / wk;
+      const int64_t wr_rows = (rows_per_cta + R - 1) / R;  // >= R rows each
+      if (wr > wr_rows) wr = (int)(wr_rows > 0 ? wr_rows : 1);
+      const double score = eff * (double)(wk * wr) / max_warps;
+      if (score > best_score + 1e-9) {
+        best_score = score;
+        best = GemvPlan{kpl, wk, wr};
       }
     }
   }
@@ -308,35 +291,38 @@ ChunkPlan plan_chunks(int64_t k) {
 
 template <int B, int KPL>
 cudaError_t launch_kpl(const WeightsView &w, const __nv_bfloat16 *x,
-                       int64_t ldx, float *y, int64_t ldy, int warps,
-                       cudaStream_t stream) {
-  using S = GemvBShape<B, KPL>;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  constexpr int kMaxRedBytes = 16 * 1024;
-  const int64_t rows_cap = kMaxRedBytes / (warps * B * 4);
-  int64_t ctas = (int64_t)sms * kCtasPerSm;
-  if ((w.n + ctas - 1) / ctas > rows_cap) ctas = (w.n + rows_cap - 1) / rows_cap;
-  if (ctas > w.n) ctas = w.n;
+                       int64_t ldx, float *y, int64_t ldy, int64_t ctas,
+                       const GemvPlan &p, cudaStream_t stream) {
   const int rows_max = (int)((w.n + ctas - 1) / ctas);
-  const size_t smem = kLutBytes + (size_t)warps * S::RING +
-                      (size_t)warps * rows_max * B * sizeof(float);
+  const size_t smem =
+      kLutBytes + (size_t)p.wk * rows_max * B * sizeof(float);
   auto kern = gemv_b_kernel<B, KPL>;
   cudaError_t e = cudaFuncSetAttribute(
       kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<(unsigned)ctas, warps * 32, smem, stream>>>(
-      w.codes, w.n, w.k, w.lut, w.scales, w.rps, x, ldx, y, ldy, rows_max);
+  kern<<<(unsigned)ctas, p.wk * p.wr * 32, smem, stream>>>(
+      w.codes, w.n, w.k, w.lut, w.scales, w.rps, x, ldx, y, ldy, p.wk,
+      rows_max);
   return cudaGetLastError();
 }
 
 template <int B>
 cudaError_t launch_b(const WeightsView &w, const __nv_bfloat16 *x, int64_t ldx,
                      float *y, int64_t ldy, cudaStream_t stream) {
-  const ChunkPlan p = plan_chunks(w.k);
-  if (p.kpl == 16) return launch_kpl<B, 16>(w, x, ldx, y, ldy, p.warps, stream);
-  return launch_kpl<B, 8>(w, x, ldx, y, ldy, p.warps, stream);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  constexpr int kMaxWarps = GemvBCfg<B>::kMaxThreads / 32;
+  int64_t ctas = sms;
+  // keep the partial-sum buffer small (<= 96 KB): more CTAs for tall shapes
+  const int64_t rows_cap = (96 * 1024) / (kMaxWarps * B * 4);
+  if ((w.n + ctas - 1) / ctas > rows_cap) ctas = (w.n + rows_cap - 1) / rows_cap;
+  if (ctas > w.n) ctas = w.n;
+  const GemvPlan p =
+      plan_gemv(w.k, (w.n + ctas - 1) / ctas, kMaxWarps, GemvBCfg<B>::R);
+  if (p.kpl == 16)
+    return launch_kpl<B, 16>(w, x, ldx, y, ldy, ctas, p, stream);
+  return launch_kpl<B, 8>(w, x, ldx, y, ldy, ctas, p, stream);
 }
 
 }  // namespace
