@@ -130,12 +130,12 @@ __global__ void __launch_bounds__(GemvBCfg<B>::kMaxThreads, 1)
   auto kb_of = [&](int ci) -> int64_t {
     return (wk + (int64_t)ci * wk_count) * KC + (int64_t)lane * KPL;
   };
-  // Codes of item i (chunk i / ng, row group i % ng); 121 (weight 0) where
-  // there is nothing to load.
-  auto load_group = [&](int i, uint32_t (&cw)[R][NW]) {
-    const int ci = ng ? i / ng : 0, g = ng ? i % ng : 0;
+  // Codes of chunk ci, row group g; 121 (weight 0) where there is nothing to
+  // load. (No integer division in the loop: divisions run on the slow
+  // conversion pipe.)
+  auto load_group = [&](int ci, int g, uint32_t (&cw)[R][NW]) {
     const int64_t kb = kb_of(ci);
-    const bool ok_i = i < total && kb < k;
+    const bool ok_i = ci < nc_w && kb < k;
 #pragma unroll
     for (int r = 0; r < R; ++r) {
 #pragma unroll
@@ -174,7 +174,7 @@ __global__ void __launch_bounds__(GemvBCfg<B>::kMaxThreads, 1)
 
   // Start the first loads, then build the code book while they fly.
   uint32_t cw[R][NW], cn[R][NW];
-  load_group(0, cw);
+  load_group(0, 0, cw);
   load_x(0);
   // Replicate the code book, coalesced loads and conflict-free 16 B stores:
   // entry e's 32 lane copies are 8 float4 chunks, written in rotated order.
@@ -194,9 +194,10 @@ __global__ void __launch_bounds__(GemvBCfg<B>::kMaxThreads, 1)
   const uint32_t lane4 = (uint32_t)lane * 4u;
   float xv[B][KPL];
   bool lane_ok = false;
+  int ci = 0, g = 0;  // current chunk and row group
   for (int i = 0; i < total; ++i) {
-    load_group(i + 1, cn);  // one row group ahead
-    const int ci = i / ng, g = i % ng;
+    const bool wrap = g + 1 == ng;
+    load_group(wrap ? ci + 1 : ci, wrap ? 0 : g + 1, cn);  // one group ahead
     if (g == 0) {
       lane_ok = kb_of(ci) < k;
 #pragma unroll
@@ -246,6 +247,12 @@ __global__ void __launch_bounds__(GemvBCfg<B>::kMaxThreads, 1)
     for (int r = 0; r < R; ++r)
 #pragma unroll
       for (int q = 0; q < NW; ++q) cw[r][q] = cn[r][q];
+    if (wrap) {
+      ++ci;
+      g = 0;
+    } else {
+      ++g;
+    }
   }
   __syncthreads();
   for (int i = threadIdx.x; i < rows * B; i += blockDim.x) {
