@@ -53,12 +53,14 @@ __device__ __forceinline__ float2 bf16x2_to_float2(uint32_t u) {
   return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
 }
 
-// Code-book value of byte q of word w for this lane (lane4 = 4 * lane): the
-// byte permute yields code*256 + 4*lane.
-__device__ __forceinline__ float lut_at(const uint8_t *lut_smem, uint32_t w,
-                                        int q, uint32_t lane4) {
+// Code-book value of byte q of word w for this lane: the byte permute
+// yields code*256 + 4*lane, added to the table's 32-bit shared address.
+__device__ __forceinline__ float lut_at(uint32_t lut_base, uint32_t w, int q,
+                                        uint32_t lane4) {
   const uint32_t a = __byte_perm(w, lane4, 0x5504u | ((uint32_t)q << 4));
-  return *reinterpret_cast<const float *>(lut_smem + a);
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(lut_base + a));
+  return v;
 }
 
 // Reduce M (power of two, <= 32) per-lane values across the warp. On return
@@ -94,7 +96,7 @@ constexpr int pow2_ceil(int v) {
 template <int B>
 struct GemvBCfg {
   static constexpr int R = 2;                         // rows per group
-  static constexpr int kMaxThreads = (B == 1) ? 1024 : 512;
+  static constexpr int kMaxThreads = (B == 1) ? 768 : 512;
 };
 
 
@@ -122,6 +124,7 @@ __global__ void __launch_bounds__(GemvBCfg<B>::kMaxThreads, 1)
   const int r_begin = rows * wr / wr_count;
   const int my_rows = rows * (wr + 1) / wr_count - r_begin;
   const uint8_t *crow = codes + (row_lo + r_begin) * k;
+  const uint32_t kstride = (uint32_t)k;  // row pitch (k < 2^32)
   const int64_t nchunks = (k + KC - 1) / KC;
   const int nc_w = (int)((nchunks - wk + wk_count - 1) / wk_count);
   const int ng = (my_rows + R - 1) / R;
@@ -142,7 +145,7 @@ __global__ void __launch_bounds__(GemvBCfg<B>::kMaxThreads, 1)
       for (int q = 0; q < NW; ++q) cw[r][q] = 0x79797979u;
       const int row = g * R + r;
       if (ok_i && row < my_rows) {
-        const uint8_t *p = crow + (int64_t)row * k + kb;
+        const uint8_t *p = crow + (int64_t)row * kstride + kb;
         if constexpr (KPL == 16) {
           const uint4 v = ld_stream16(p);
           cw[r][0] = v.x; cw[r][1] = v.y; cw[r][2] = v.z; cw[r][3] = v.w;
@@ -192,6 +195,7 @@ __global__ void __launch_bounds__(GemvBCfg<B>::kMaxThreads, 1)
   __syncthreads();
 
   const uint32_t lane4 = (uint32_t)lane * 4u;
+  const uint32_t lut_base = (uint32_t)__cvta_generic_to_shared(smem);
   float xv[B][KPL];
   bool lane_ok = false;
   int ci = 0, g = 0;  // current chunk and row group
@@ -221,7 +225,7 @@ __global__ void __launch_bounds__(GemvBCfg<B>::kMaxThreads, 1)
         for (int q = 0; q < NW; ++q)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float wv = lut_at(smem, cw[r][q], e, lane4);
+            const float wv = lut_at(lut_base, cw[r][q], e, lane4);
 #pragma unroll
             for (int b = 0; b < B; ++b)
               acc[r][b] = fmaf(wv, xv[b][q * 4 + e], acc[r][b]);
@@ -274,10 +278,11 @@ struct GemvPlan {
   int wr;
 };
 
-GemvPlan plan_gemv(int64_t k, int64_t rows_per_cta, int max_warps, int R) {
+GemvPlan plan_gemv(int64_t k, int64_t rows_per_cta, int max_warps, int R,
+                   int kpl_max) {
   GemvPlan best{8, 1, 1};
   double best_score = -1.0;
-  for (int kpl = 16; kpl >= 8; kpl /= 2) {
+  for (int kpl = kpl_max; kpl >= 8; kpl /= 2) {
     const int64_t nchunks = (k + 32 * kpl - 1) / (32 * kpl);
     const double useful = (double)k / (32.0 * kpl);
     for (int wk = 1; wk <= max_warps && wk <= nchunks; ++wk) {
@@ -325,10 +330,13 @@ cudaError_t launch_b(const WeightsView &w, const __nv_bfloat16 *x, int64_t ldx,
   const int64_t rows_cap = (96 * 1024) / (kMaxWarps * B * 4);
   if ((w.n + ctas - 1) / ctas > rows_cap) ctas = (w.n + rows_cap - 1) / rows_cap;
   if (ctas > w.n) ctas = w.n;
-  const GemvPlan p =
-      plan_gemv(w.k, (w.n + ctas - 1) / ctas, kMaxWarps, GemvBCfg<B>::R);
-  if (p.kpl == 16)
-    return launch_kpl<B, 16>(w, x, ldx, y, ldy, ctas, p, stream);
+  constexpr int kKplMax = (B <= 2) ? 16 : 8;  // register budget
+  const GemvPlan p = plan_gemv(w.k, (w.n + ctas - 1) / ctas, kMaxWarps,
+                               GemvBCfg<B>::R, kKplMax);
+  if constexpr (kKplMax == 16) {
+    if (p.kpl == 16)
+      return launch_kpl<B, 16>(w, x, ldx, y, ldy, ctas, p, stream);
+  }
   return launch_kpl<B, 8>(w, x, ldx, y, ldy, ctas, p, stream);
 }
 
