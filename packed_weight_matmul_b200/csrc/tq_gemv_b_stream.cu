@@ -1,0 +1,350 @@
+// Format B fused GEMV at batch 1 and 2, streamed by the TMA engine
+// (alphaneural.io page, sections 3.2, 3.3 and 4.2):
+//   y[b][n] = rho[n / rps] * sum_k LUT[code[n][k]] * x[b][k].
+//
+// The matrix is read once at HBM speed only if enough bytes are in flight
+// per SM; register prefetch by warps cannot hold enough of them. So:
+//   - One CTA per SM owns rows [i*n/P, (i+1)*n/P): one contiguous span of
+//     codes. Warp 0 (one elected lane) streams that span through a ring of S
+//     shared-memory stages with 1-D bulk copies, one row segment of C bytes
+//     (C <= 16 KB, a multiple of 512 unless it is a whole row) per stage, each
+//     completing on its stage's mbarrier as transaction bytes.
+//   - The other warps consume segments round-robin: each lane takes 16 codes
+//     per 512-byte step, looks them up in a per-lane copy of the code book
+//     (entry e of lane l at byte e*256 + 4*l: conflict-free; the byte permute
+//     of the code word is the whole address when the table sits at a 64 KB
+//     aligned shared address, else one add), multiplies by x held in shared
+//     memory as fp32 (permuted so a warp's 16-byte reads are conflict-free),
+//     reduces the segment across the warp, stores one partial per segment and
+//     releases the stage.
+//   - At the end the segments of each row are summed in order (deterministic)
+//     and rho is applied to the sum.
+//   - Every wait is bounded; on a time-out the CTA writes NaN to its outputs,
+//     waits (bounded) for its copies in flight and exits.
+#include "tq_common.cuh"
+#include "tq_linear.cuh"
+#include "tq_sm100_async.cuh"
+
+namespace tq {
+namespace {
+
+constexpr int kLutBytes = 256 * 256;   // 256 entries x 32 lane copies x 4 B
+constexpr int kReservedSmem = 1024;    // system shared memory below the CTA's
+constexpr int kConsumerWarps = 15;
+constexpr int kThreads = 32 * (1 + kConsumerWarps);
+constexpr int kMaxStages = 16;
+constexpr int kStepBytes = 512;        // codes per warp step (16 per lane)
+
+__device__ __forceinline__ float lds_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ uint4 lds_u32x4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ float4 lds_f32x4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr));
+  return v;
+}
+
+struct StreamParams {
+  int seg_bytes;   // C
+  int nseg;        // segments per row
+  int stage_pitch; // bytes between ring stages
+  int stages;      // S
+  int x_off, part_off, bar_off, lut_off, ring_off;
+  int paged;       // table placed at a 64 KB aligned shared address
+  int rows_max;
+  size_t smem;
+};
+
+// One segment: sum over its codes of LUT[code] * x, for this lane.
+template <int B, bool PAGED>
+__device__ __forceinline__ void segment_dot(uint32_t buf, int seg_bytes,
+                                            int T0, int lane, uint32_t xs,
+                                            uint32_t perm_op, uint32_t fix,
+                                            float (&acc)[B]) {
+#pragma unroll 2
+  for (int t = 0; t * kStepBytes < seg_bytes; ++t) {
+    const int off = t * kStepBytes + lane * 16;
+    if (off < seg_bytes) {
+      const uint4 cv = lds_u32x4(buf + off);
+      const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w};
+      const uint32_t xa = xs + (uint32_t)(((T0 + t) * 4 * 32 + lane) * B * 16);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float xv[B][4];
+#pragma unroll
+        for (int b = 0; b < B; ++b) {
+          const float4 f = lds_f32x4(xa + (q * 32 * B + b) * 16);
+          xv[b][0] = f.x; xv[b][1] = f.y; xv[b][2] = f.z; xv[b][3] = f.w;
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t a =
+              __byte_perm(cw[q], perm_op, 0x7604u | ((uint32_t)e << 4));
+          const float wv = lds_f32(PAGED ? a : a + fix);
+#pragma unroll
+          for (int b = 0; b < B; ++b) acc[b] = fmaf(wv, xv[b][e], acc[b]);
+        }
+      }
+    }
+  }
+}
+
+template <int B>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemv_b_stream_kernel(const uint8_t *__restrict__ codes, int64_t n,
+                         int64_t k, const float *__restrict__ lut,
+                         const uint16_t *__restrict__ rho, int rps,
+                         const __nv_bfloat16 *__restrict__ x, int64_t ldx,
+                         float *__restrict__ y, int64_t ldy, StreamParams P) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const uint32_t sbase = smem_u32(smem);
+  // set by any thread whose bounded wait timed out
+  volatile int &abort_flag =
+      *reinterpret_cast<int *>(smem + P.bar_off + 16 * kMaxStages);
+  const uint32_t xs = sbase + P.x_off;
+  const uint32_t ring = sbase + P.ring_off;
+  const uint32_t lut_addr = sbase + P.lut_off;
+  const uint32_t full0 = sbase + P.bar_off;                // full[s]
+  const uint32_t empty0 = full0 + 8 * P.stages;            // empty[s]
+  float *part = reinterpret_cast<float *>(smem + P.part_off);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t row_lo = (int64_t)blockIdx.x * n / gridDim.x;
+  const int rows = (int)((int64_t)(blockIdx.x + 1) * n / gridDim.x - row_lo);
+  const int nchunks = rows * P.nseg;
+  const int C = P.seg_bytes;
+  const uint8_t *span = codes + row_lo * k;
+
+  auto src_of = [&](int j) -> const uint8_t * {
+    const int r = j / P.nseg, s = j - r * P.nseg;
+    return span + (int64_t)r * k + (int64_t)s * C;
+  };
+
+  // Barriers, then the first S copies right away (before any staging).
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    for (int s = 0; s < P.stages; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    mbar_init_fence();
+    for (int j = 0; j < P.stages && j < nchunks; ++j) {
+      mbar_arrive_expect_tx(full0 + 8 * j, (uint32_t)C);
+      bulk_g2s(ring + j * P.stage_pitch, src_of(j), (uint32_t)C, full0 + 8 * j);
+    }
+  }
+
+  // Stage x as fp32: element k = 512*T + 16*l + 4*q + i of batch b goes to
+  // float index (((T*4 + q)*32 + l)*B + b)*4 + i. 8 elements per load.
+  float *xsp = reinterpret_cast<float *>(smem + P.x_off);
+  const int kpad = (int)((k + kStepBytes - 1) / kStepBytes) * kStepBytes;
+  for (int v = threadIdx.x; v < kpad / 8; v += blockDim.x) {
+    const int kk = v * 8;
+    const int T = kk >> 9, l = (kk >> 4) & 31, q0 = (kk >> 2) & 3;
+#pragma unroll
+    for (int b = 0; b < B; ++b) {
+      uint4 raw = make_uint4(0, 0, 0, 0);
+      if (kk < k) raw = *reinterpret_cast<const uint4 *>(x + b * ldx + kk);
+      const uint32_t wd[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float4 f;
+        f.x = __uint_as_float(wd[2 * h] << 16);
+        f.y = __uint_as_float(wd[2 * h] & 0xFFFF0000u);
+        f.z = __uint_as_float(wd[2 * h + 1] << 16);
+        f.w = __uint_as_float(wd[2 * h + 1] & 0xFFFF0000u);
+        const int idx = ((((T * 4 + q0 + h) * 32 + l) * B) + b) * 4;
+        *reinterpret_cast<float4 *>(xsp + idx) = f;
+      }
+    }
+  }
+  // Code book, one copy per lane, conflict-free rotated 16-byte stores.
+  for (int e = threadIdx.x; e < 256; e += blockDim.x) {
+    const float v = __ldg(lut + e);
+    const float4 v4 = make_float4(v, v, v, v);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int jj = (j + e) & 7;
+      *reinterpret_cast<float4 *>(smem + P.lut_off + e * 256 + jj * 16) = v4;
+    }
+  }
+  __syncthreads();
+
+  if (warp == 0) {
+    // Producer: refill each stage once its consumer has released it.
+    if (lane == 0) {
+      for (int j = P.stages; j < nchunks && !abort_flag; ++j) {
+        const int s = j % P.stages;
+        if (!mbar_wait(empty0 + 8 * s, ((j / P.stages) - 1) & 1)) {
+          abort_flag = 1;
+          break;
+        }
+        mbar_arrive_expect_tx(full0 + 8 * s, (uint32_t)C);
+        bulk_g2s(ring + s * P.stage_pitch, src_of(j), (uint32_t)C,
+                 full0 + 8 * s);
+      }
+    }
+  } else {
+    const bool paged = P.paged && (lut_addr & 0xFFFFu) == 0;
+    const uint32_t perm_op =
+        (paged ? (lut_addr & 0xFFFF0000u) : 0u) | ((uint32_t)lane * 4u);
+    for (int j = warp - 1; j < nchunks; j += kConsumerWarps) {
+      const int s = j % P.stages;
+      if (!mbar_wait(full0 + 8 * s, (j / P.stages) & 1)) {
+        abort_flag = 1;
+        break;
+      }
+      const int seg = j % P.nseg;
+      const int T0 = seg * C / kStepBytes;  // C is a multiple of 512 if nseg > 1
+      float acc[B];
+#pragma unroll
+      for (int b = 0; b < B; ++b) acc[b] = 0.0f;
+      const uint32_t buf = ring + s * P.stage_pitch;
+      if (paged)
+        segment_dot<B, true>(buf, C, T0, lane, xs, perm_op, 0u, acc);
+      else
+        segment_dot<B, false>(buf, C, T0, lane, xs, perm_op, lut_addr, acc);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty0 + 8 * s);  // stage reads are done
+#pragma unroll
+      for (int b = 0; b < B; ++b) {
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1)
+          acc[b] += __shfl_xor_sync(0xFFFFFFFFu, acc[b], o);
+        if (lane == 0) part[j * B + b] = acc[b];
+      }
+      if (abort_flag) break;
+    }
+  }
+  __syncthreads();
+
+  if (abort_flag) {
+    // Give the copies still in flight (at most S) a bounded chance to land
+    // before the CTA's shared memory is released; outputs are poisoned.
+    if (threadIdx.x == 0) {
+      const int last = nchunks < P.stages ? nchunks : P.stages;
+      for (int j = nchunks - last; j < nchunks; ++j)
+        (void)mbar_wait(full0 + 8 * (j % P.stages), (j / P.stages) & 1);
+    }
+    for (int i = threadIdx.x; i < rows * B; i += blockDim.x)
+      y[(int64_t)(i % B) * ldy + row_lo + i / B] = __int_as_float(0x7FC00000);
+    return;
+  }
+  for (int i = threadIdx.x; i < rows * B; i += blockDim.x) {
+    const int r = i / B, b = i % B;
+    float sum = 0.0f;
+    for (int s = 0; s < P.nseg; ++s) sum += part[(r * P.nseg + s) * B + b];
+    const int64_t grow = row_lo + r;
+    const float scale =
+        rho ? __half2float(__ushort_as_half(rho[grow / rps])) : 1.0f;
+    y[(int64_t)b * ldy + grow] = scale * sum;
+  }
+}
+
+// Lay out shared memory for one shape; stages == 0 when it does not fit.
+StreamParams plan_stream(int64_t n, int64_t k, int B, int64_t ctas,
+                         int max_smem) {
+  StreamParams P{};
+  P.rows_max = (int)((n + ctas - 1) / ctas);
+  int nseg = 0;
+  for (int s = 1; s <= 64; ++s) {
+    if (k % s) continue;
+    const int64_t C = k / s;
+    if (C > 16384) continue;
+    if (s > 1 && C % kStepBytes) continue;
+    nseg = s;
+    break;
+  }
+  if (nseg == 0) return P;
+  P.nseg = nseg;
+  P.seg_bytes = (int)(k / nseg);
+  P.stage_pitch = (P.seg_bytes + 127) / 128 * 128;
+  const int64_t kpad = (k + kStepBytes - 1) / kStepBytes * kStepBytes;
+  const int64_t x_bytes = kpad * B * 4;
+  const int64_t part_bytes = (int64_t)P.rows_max * nseg * B * 4;
+  P.x_off = 0;
+  P.part_off = (int)x_bytes;
+  P.bar_off = (int)((x_bytes + part_bytes + 15) / 16 * 16);
+  const int64_t front = (P.bar_off + 16 * kMaxStages + 16 + 255) / 256 * 256;
+  // (a) code book at a 64 KB aligned shared address, ring after it
+  int64_t lut_a = 65536 - kReservedSmem;
+  while (lut_a < front) lut_a += 65536;
+  const int64_t stages_a = (max_smem - (lut_a + kLutBytes)) / P.stage_pitch;
+  // (b) code book right after the front, ring after it
+  const int64_t lut_b = front;
+  const int64_t stages_b = (max_smem - (lut_b + kLutBytes)) / P.stage_pitch;
+  const bool use_a = stages_a >= 4 && stages_a + 2 >= stages_b;
+  const int64_t lut = use_a ? lut_a : lut_b;
+  int64_t stages = use_a ? stages_a : stages_b;
+  if (stages > kMaxStages) stages = kMaxStages;
+  if (stages < 2) return P;
+  P.paged = use_a ? 1 : 0;
+  P.lut_off = (int)lut;
+  P.ring_off = (int)(lut + kLutBytes);
+  P.stages = (int)stages;
+  P.smem = (size_t)P.ring_off + (size_t)P.stages * P.stage_pitch;
+  return P;
+}
+
+struct Device {
+  int sms;
+  int max_smem;
+};
+
+Device device_props() {
+  Device d{148, 227 * 1024};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaDeviceGetAttribute(&d.max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin,
+                         dev);
+  return d;
+}
+
+template <int B>
+cudaError_t launch_stream(const WeightsView &w, const __nv_bfloat16 *x,
+                          int64_t ldx, float *y, int64_t ldy,
+                          cudaStream_t stream) {
+  const Device d = device_props();
+  const int64_t ctas = d.sms < w.n ? d.sms : w.n;
+  const StreamParams P = plan_stream(w.n, w.k, B, ctas, d.max_smem);
+  auto kern = gemv_b_stream_kernel<B>;
+  cudaError_t e = cudaFuncSetAttribute(
+      kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P.smem);
+  if (e != cudaSuccess) return e;
+  kern<<<(unsigned)ctas, kThreads, P.smem, stream>>>(
+      w.codes, w.n, w.k, w.lut, w.scales, w.rps, x, ldx, y, ldy, P);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool gemv_b_stream_supported(const WeightsView &w, int64_t batch) {
+  if (w.format != TQ_FMT_B || batch < 1 || batch > 2) return false;
+  if (w.k >= ((int64_t)1 << 24)) return false;
+  const Device d = device_props();
+  const int64_t ctas = d.sms < w.n ? d.sms : w.n;
+  return plan_stream(w.n, w.k, (int)batch, ctas, d.max_smem).stages >= 2;
+}
+
+cudaError_t gemv_b_stream(const WeightsView &w, const __nv_bfloat16 *x,
+                          int64_t batch, int64_t ldx, float *y, int64_t ldy,
+                          cudaStream_t stream) {
+  if (batch == 1) return launch_stream<1>(w, x, ldx, y, ldy, stream);
+  return launch_stream<2>(w, x, ldx, y, ldy, stream);
+}
+
+}  // namespace tq
