@@ -2,23 +2,25 @@
 // (alphaneural.io page, sections 3.2, 3.3 and 4.2):
 //   y[b][n] = rho[n / rps] * sum_k LUT[code[n][k]] * x[b][k].
 //
-// The matrix is read once at HBM speed only if enough bytes are in flight
-// per SM; register prefetch by warps cannot hold enough of them. So:
-//   - One CTA per SM owns rows [i*n/P, (i+1)*n/P): one contiguous span of
-//     codes. Warp 0 (one elected lane) streams that span through a ring of S
-//     shared-memory stages with 1-D bulk copies, one row segment of C bytes
-//     (C <= 16 KB, a multiple of 512 unless it is a whole row) per stage, each
-//     completing on its stage's mbarrier as transaction bytes.
-//   - The other warps consume segments round-robin: each lane takes 16 codes
-//     per 512-byte step, looks them up in a per-lane copy of the code book
-//     (entry e of lane l at byte e*256 + 4*l: conflict-free; the byte permute
-//     of the code word is the whole address when the table sits at a 64 KB
-//     aligned shared address, else one add), multiplies by x held in shared
-//     memory as fp32 (permuted so a warp's 16-byte reads are conflict-free),
-//     reduces the segment across the warp, stores one partial per segment and
-//     releases the stage.
-//   - At the end the segments of each row are summed in order (deterministic)
-//     and rho is applied to the sum.
+// Two limits decide this kernel: bytes in flight per SM (warps prefetching
+// into registers cannot hold enough) and shared-memory bandwidth (128 B per
+// clock per SM, which the per-lane code-book lookups already half use).
+//   - One CTA per SM owns rows [i*n/P, (i+1)*n/P). Warp 0 (one elected lane)
+//     streams them through a ring of S shared-memory stages with 1-D bulk
+//     copies: a stage holds a quad of 4 rows x one segment of C bytes (4
+//     copies completing on the stage's mbarrier as transaction bytes).
+//   - W consumer warps, W dividing S: stage s is always consumed by warp
+//     s mod W, so each mbarrier's phases are awaited in order by one warp.
+//   - A consumer warp's lanes are 4 rows x 8 k-parts: per 128-byte step a
+//     lane takes 16 codes of its row, looks them up in its own copy of the
+//     code book (entry e of lane l at byte e*256 + 4*l: conflict-free; the
+//     byte permute of the code word is the whole address when the table sits
+//     at a 64 KB aligned shared address, else one add) and multiplies by x
+//     held in shared memory as fp32. The 4 rows of a k-part read the same x
+//     bytes (broadcast), so x costs a quarter of the lookups' bandwidth.
+//   - Per stage the 8 k-parts of each row are reduced with 3 shuffles and one
+//     partial per (row, segment) is stored; the segments of a row are summed
+//     in order at the end (deterministic) and rho is applied to the sum.
 //   - Every wait is bounded; on a time-out the CTA writes NaN to its outputs,
 //     waits (bounded) for its copies in flight and exits.
 #include "tq_common.cuh"
@@ -30,10 +32,11 @@ namespace {
 
 constexpr int kLutBytes = 256 * 256;   // 256 entries x 32 lane copies x 4 B
 constexpr int kReservedSmem = 1024;    // system shared memory below the CTA's
-constexpr int kConsumerWarps = 15;
-constexpr int kThreads = 32 * (1 + kConsumerWarps);
+constexpr int kMaxConsumers = 15;
 constexpr int kMaxStages = 16;
-constexpr int kStepBytes = 512;        // codes per warp step (16 per lane)
+constexpr int kRows = 4;               // rows per stage
+constexpr int kParts = 8;              // k-parts (lanes) per row
+constexpr int kStep = 16 * kParts;     // codes per row per warp step (128)
 
 __device__ __forceinline__ float lds_f32(uint32_t addr) {
   float v;
@@ -58,35 +61,38 @@ __device__ __forceinline__ float4 lds_f32x4(uint32_t addr) {
 }
 
 struct StreamParams {
-  int seg_bytes;   // C
-  int nseg;        // segments per row
-  int stage_pitch; // bytes between ring stages
-  int stages;      // S
+  int seg_bytes;    // C: codes per row per stage
+  int nseg;         // segments per row
+  int row_pitch;    // bytes between the 4 rows of a stage
+  int stage_pitch;  // bytes between ring stages
+  int stages;       // S
+  int consumers;    // W, divides S
   int x_off, part_off, bar_off, lut_off, ring_off;
-  int paged;       // table placed at a 64 KB aligned shared address
+  int paged;        // table placed at a 64 KB aligned shared address
   int rows_max;
   size_t smem;
 };
 
-// One segment: sum over its codes of LUT[code] * x, for this lane.
+// Dot of one row segment (this lane's k-part) with x.
 template <int B, bool PAGED>
-__device__ __forceinline__ void segment_dot(uint32_t buf, int seg_bytes,
-                                            int T0, int lane, uint32_t xs,
+__device__ __forceinline__ void segment_dot(uint32_t rowbuf, int seg_bytes,
+                                            int T0, int p, uint32_t xs,
                                             uint32_t perm_op, uint32_t fix,
                                             float (&acc)[B]) {
 #pragma unroll 2
-  for (int t = 0; t * kStepBytes < seg_bytes; ++t) {
-    const int off = t * kStepBytes + lane * 16;
+  for (int t = 0; t * kStep < seg_bytes; ++t) {
+    const int off = t * kStep + p * 16;
     if (off < seg_bytes) {
-      const uint4 cv = lds_u32x4(buf + off);
+      const uint4 cv = lds_u32x4(rowbuf + off);
       const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w};
-      const uint32_t xa = xs + (uint32_t)(((T0 + t) * 4 * 32 + lane) * B * 16);
+      // x chunk (T, q, part p) at byte ((T*4 + q)*8 + p)*16*B + b*16
+      const uint32_t xa = xs + (uint32_t)(((T0 + t) * 4 * kParts + p) * B * 16);
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         float xv[B][4];
 #pragma unroll
         for (int b = 0; b < B; ++b) {
-          const float4 f = lds_f32x4(xa + (q * 32 * B + b) * 16);
+          const float4 f = lds_f32x4(xa + (q * kParts * B + b) * 16);
           xv[b][0] = f.x; xv[b][1] = f.y; xv[b][2] = f.z; xv[b][3] = f.w;
         }
 #pragma unroll
@@ -103,7 +109,7 @@ __device__ __forceinline__ void segment_dot(uint32_t buf, int seg_bytes,
 }
 
 template <int B>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(32 * (1 + kMaxConsumers), 1)
     gemv_b_stream_kernel(const uint8_t *__restrict__ codes, int64_t n,
                          int64_t k, const float *__restrict__ lut,
                          const uint16_t *__restrict__ rho, int rps,
@@ -111,29 +117,38 @@ __global__ void __launch_bounds__(kThreads, 1)
                          float *__restrict__ y, int64_t ldy, StreamParams P) {
   extern __shared__ __align__(128) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
-  // set by any thread whose bounded wait timed out
-  volatile int &abort_flag =
-      *reinterpret_cast<int *>(smem + P.bar_off + 16 * kMaxStages);
   const uint32_t xs = sbase + P.x_off;
   const uint32_t ring = sbase + P.ring_off;
   const uint32_t lut_addr = sbase + P.lut_off;
-  const uint32_t full0 = sbase + P.bar_off;                // full[s]
-  const uint32_t empty0 = full0 + 8 * P.stages;            // empty[s]
+  const uint32_t full0 = sbase + P.bar_off;      // full[s]
+  const uint32_t empty0 = full0 + 8 * P.stages;  // empty[s]
   float *part = reinterpret_cast<float *>(smem + P.part_off);
+  // set by any thread whose bounded wait timed out
+  volatile int &abort_flag =
+      *reinterpret_cast<int *>(smem + P.bar_off + 16 * kMaxStages);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t row_lo = (int64_t)blockIdx.x * n / gridDim.x;
   const int rows = (int)((int64_t)(blockIdx.x + 1) * n / gridDim.x - row_lo);
-  const int nchunks = rows * P.nseg;
+  const int quads = (rows + kRows - 1) / kRows;
+  const int nchunks = quads * P.nseg;
   const int C = P.seg_bytes;
   const uint8_t *span = codes + row_lo * k;
 
-  auto src_of = [&](int j) -> const uint8_t * {
-    const int r = j / P.nseg, s = j - r * P.nseg;
-    return span + (int64_t)r * k + (int64_t)s * C;
+  // Issue stage j (row quad j / nseg, segment j % nseg) into ring slot s.
+  auto issue = [&](int j, int s) {
+    const int q = j / P.nseg, seg = j - q * P.nseg;
+    const int r0 = q * kRows;
+    const int nr = rows - r0 < kRows ? rows - r0 : kRows;
+    const uint32_t bar = full0 + 8 * s;
+    mbar_arrive_expect_tx(bar, (uint32_t)(nr * C));
+    for (int r = 0; r < nr; ++r)
+      bulk_g2s(ring + s * P.stage_pitch + r * P.row_pitch,
+               span + (int64_t)(r0 + r) * k + (int64_t)seg * C, (uint32_t)C,
+               bar);
   };
 
-  // Barriers, then the first S copies right away (before any staging).
+  // Barriers, then the first S stages right away (before any staging).
   if (threadIdx.x == 0) {
     abort_flag = 0;
     for (int s = 0; s < P.stages; ++s) {
@@ -141,19 +156,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(empty0 + 8 * s, 1);
     }
     mbar_init_fence();
-    for (int j = 0; j < P.stages && j < nchunks; ++j) {
-      mbar_arrive_expect_tx(full0 + 8 * j, (uint32_t)C);
-      bulk_g2s(ring + j * P.stage_pitch, src_of(j), (uint32_t)C, full0 + 8 * j);
-    }
+    for (int j = 0; j < P.stages && j < nchunks; ++j) issue(j, j);
   }
 
-  // Stage x as fp32: element k = 512*T + 16*l + 4*q + i of batch b goes to
-  // float index (((T*4 + q)*32 + l)*B + b)*4 + i. 8 elements per load.
+  // Stage x as fp32: element k = 128*T + 16*p + 4*q + i of batch b goes to
+  // float index (((T*4 + q)*8 + p)*B + b)*4 + i. 8 elements per load.
   float *xsp = reinterpret_cast<float *>(smem + P.x_off);
-  const int kpad = (int)((k + kStepBytes - 1) / kStepBytes) * kStepBytes;
+  const int kpad = (int)((k + kStep - 1) / kStep) * kStep;
   for (int v = threadIdx.x; v < kpad / 8; v += blockDim.x) {
     const int kk = v * 8;
-    const int T = kk >> 9, l = (kk >> 4) & 31, q0 = (kk >> 2) & 3;
+    const int T = kk >> 7, pp = (kk >> 4) & 7, q0 = (kk >> 2) & 3;
 #pragma unroll
     for (int b = 0; b < B; ++b) {
       uint4 raw = make_uint4(0, 0, 0, 0);
@@ -166,7 +178,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         f.y = __uint_as_float(wd[2 * h] & 0xFFFF0000u);
         f.z = __uint_as_float(wd[2 * h + 1] << 16);
         f.w = __uint_as_float(wd[2 * h + 1] & 0xFFFF0000u);
-        const int idx = ((((T * 4 + q0 + h) * 32 + l) * B) + b) * 4;
+        const int idx = ((((T * 4 + q0 + h) * kParts + pp) * B) + b) * 4;
         *reinterpret_cast<float4 *>(xsp + idx) = f;
       }
     }
@@ -192,39 +204,42 @@ __global__ void __launch_bounds__(kThreads, 1)
           abort_flag = 1;
           break;
         }
-        mbar_arrive_expect_tx(full0 + 8 * s, (uint32_t)C);
-        bulk_g2s(ring + s * P.stage_pitch, src_of(j), (uint32_t)C,
-                 full0 + 8 * s);
+        issue(j, s);
       }
     }
   } else {
+    const int wc = warp - 1;  // consumer index; owns stages s = wc mod W
+    const int r = lane / kParts, p = lane % kParts;
     const bool paged = P.paged && (lut_addr & 0xFFFFu) == 0;
     const uint32_t perm_op =
         (paged ? (lut_addr & 0xFFFF0000u) : 0u) | ((uint32_t)lane * 4u);
-    for (int j = warp - 1; j < nchunks; j += kConsumerWarps) {
+    for (int j = wc; j < nchunks; j += P.consumers) {
       const int s = j % P.stages;
       if (!mbar_wait(full0 + 8 * s, (j / P.stages) & 1)) {
         abort_flag = 1;
         break;
       }
-      const int seg = j % P.nseg;
-      const int T0 = seg * C / kStepBytes;  // C is a multiple of 512 if nseg > 1
+      const int q = j / P.nseg, seg = j - q * P.nseg;
+      const int row = q * kRows + r;
       float acc[B];
 #pragma unroll
       for (int b = 0; b < B; ++b) acc[b] = 0.0f;
-      const uint32_t buf = ring + s * P.stage_pitch;
-      if (paged)
-        segment_dot<B, true>(buf, C, T0, lane, xs, perm_op, 0u, acc);
-      else
-        segment_dot<B, false>(buf, C, T0, lane, xs, perm_op, lut_addr, acc);
+      if (row < rows) {
+        const uint32_t rowbuf = ring + s * P.stage_pitch + r * P.row_pitch;
+        const int T0 = seg * C / kStep;  // C % 128 == 0 when nseg > 1
+        if (paged)
+          segment_dot<B, true>(rowbuf, C, T0, p, xs, perm_op, 0u, acc);
+        else
+          segment_dot<B, false>(rowbuf, C, T0, p, xs, perm_op, lut_addr, acc);
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(empty0 + 8 * s);  // stage reads are done
 #pragma unroll
       for (int b = 0; b < B; ++b) {
 #pragma unroll
-        for (int o = 16; o >= 1; o >>= 1)
+        for (int o = kParts / 2; o >= 1; o >>= 1)
           acc[b] += __shfl_xor_sync(0xFFFFFFFFu, acc[b], o);
-        if (lane == 0) part[j * B + b] = acc[b];
+        if (p == 0 && row < rows) part[(row * P.nseg + seg) * B + b] = acc[b];
       }
       if (abort_flag) break;
     }
@@ -232,8 +247,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
 
   if (abort_flag) {
-    // Give the copies still in flight (at most S) a bounded chance to land
-    // before the CTA's shared memory is released; outputs are poisoned.
+    // Give the copies still in flight (at most S stages) a bounded chance to
+    // land before the CTA's shared memory is released; outputs are poisoned.
     if (threadIdx.x == 0) {
       const int last = nchunks < P.stages ? nchunks : P.stages;
       for (int j = nchunks - last; j < nchunks; ++j)
@@ -244,10 +259,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     return;
   }
   for (int i = threadIdx.x; i < rows * B; i += blockDim.x) {
-    const int r = i / B, b = i % B;
+    const int rr = i / B, b = i % B;
     float sum = 0.0f;
-    for (int s = 0; s < P.nseg; ++s) sum += part[(r * P.nseg + s) * B + b];
-    const int64_t grow = row_lo + r;
+    for (int sg = 0; sg < P.nseg; ++sg) sum += part[(rr * P.nseg + sg) * B + b];
+    const int64_t grow = row_lo + rr;
     const float scale =
         rho ? __half2float(__ushort_as_half(rho[grow / rps])) : 1.0f;
     y[(int64_t)b * ldy + grow] = scale * sum;
@@ -260,21 +275,23 @@ StreamParams plan_stream(int64_t n, int64_t k, int B, int64_t ctas,
   StreamParams P{};
   P.rows_max = (int)((n + ctas - 1) / ctas);
   int nseg = 0;
-  for (int s = 1; s <= 64; ++s) {
+  for (int s = 1; s <= 256; ++s) {
     if (k % s) continue;
     const int64_t C = k / s;
-    if (C > 16384) continue;
-    if (s > 1 && C % kStepBytes) continue;
+    if (C > 4096) continue;
+    if (s > 1 && C % kStep) continue;
     nseg = s;
     break;
   }
   if (nseg == 0) return P;
   P.nseg = nseg;
   P.seg_bytes = (int)(k / nseg);
-  P.stage_pitch = (P.seg_bytes + 127) / 128 * 128;
-  const int64_t kpad = (k + kStepBytes - 1) / kStepBytes * kStepBytes;
+  P.row_pitch = (P.seg_bytes + 127) / 128 * 128;
+  P.stage_pitch = kRows * P.row_pitch;
+  const int64_t kpad = (k + kStep - 1) / kStep * kStep;
   const int64_t x_bytes = kpad * B * 4;
-  const int64_t part_bytes = (int64_t)P.rows_max * nseg * B * 4;
+  const int64_t quads = (P.rows_max + kRows - 1) / kRows;
+  const int64_t part_bytes = quads * kRows * nseg * B * 4;
   P.x_off = 0;
   P.part_off = (int)x_bytes;
   P.bar_off = (int)((x_bytes + part_bytes + 15) / 16 * 16);
@@ -286,15 +303,27 @@ StreamParams plan_stream(int64_t n, int64_t k, int B, int64_t ctas,
   // (b) code book right after the front, ring after it
   const int64_t lut_b = front;
   const int64_t stages_b = (max_smem - (lut_b + kLutBytes)) / P.stage_pitch;
-  const bool use_a = stages_a >= 4 && stages_a + 2 >= stages_b;
+  const bool use_a = stages_a >= 6 && stages_a + 2 >= stages_b;
   const int64_t lut = use_a ? lut_a : lut_b;
-  int64_t stages = use_a ? stages_a : stages_b;
-  if (stages > kMaxStages) stages = kMaxStages;
-  if (stages < 2) return P;
+  int64_t smax = use_a ? stages_a : stages_b;
+  if (smax > kMaxStages) smax = kMaxStages;
+  // consumers must divide the stage count: pick the pair with most consumers
+  int best_s = 0, best_w = 0;
+  for (int s = (int)smax; s >= 2; --s)
+    for (int w = kMaxConsumers; w >= 1; --w)
+      if (s % w == 0) {
+        if (w > best_w) {
+          best_w = w;
+          best_s = s;
+        }
+        break;
+      }
+  if (best_s < 2) return P;
   P.paged = use_a ? 1 : 0;
   P.lut_off = (int)lut;
   P.ring_off = (int)(lut + kLutBytes);
-  P.stages = (int)stages;
+  P.stages = best_s;
+  P.consumers = best_w;
   P.smem = (size_t)P.ring_off + (size_t)P.stages * P.stage_pitch;
   return P;
 }
@@ -325,7 +354,7 @@ cudaError_t launch_stream(const WeightsView &w, const __nv_bfloat16 *x,
   cudaError_t e = cudaFuncSetAttribute(
       kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P.smem);
   if (e != cudaSuccess) return e;
-  kern<<<(unsigned)ctas, kThreads, P.smem, stream>>>(
+  kern<<<(unsigned)ctas, 32 * (1 + P.consumers), P.smem, stream>>>(
       w.codes, w.n, w.k, w.lut, w.scales, w.rps, x, ldx, y, ldy, P);
   return cudaGetLastError();
 }
