@@ -7,8 +7,9 @@
 // clock per SM, which the per-lane code-book lookups already half use).
 //   - One CTA per SM owns rows [i*n/P, (i+1)*n/P). Warp 0 (one elected lane)
 //     streams them through a ring of S shared-memory stages with 1-D bulk
-//     copies: a stage holds a quad of 4 rows x one segment of C bytes (4
-//     copies completing on the stage's mbarrier as transaction bytes).
+//     copies: a stage holds a quad of 4 rows x one segment of C <= 1 KB (4
+//     copies completing on the stage's mbarrier as transaction bytes); small
+//     stages keep both the stage count and the consumer count high.
 //   - W consumer warps, W dividing S: stage s is always consumed by warp
 //     s mod W, so each mbarrier's phases are awaited in order by one warp.
 //   - A consumer warp's lanes are 4 rows x 8 k-parts: per 128-byte step a
@@ -32,8 +33,8 @@ namespace {
 
 constexpr int kLutBytes = 256 * 256;   // 256 entries x 32 lane copies x 4 B
 constexpr int kReservedSmem = 1024;    // system shared memory below the CTA's
-constexpr int kMaxConsumers = 15;
-constexpr int kMaxStages = 16;
+constexpr int kMaxConsumers = 16;
+constexpr int kMaxStages = 32;
 constexpr int kRows = 4;               // rows per stage
 constexpr int kParts = 8;              // k-parts (lanes) per row
 constexpr int kStep = 16 * kParts;     // codes per row per warp step (128)
@@ -278,7 +279,7 @@ StreamParams plan_stream(int64_t n, int64_t k, int B, int64_t ctas,
   for (int s = 1; s <= 256; ++s) {
     if (k % s) continue;
     const int64_t C = k / s;
-    if (C > 4096) continue;
+    if (C > 1024) continue;
     if (s > 1 && C % kStep) continue;
     nseg = s;
     break;
