@@ -10,8 +10,10 @@
 //     copies: a stage holds a quad of 4 rows x one segment of C <= 1 KB (4
 //     copies completing on the stage's mbarrier as transaction bytes); small
 //     stages keep both the stage count and the consumer count high.
-//   - W consumer warps, W dividing S: stage s is always consumed by warp
-//     s mod W, so each mbarrier's phases are awaited in order by one warp.
+//   - W = 8 consumer warps, W dividing S and S >= 3W: stage s is always
+//     consumed by warp s mod W, so each mbarrier's phases are awaited in
+//     order by one warp, and each warp has its next stages in flight while
+//     it works on one.
 //   - A consumer warp's lanes are 4 rows x 8 k-parts: per 128-byte step a
 //     lane takes 16 codes of its row, looks them up in its own copy of the
 //     code book (entry e of lane l at byte e*256 + 4*l: conflict-free; the
@@ -271,61 +273,60 @@ __global__ void __launch_bounds__(32 * (1 + kMaxConsumers), 1)
 }
 
 // Lay out shared memory for one shape; stages == 0 when it does not fit.
+// Each of the 8 consumer warps owns S/8 >= 3 stages, so that while it works
+// on one stage its next ones are already being filled.
 StreamParams plan_stream(int64_t n, int64_t k, int B, int64_t ctas,
                          int max_smem) {
+  constexpr int kConsumers = 8;
+  constexpr int kMinStages = 3 * kConsumers;
   StreamParams P{};
   P.rows_max = (int)((n + ctas - 1) / ctas);
-  int nseg = 0;
-  for (int s = 1; s <= 256; ++s) {
-    if (k % s) continue;
-    const int64_t C = k / s;
-    if (C > 1024) continue;
-    if (s > 1 && C % kStep) continue;
-    nseg = s;
-    break;
-  }
-  if (nseg == 0) return P;
-  P.nseg = nseg;
-  P.seg_bytes = (int)(k / nseg);
-  P.row_pitch = (P.seg_bytes + 127) / 128 * 128;
-  P.stage_pitch = kRows * P.row_pitch;
   const int64_t kpad = (k + kStep - 1) / kStep * kStep;
   const int64_t x_bytes = kpad * B * 4;
-  const int64_t quads = (P.rows_max + kRows - 1) / kRows;
-  const int64_t part_bytes = quads * kRows * nseg * B * 4;
   P.x_off = 0;
   P.part_off = (int)x_bytes;
-  P.bar_off = (int)((x_bytes + part_bytes + 15) / 16 * 16);
-  const int64_t front = (P.bar_off + 16 * kMaxStages + 16 + 255) / 256 * 256;
-  // (a) code book at a 64 KB aligned shared address, ring after it
-  int64_t lut_a = 65536 - kReservedSmem;
-  while (lut_a < front) lut_a += 65536;
-  const int64_t stages_a = (max_smem - (lut_a + kLutBytes)) / P.stage_pitch;
-  // (b) code book right after the front, ring after it
-  const int64_t lut_b = front;
-  const int64_t stages_b = (max_smem - (lut_b + kLutBytes)) / P.stage_pitch;
-  const bool use_a = stages_a >= 6 && stages_a + 2 >= stages_b;
-  const int64_t lut = use_a ? lut_a : lut_b;
-  int64_t smax = use_a ? stages_a : stages_b;
-  if (smax > kMaxStages) smax = kMaxStages;
-  // consumers must divide the stage count: pick the pair with most consumers
-  int best_s = 0, best_w = 0;
-  for (int s = (int)smax; s >= 2; --s)
-    for (int w = kMaxConsumers; w >= 1; --w)
-      if (s % w == 0) {
-        if (w > best_w) {
-          best_w = w;
-          best_s = s;
-        }
-        break;
-      }
-  if (best_s < 2) return P;
-  P.paged = use_a ? 1 : 0;
-  P.lut_off = (int)lut;
-  P.ring_off = (int)(lut + kLutBytes);
-  P.stages = best_s;
-  P.consumers = best_w;
-  P.smem = (size_t)P.ring_off + (size_t)P.stages * P.stage_pitch;
+  const int64_t quads = (P.rows_max + kRows - 1) / kRows;
+  // The largest segment C (dividing k; a multiple of 128 unless it is the
+  // whole row) that still leaves room for kMinStages stages.
+  for (int cmax = 2048; cmax >= kStep; cmax /= 2) {
+    int nseg = 0;
+    for (int s = 1; s <= 1024; ++s) {
+      if (k % s) continue;
+      const int64_t C = k / s;
+      if (C > cmax) continue;
+      if (s > 1 && C % kStep) continue;
+      nseg = s;
+      break;
+    }
+    if (nseg == 0) continue;
+    const int seg = (int)(k / nseg);
+    const int row_pitch = (seg + 127) / 128 * 128;
+    const int stage_pitch = kRows * row_pitch;
+    const int64_t part_bytes = quads * kRows * nseg * B * 4;
+    const int bar_off = (int)((x_bytes + part_bytes + 15) / 16 * 16);
+    const int64_t front = (bar_off + 16 * kMaxStages + 16 + 255) / 256 * 256;
+    int64_t lut_a = 65536 - kReservedSmem;  // 64 KB aligned shared address
+    while (lut_a < front) lut_a += 65536;
+    const int64_t st_a = (max_smem - (lut_a + kLutBytes)) / stage_pitch;
+    const int64_t st_b = (max_smem - (front + kLutBytes)) / stage_pitch;
+    const bool use_a = st_a >= kMinStages;
+    int64_t st = use_a ? st_a : st_b;
+    if (st > kMaxStages) st = kMaxStages;
+    st = st / kConsumers * kConsumers;
+    if (st < kMinStages) continue;
+    P.nseg = nseg;
+    P.seg_bytes = seg;
+    P.row_pitch = row_pitch;
+    P.stage_pitch = stage_pitch;
+    P.bar_off = bar_off;
+    P.paged = use_a ? 1 : 0;
+    P.lut_off = (int)(use_a ? lut_a : front);
+    P.ring_off = P.lut_off + kLutBytes;
+    P.stages = (int)st;
+    P.consumers = kConsumers;
+    P.smem = (size_t)P.ring_off + (size_t)P.stages * P.stage_pitch;
+    return P;
+  }
   return P;
 }
 
