@@ -1,0 +1,379 @@
+// Fused packed GEMM on the fifth-generation tensor cores (tcgen05), for the
+// batches where x * W_hat^T is a real contraction (batch >= 8 here):
+//   Format A: y[b][n] = sum_p sum_g s_p[n][g] sum_{j in g} t_p[n][j] x[b][j]
+//             (precisit.com page, "Three values and a shared scale"; second
+//             plane per the FUCINA README, "The method")
+//   Format B: y[b][n] = rho[n / rps] * sum_k LUT[code[n][k]] x[b][k]
+//             (alphaneural.io page, sections 3.2, 3.3 and 4.2)
+//
+// One CTA computes a 128-row tile of y^T over the whole of K for N = batch
+// rounded up to 16 (<= 64), accumulating in tensor memory (128 lanes x N
+// fp32 columns). Per 64-wide K block (and per plane):
+//   - 8 decoder warps (two per TMEM lane quarter) turn the codes of their
+//     rows into bf16 operands, written straight into shared memory in the
+//     K-major canonical layout, and stage the x tile beside them. Each weight
+//     w is split into w_hi = bf16(w) and w_lo = bf16(w - w_hi): two MMAs
+//     (hi, then lo) give products exact to ~2^-16 relative, well inside the
+//     2e-3 tolerance, with bf16 x used as is. For Format A, s*t splits
+//     exactly (an fp16 scale has 11 significant bits: 8 in s_hi, 3 in s_lo).
+//   - One thread issues the 2 x 4 MMAs (M=128, N, K=16) of the block and
+//     commits them to the stage's mbarrier, which frees the stage for the
+//     decoders. The codes are never written out as a bf16 matrix.
+//   - After the last block the accumulator is read back with tcgen05.ld,
+//     rho applied (Format B) and y stored.
+// Waits are bounded; on a time-out the CTA writes NaN to its outputs, gives
+// in-flight MMAs a bounded chance to finish, frees its tensor memory and
+// exits.
+#include "tq_common.cuh"
+#include "tq_linear.cuh"
+#include "tq_sm100_async.cuh"
+#include "tq_sm100_mma.cuh"
+
+namespace tq {
+namespace {
+
+constexpr int kTileM = 128;
+constexpr int kBlockK = 64;                       // k per stage
+constexpr int kDecoderWarps = 8;
+constexpr int kThreads = 32 * (1 + kDecoderWarps);
+constexpr int kStages = 4;
+constexpr int kSubTileA = kTileM * 32;            // one k16 step of A: 4 KB
+constexpr int kATile = 4 * kSubTileA;             // 64 k of A (hi or lo): 16 KB
+constexpr int kLutStride = 128;                   // 32 lane copies x 4 B
+constexpr int kLutBytes = 256 * kLutStride;       // 32 KB
+constexpr int kMaxN = 64;
+
+// Offset of element (row r, k in [0,64)) inside an A (or x) K-block tile:
+// four k16 sub-tiles of rows*32 bytes, each in the canonical K-major layout
+// (LBO = 128: the second 8-k column; SBO = 256: the next 8 rows).
+__device__ __forceinline__ uint32_t tile_off(int r, int k, int rows) {
+  return (uint32_t)((k >> 4) * rows * 32 + (r >> 3) * 256 +
+                    ((k >> 3) & 1) * 128 + (r & 7) * 16 + (k & 7) * 2);
+}
+
+struct TcParams {
+  int n_pad;        // N of the MMA (batch rounded up to 16)
+  int stage_bytes;  // A hi + A lo + x tile
+  int x_off;        // x tile offset inside a stage
+  int ring_off, lut_off, bar_off, tmem_slot_off;
+  size_t smem;
+};
+
+__device__ __forceinline__ uint32_t bf16_bits_rn(float v) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(v));
+}
+
+// Format B: 8 codes (two words) of one row -> 4 hi and 4 lo bf16 pairs. The
+// table word of code c for this lane holds bf16(w) | bf16(w - bf16(w)) << 16.
+__device__ __forceinline__ void decode8_b(uint32_t w0, uint32_t w1,
+                                          uint32_t lut_base, uint32_t lane8,
+                                          uint32_t (&hi)[4],
+                                          uint32_t (&lo)[4]) {
+  uint32_t v[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const uint32_t w = e < 4 ? w0 : w1;
+    const uint32_t a2 = __byte_perm(w, lane8, 0x5504u | ((uint32_t)(e & 3) << 4));
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v[e]) : "r"(lut_base + (a2 >> 1)));
+  }
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    hi[q] = __byte_perm(v[2 * q], v[2 * q + 1], 0x5410u);
+    lo[q] = __byte_perm(v[2 * q], v[2 * q + 1], 0x7632u);
+  }
+}
+
+// Format A: trits 8c..8c+7 of a group given as bit masks (bit j: t_j != 0,
+// t_j < 0) -> 4 hi and 4 lo pairs of s*t.
+__device__ __forceinline__ void decode8_a(uint64_t nz, uint64_t neg, int c,
+                                          uint32_t s_hi, uint32_t s_lo,
+                                          uint32_t (&hi)[4],
+                                          uint32_t (&lo)[4]) {
+  const uint32_t z8 = (uint32_t)(nz >> (8 * c)) & 0xFFu;
+  const uint32_t n8 = (uint32_t)(neg >> (8 * c)) & 0xFFu;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t h = 0, l = 0;
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int j = 2 * q + e;
+      const uint32_t on = (z8 >> j) & 1u, sg = ((n8 >> j) & 1u) << 15;
+      const uint32_t vh = on ? (s_hi ^ sg) : 0u;
+      const uint32_t vl = on ? (s_lo ^ sg) : 0u;
+      h |= vh << (16 * e);
+      l |= vl << (16 * e);
+    }
+    hi[q] = h;
+    lo[q] = l;
+  }
+}
+
+template <int FMT>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_tc_kernel(WeightsView w, const __nv_bfloat16 *__restrict__ x,
+                   int64_t batch, int64_t ldx, float *__restrict__ y,
+                   int64_t ldy, TcParams P) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t ring = sbase + P.ring_off;
+  const uint32_t full0 = sbase + P.bar_off;           // full[s]: decoders done
+  const uint32_t empty0 = full0 + 8 * kStages;        // empty[s]: MMAs done
+  const uint32_t acc_bar = empty0 + 8 * kStages;      // accumulator ready
+  volatile uint32_t &tmem_slot =
+      *reinterpret_cast<uint32_t *>(smem + P.tmem_slot_off);
+  volatile int &abort_flag =
+      *reinterpret_cast<int *>(smem + P.tmem_slot_off + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t row0 = (int64_t)blockIdx.x * kTileM;
+  const int N = P.n_pad;
+  const int64_t K = w.k;
+  const int kblocks = (int)((K + kBlockK - 1) / kBlockK);
+  const int planes = FMT == TQ_FMT_A ? w.planes : 1;
+  const int iters = planes * kblocks;
+  const uint32_t idesc = idesc_bf16_f32(kTileM, N);
+
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(full0 + 8 * s, kDecoderWarps);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    mbar_init(acc_bar, 1);
+    mbar_init_fence();
+  }
+  if (warp == 0) tmem_alloc(sbase + P.tmem_slot_off, 64);
+  // Lookup tables.
+  if constexpr (FMT == TQ_FMT_B) {
+    // entry e, lane copy l at e*128 + 4*l: bf16(w) | bf16(w - bf16(w)) << 16
+    for (int e = threadIdx.x; e < 256; e += blockDim.x) {
+      const float v = __ldg(w.lut + e);
+      const uint32_t h = bf16_bits_rn(v);
+      const float hv = __uint_as_float(h << 16);
+      const uint32_t l = bf16_bits_rn(v - hv);
+      const uint32_t word = h | (l << 16);
+      const uint4 w4 = make_uint4(word, word, word, word);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int jj = (j + e) & 7;
+        *reinterpret_cast<uint4 *>(smem + P.lut_off + e * kLutStride + jj * 16) =
+            w4;
+      }
+    }
+  } else {
+    // byte -> trit masks of its 5 digits: bits 0-4 t != 0, bits 5-9 t < 0
+    uint16_t *tab = reinterpret_cast<uint16_t *>(smem + P.lut_off);
+    for (int b = threadIdx.x; b < 256; b += blockDim.x) {
+      uint32_t m = 0, rest = b < 243 ? b : 121;
+#pragma unroll
+      for (int i = 0; i < 5; ++i) {
+        const uint32_t d = rest % 3;
+        rest /= 3;
+        if (d != 1) m |= 1u << i;
+        if (d == 0) m |= 1u << (5 + i);
+      }
+      tab[b] = (uint16_t)m;
+    }
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = tmem_slot;
+
+  if (warp == 0) {
+    // ---- MMA issuer ----
+    if (lane == 0) {
+      int it = 0;
+      for (; it < iters; ++it) {
+        const int s = it % kStages;
+        if (!mbar_wait(full0 + 8 * s, (it / kStages) & 1)) {
+          abort_flag = 1;
+          break;
+        }
+        tc_fence_after_sync();
+        const uint32_t st = ring + s * P.stage_bytes;
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint64_t ah = smem_desc_kmajor(st + ks * kSubTileA, 128, 256);
+          const uint64_t al =
+              smem_desc_kmajor(st + kATile + ks * kSubTileA, 128, 256);
+          const uint64_t bx =
+              smem_desc_kmajor(st + P.x_off + ks * N * 32, 128, 256);
+          mma_bf16(tmem, ah, bx, idesc, (it > 0 || ks > 0) ? 1u : 0u);
+          mma_bf16(tmem, al, bx, idesc, 1u);
+        }
+        mma_commit(empty0 + 8 * s);  // frees the stage when these finish
+      }
+      mma_commit(acc_bar);  // after every MMA issued above
+    }
+  } else {
+    // ---- decoders ----
+    const int wid = warp - 1;
+    const int quarter = warp & 3;  // TMEM lanes this warp may access
+    const int h = wid >> 2;        // which half of the 64 k of a block
+    const int r = quarter * 32 + lane;
+    const int64_t grow = row0 + r;
+    const bool row_ok = grow < w.n;
+    const uint32_t lane8 = (uint32_t)lane * 8u;
+    const uint32_t lut_base = sbase + P.lut_off;
+    const int64_t gpr = K / 64;  // Format A groups per row (G = 64)
+    for (int it = 0; it < iters && !abort_flag; ++it) {
+      const int s = it % kStages;
+      const int plane = it / kblocks, kb = it - plane * kblocks;
+      const int64_t k0 = (int64_t)kb * kBlockK;
+      // fetch this row's codes for the block before waiting for the stage
+      uint32_t cw[8];
+      uint64_t nz = 0, neg = 0;
+      uint32_t s_hi = 0, s_lo = 0;
+      if constexpr (FMT == TQ_FMT_B) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) cw[q] = 0x79797979u;  // code 121: weight 0
+        const int64_t kk = k0 + 32 * h;
+        if (row_ok) {
+          const uint8_t *p = w.codes + grow * K + kk;
+          if (kk < K) {
+            const uint4 a = *reinterpret_cast<const uint4 *>(p);
+            cw[0] = a.x; cw[1] = a.y; cw[2] = a.z; cw[3] = a.w;
+          }
+          if (kk + 16 < K) {
+            const uint4 b = *reinterpret_cast<const uint4 *>(p + 16);
+            cw[4] = b.x; cw[5] = b.y; cw[6] = b.z; cw[7] = b.w;
+          }
+        }
+      } else {
+        if (row_ok) {
+          const int64_t gi = grow * gpr + kb;
+          const uint8_t *cb = w.codes + plane * w.codes_plane_stride + gi * 13;
+          const uint16_t *tab = reinterpret_cast<const uint16_t *>(smem + P.lut_off);
+#pragma unroll
+          for (int m = 0; m < 13; ++m) {
+            const uint32_t e = tab[__ldg(cb + m)];
+            nz |= (uint64_t)(e & 31u) << (5 * m);
+            neg |= (uint64_t)((e >> 5) & 31u) << (5 * m);
+          }
+          const float sf = __half2float(__ushort_as_half(
+              __ldg(w.scales + plane * w.scales_plane_stride + gi)));
+          s_hi = bf16_bits_rn(sf);
+          s_lo = bf16_bits_rn(sf - __uint_as_float(s_hi << 16));
+        }
+      }
+      if (it >= kStages &&
+          !mbar_wait(empty0 + 8 * s, ((it / kStages) - 1) & 1)) {
+        abort_flag = 1;
+        break;
+      }
+      uint8_t *st = smem + P.ring_off + s * P.stage_bytes;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        const int c = 4 * h + cc;  // 8-k chunk of the block
+        uint32_t hi[4], lo[4];
+        if constexpr (FMT == TQ_FMT_B)
+          decode8_b(cw[2 * cc], cw[2 * cc + 1], lut_base, lane8, hi, lo);
+        else
+          decode8_a(nz, neg, c, s_hi, s_lo, hi, lo);
+        const uint32_t off = tile_off(r, 8 * c, kTileM);
+        *reinterpret_cast<uint4 *>(st + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4 *>(st + kATile + off) =
+            make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      }
+      // x tile: N rows x 64 k, 16 bytes per chunk, zero past batch and K
+      for (int id = wid * 32 + lane; id < N * 8; id += kDecoderWarps * 32) {
+        const int n = id >> 3, c = id & 7;
+        const int64_t kk = k0 + 8 * c;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (n < batch && kk < K)
+          v = *reinterpret_cast<const uint4 *>(x + (int64_t)n * ldx + kk);
+        *reinterpret_cast<uint4 *>(st + P.x_off + tile_off(n, 8 * c, N)) = v;
+      }
+      fence_async_shared();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(full0 + 8 * s);
+    }
+    // ---- epilogue: warps of the first half read their TMEM lane quarter ----
+    if (h == 0) {
+      const bool ok = mbar_wait(acc_bar, 0);
+      if (!ok) abort_flag = 1;
+      tc_fence_after_sync();
+      float scale = 1.0f;
+      if constexpr (FMT == TQ_FMT_B) {
+        if (row_ok && w.scales != nullptr)
+          scale = __half2float(__ushort_as_half(w.scales[grow / w.rps]));
+      }
+      for (int cb = 0; cb < N / 16; ++cb) {
+        uint32_t v[16];
+        tmem_ld16(tmem + ((uint32_t)(quarter * 32) << 16) + cb * 16, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int b = cb * 16 + i;
+          if (row_ok && b < batch) {
+            const float val = abort_flag ? __int_as_float(0x7FC00000)
+                                         : scale * __uint_as_float(v[i]);
+            y[(int64_t)b * ldy + grow] = val;
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, 64);
+  }
+}
+
+TcParams plan_tc(int fmt, int64_t batch) {
+  TcParams P{};
+  const int64_t b = batch < kMaxN ? batch : kMaxN;
+  P.n_pad = (int)((b + 15) / 16 * 16);
+  P.stage_bytes = 2 * kATile + P.n_pad * kBlockK * 2;
+  P.x_off = 2 * kATile;
+  P.ring_off = 0;
+  P.lut_off = kStages * P.stage_bytes;
+  const int table = fmt == TQ_FMT_B ? kLutBytes : 512;
+  P.bar_off = P.lut_off + table;
+  P.tmem_slot_off = P.bar_off + (2 * kStages + 1) * 8 + 8;
+  P.smem = (size_t)P.tmem_slot_off + 16;
+  return P;
+}
+
+template <int FMT>
+cudaError_t launch_tc(const WeightsView &w, const __nv_bfloat16 *x,
+                      int64_t batch, int64_t ldx, float *y, int64_t ldy,
+                      cudaStream_t stream) {
+  const TcParams P = plan_tc(FMT, batch);
+  auto kern = gemm_tc_kernel<FMT>;
+  cudaError_t e = cudaFuncSetAttribute(
+      kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P.smem);
+  if (e != cudaSuccess) return e;
+  const unsigned ctas = (unsigned)((w.n + kTileM - 1) / kTileM);
+  kern<<<ctas, kThreads, P.smem, stream>>>(w, x, batch, ldx, y, ldy, P);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool gemm_tc_supported(const WeightsView &w, int64_t batch) {
+  if (batch < 1) return false;
+  if (w.format == TQ_FMT_B) return true;
+  return w.format == TQ_FMT_A && w.group == 64;
+}
+
+cudaError_t gemm_tc(const WeightsView &w, const __nv_bfloat16 *x,
+                    int64_t batch, int64_t ldx, float *y, int64_t ldy,
+                    cudaStream_t stream) {
+  for (int64_t b0 = 0; b0 < batch; b0 += kMaxN) {
+    const int64_t nb = batch - b0 < kMaxN ? batch - b0 : kMaxN;
+    const cudaError_t e =
+        w.format == TQ_FMT_B
+            ? launch_tc<TQ_FMT_B>(w, x + b0 * ldx, nb, ldx, y + b0 * ldy, ldy,
+                                  stream)
+            : launch_tc<TQ_FMT_A>(w, x + b0 * ldx, nb, ldx, y + b0 * ldy, ldy,
+                                  stream);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace tq

@@ -95,7 +95,7 @@ constexpr int pow2_ceil(int v) {
 
 template <int B>
 struct GemvBCfg {
-  static constexpr int R = 2;                         // rows per group
+  static constexpr int R = (B <= 2) ? 4 : 2;          // rows per group
   static constexpr int kMaxThreads = (B == 1) ? 768 : 512;
 };
 

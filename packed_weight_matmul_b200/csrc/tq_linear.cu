@@ -6,12 +6,11 @@ namespace tq {
 cudaError_t launch_linear(const WeightsView &w, const __nv_bfloat16 *x,
                           int64_t batch, int64_t ldx, float *y, int64_t ldy,
                           cudaStream_t stream) {
-  if (gemv_b_stream_supported(w, batch))
-    return gemv_b_stream(w, x, batch, ldx, y, ldy, stream);
-  if (gemv_b_rows_supported(w, batch))
-    return gemv_b_rows(w, x, batch, ldx, y, ldy, stream);
   if (gemv_b_supported(w, batch))
     return gemv_b(w, x, batch, ldx, y, ldy, stream);
+  const int64_t tc_min_batch = w.format == TQ_FMT_B ? 5 : 2;
+  if (batch >= tc_min_batch && gemm_tc_supported(w, batch))
+    return gemm_tc(w, x, batch, ldx, y, ldy, stream);
   return linear_simple(w, x, batch, ldx, y, ldy, stream);
 }
 

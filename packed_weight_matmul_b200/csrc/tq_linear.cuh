@@ -27,4 +27,11 @@ cudaError_t gemv_b_stream(const WeightsView &w, const __nv_bfloat16 *x,
                           int64_t batch, int64_t ldx, float *y, int64_t ldy,
                           cudaStream_t stream);
 
+// Batches that are a real contraction: tcgen05 MMAs on decoded bf16 hi/lo
+// operands, accumulator in tensor memory.
+bool gemm_tc_supported(const WeightsView &w, int64_t batch);
+cudaError_t gemm_tc(const WeightsView &w, const __nv_bfloat16 *x,
+                    int64_t batch, int64_t ldx, float *y, int64_t ldy,
+                    cudaStream_t stream);
+
 }  // namespace tq
