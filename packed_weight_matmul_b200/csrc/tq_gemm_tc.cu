@@ -24,6 +24,8 @@
 // Waits are bounded; on a time-out the CTA writes NaN to its outputs, gives
 // in-flight MMAs a bounded chance to finish, frees its tensor memory and
 // exits.
+#include <cooperative_groups.h>
+
 #include "tq_common.cuh"
 #include "tq_linear.cuh"
 #include "tq_sm100_async.cuh"
@@ -52,6 +54,7 @@ __device__ __forceinline__ uint32_t tile_off(int r, int k, int rows) {
 }
 
 struct TcParams {
+  int ks_count;     // CTAs per cluster, each taking a slice of K
   int n_pad;        // N of the MMA (batch rounded up to 16)
   int stage_bytes;  // A hi + A lo + x tile
   int x_off;        // x tile offset inside a stage
@@ -125,12 +128,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       *reinterpret_cast<int *>(smem + P.tmem_slot_off + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t row0 = (int64_t)blockIdx.x * kTileM;
+  const int ks = blockIdx.x % P.ks_count;  // rank in the cluster
+  const int64_t row0 = (int64_t)(blockIdx.x / P.ks_count) * kTileM;
   const int N = P.n_pad;
   const int64_t K = w.k;
   const int kblocks = (int)((K + kBlockK - 1) / kBlockK);
   const int planes = FMT == TQ_FMT_A ? w.planes : 1;
-  const int iters = planes * kblocks;
+  const int iters_all = planes * kblocks;
+  // this CTA's slice of the (plane, k-block) iterations
+  const int it_begin = (int)((int64_t)iters_all * ks / P.ks_count);
+  const int iters = (int)((int64_t)iters_all * (ks + 1) / P.ks_count) - it_begin;
   const uint32_t idesc = idesc_bf16_f32(kTileM, N);
 
   if (threadIdx.x == 0) {
@@ -217,42 +224,86 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane8 = (uint32_t)lane * 8u;
     const uint32_t lut_base = sbase + P.lut_off;
     const int64_t gpr = K / 64;  // Format A groups per row (G = 64)
-    for (int it = 0; it < iters && !abort_flag; ++it) {
-      const int s = it % kStages;
-      const int plane = it / kblocks, kb = it - plane * kblocks;
-      const int64_t k0 = (int64_t)kb * kBlockK;
-      // fetch this row's codes for the block before waiting for the stage
-      uint32_t cw[8];
-      uint64_t nz = 0, neg = 0;
-      uint32_t s_hi = 0, s_lo = 0;
-      if constexpr (FMT == TQ_FMT_B) {
+    // Raw codes of one block, fetched a block ahead of their use.
+    struct Raw {
+      uint32_t cw[8];     // Format B: 32 codes; Format A: 16-byte window
+      uint32_t shift;     // Format A: byte offset of the group in the window
+      uint32_t scale;     // Format A: fp16 scale bits
+    };
+    const int64_t plane_bytes = w.n * gpr * 13;  // Format A code bytes per plane
+    auto fetch = [&](int it, Raw &raw) {
 #pragma unroll
-        for (int q = 0; q < 8; ++q) cw[q] = 0x79797979u;  // code 121: weight 0
-        const int64_t kk = k0 + 32 * h;
-        if (row_ok) {
-          const uint8_t *p = w.codes + grow * K + kk;
-          if (kk < K) {
-            const uint4 a = *reinterpret_cast<const uint4 *>(p);
-            cw[0] = a.x; cw[1] = a.y; cw[2] = a.z; cw[3] = a.w;
-          }
-          if (kk + 16 < K) {
-            const uint4 b = *reinterpret_cast<const uint4 *>(p + 16);
-            cw[4] = b.x; cw[5] = b.y; cw[6] = b.z; cw[7] = b.w;
-          }
+      for (int q = 0; q < 8; ++q) raw.cw[q] = 0x79797979u;  // code 121: weight 0
+      raw.shift = 0;
+      raw.scale = 0;
+      if (it >= iters || !row_ok) return;
+      const int gi_it = it_begin + it;
+      const int plane = gi_it / kblocks, kb = gi_it - plane * kblocks;
+      if constexpr (FMT == TQ_FMT_B) {
+        const int64_t kk = (int64_t)kb * kBlockK + 32 * h;
+        const uint8_t *p = w.codes + grow * K + kk;
+        if (kk < K) {
+          const uint4 a = *reinterpret_cast<const uint4 *>(p);
+          raw.cw[0] = a.x; raw.cw[1] = a.y; raw.cw[2] = a.z; raw.cw[3] = a.w;
+        }
+        if (kk + 16 < K) {
+          const uint4 b = *reinterpret_cast<const uint4 *>(p + 16);
+          raw.cw[4] = b.x; raw.cw[5] = b.y; raw.cw[6] = b.z; raw.cw[7] = b.w;
         }
       } else {
+        const int64_t gi = grow * gpr + kb;
+        const uint8_t *plane_base = w.codes + plane * w.codes_plane_stride;
+        const int64_t off = gi * 13;
+        const int64_t base = off & ~(int64_t)3;
+        raw.shift = (uint32_t)(off - base);
+        if (base + 16 <= plane_bytes) {  // 4 aligned words hold the group
+          const uint32_t *p4 = reinterpret_cast<const uint32_t *>(plane_base + base);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) raw.cw[q] = __ldg(p4 + q);
+        } else {  // last group of the plane: byte loads, never past its end
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint32_t word = 0;
+#pragma unroll
+            for (int bi = 0; bi < 4; ++bi) {
+              const int64_t o = base + 4 * q + bi;
+              if (o >= off && o < off + 13)
+                word |= (uint32_t)__ldg(plane_base + o) << (8 * bi);
+            }
+            raw.cw[q] = word;
+          }
+        }
+        raw.scale = __ldg(w.scales + plane * w.scales_plane_stride + gi);
+      }
+    };
+    Raw cur, nxt;
+    fetch(0, cur);
+    for (int it = 0; it < iters && !abort_flag; ++it) {
+      const int s = it % kStages;
+      const int kb = (it_begin + it) % kblocks;
+      const int64_t k0 = (int64_t)kb * kBlockK;
+      fetch(it + 1, nxt);  // next block's codes load during this one
+      uint32_t cw[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) cw[q] = cur.cw[q];
+      uint64_t nz = 0, neg = 0;
+      uint32_t s_hi = 0, s_lo = 0;
+      if constexpr (FMT == TQ_FMT_A) {
         if (row_ok) {
-          const int64_t gi = grow * gpr + kb;
-          const uint8_t *cb = w.codes + plane * w.codes_plane_stride + gi * 13;
-          const uint16_t *tab = reinterpret_cast<const uint16_t *>(smem + P.lut_off);
+          uint32_t v[4];
+          const uint32_t sh = 8 * cur.shift;
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            v[q] = __funnelshift_r(cw[q], q < 3 ? cw[q + 1] : 0u, sh);
+          const uint16_t *tab =
+              reinterpret_cast<const uint16_t *>(smem + P.lut_off);
 #pragma unroll
           for (int m = 0; m < 13; ++m) {
-            const uint32_t e = tab[__ldg(cb + m)];
+            const uint32_t e = tab[(v[m >> 2] >> (8 * (m & 3))) & 0xFFu];
             nz |= (uint64_t)(e & 31u) << (5 * m);
             neg |= (uint64_t)((e >> 5) & 31u) << (5 * m);
           }
-          const float sf = __half2float(__ushort_as_half(
-              __ldg(w.scales + plane * w.scales_plane_stride + gi)));
+          const float sf = __half2float(__ushort_as_half((uint16_t)cur.scale));
           s_hi = bf16_bits_rn(sf);
           s_lo = bf16_bits_rn(sf - __uint_as_float(s_hi << 16));
         }
@@ -288,10 +339,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_async_shared();
       __syncwarp();
       if (lane == 0) mbar_arrive(full0 + 8 * s);
+      cur = nxt;
     }
     // ---- epilogue: warps of the first half read their TMEM lane quarter ----
     if (h == 0) {
-      const bool ok = mbar_wait(acc_bar, 0);
+      const bool ok = iters == 0 || mbar_wait(acc_bar, 0);
       if (!ok) abort_flag = 1;
       tc_fence_after_sync();
       float scale = 1.0f;
@@ -299,6 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (row_ok && w.scales != nullptr)
           scale = __half2float(__ushort_as_half(w.scales[grow / w.rps]));
       }
+      float *part = reinterpret_cast<float *>(smem + P.ring_off);  // [128][N]
       for (int cb = 0; cb < N / 16; ++cb) {
         uint32_t v[16];
         tmem_ld16(tmem + ((uint32_t)(quarter * 32) << 16) + cb * 16, v);
@@ -306,10 +359,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int b = cb * 16 + i;
-          if (row_ok && b < batch) {
-            const float val = abort_flag ? __int_as_float(0x7FC00000)
-                                         : scale * __uint_as_float(v[i]);
-            y[(int64_t)b * ldy + grow] = val;
+          float val = iters == 0 ? 0.0f : __uint_as_float(v[i]);
+          if (abort_flag) val = __int_as_float(0x7FC00000);
+          if (P.ks_count > 1) {
+            part[r * N + b] = val;  // summed across the cluster below
+          } else if (row_ok && b < batch) {
+            y[(int64_t)b * ldy + grow] = scale * val;
           }
         }
       }
@@ -317,6 +372,31 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   tc_fence_before_sync();
   __syncthreads();
+  if (P.ks_count > 1) {
+    // Sum the cluster's partial tiles through distributed shared memory in
+    // rank order (deterministic); this CTA finishes its share of the rows.
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    cluster.sync();
+    const float *part = reinterpret_cast<const float *>(smem + P.ring_off);
+    const int r_lo = kTileM * ks / P.ks_count;
+    const int r_hi = kTileM * (ks + 1) / P.ks_count;
+    for (int i = threadIdx.x; i < (r_hi - r_lo) * N; i += blockDim.x) {
+      const int rr = r_lo + i / N, b = i % N;
+      const int64_t gr = row0 + rr;
+      if (gr >= w.n || b >= batch) continue;
+      float sum = 0.0f;
+      for (int q = 0; q < P.ks_count; ++q)
+        sum += cluster.map_shared_rank(part, q)[rr * N + b];
+      float scale = 1.0f;
+      if constexpr (FMT == TQ_FMT_B) {
+        if (w.scales != nullptr)
+          scale = __half2float(__ushort_as_half(w.scales[gr / w.rps]));
+      }
+      y[(int64_t)b * ldy + gr] = scale * sum;
+    }
+    cluster.sync();  // no CTA leaves while others read its partials
+  }
   if (warp == 0) {
     tc_fence_after_sync();
     tmem_dealloc(tmem, 64);
@@ -338,18 +418,52 @@ TcParams plan_tc(int fmt, int64_t batch) {
   return P;
 }
 
+// Cluster size (K slices per tile): the one that best fills whole waves of
+// one CTA per SM, preferring no split.
+int pick_ks(int64_t tiles, int iters, int sms) {
+  int best = 1;
+  double best_eff = 0.0;
+  for (int ks = 1; ks <= 8 && ks <= iters; ++ks) {
+    const double ctas = (double)(tiles * ks);
+    const double waves = ctas / sms;
+    const double eff = waves / ceil(waves) - 0.02 * (ks - 1);
+    if (eff > best_eff + 1e-9) {
+      best_eff = eff;
+      best = ks;
+    }
+  }
+  return best;
+}
+
 template <int FMT>
 cudaError_t launch_tc(const WeightsView &w, const __nv_bfloat16 *x,
                       int64_t batch, int64_t ldx, float *y, int64_t ldy,
                       cudaStream_t stream) {
-  const TcParams P = plan_tc(FMT, batch);
+  TcParams P = plan_tc(FMT, batch);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t tiles = (w.n + kTileM - 1) / kTileM;
+  const int kblocks = (int)((w.k + kBlockK - 1) / kBlockK);
+  const int iters = (FMT == TQ_FMT_A ? w.planes : 1) * kblocks;
+  P.ks_count = pick_ks(tiles, iters, sms);
   auto kern = gemm_tc_kernel<FMT>;
   cudaError_t e = cudaFuncSetAttribute(
       kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P.smem);
   if (e != cudaSuccess) return e;
-  const unsigned ctas = (unsigned)((w.n + kTileM - 1) / kTileM);
-  kern<<<ctas, kThreads, P.smem, stream>>>(w, x, batch, ldx, y, ldy, P);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(tiles * P.ks_count), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = P.smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)P.ks_count;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, w, x, batch, ldx, y, ldy, P);
 }
 
 }  // namespace
