@@ -253,11 +253,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         const int64_t gi = grow * gpr + kb;
         const uint8_t *plane_base = w.codes + plane * w.codes_plane_stride;
-        const int64_t off = gi * 13;
-        const int64_t base = off & ~(int64_t)3;
-        raw.shift = (uint32_t)(off - base);
-        if (base + 16 <= plane_bytes) {  // 4 aligned words hold the group
-          const uint32_t *p4 = reinterpret_cast<const uint32_t *>(plane_base + base);
+        const uint8_t *grp = plane_base + gi * 13;
+        // 4-byte aligned window on the absolute address (a plane may start
+        // at any byte); it never starts before the 16-byte aligned buffer
+        // and is used only when it ends inside this plane's data.
+        const uint8_t *win = reinterpret_cast<const uint8_t *>(
+            reinterpret_cast<uintptr_t>(grp) & ~(uintptr_t)3);
+        raw.shift = (uint32_t)(grp - win);
+        if (win + 16 <= plane_base + plane_bytes) {
+          const uint32_t *p4 = reinterpret_cast<const uint32_t *>(win);
 #pragma unroll
           for (int q = 0; q < 4; ++q) raw.cw[q] = __ldg(p4 + q);
         } else {  // last group of the plane: byte loads, never past its end
@@ -266,9 +270,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t word = 0;
 #pragma unroll
             for (int bi = 0; bi < 4; ++bi) {
-              const int64_t o = base + 4 * q + bi;
-              if (o >= off && o < off + 13)
-                word |= (uint32_t)__ldg(plane_base + o) << (8 * bi);
+              const uint8_t *b = win + 4 * q + bi;
+              if (b >= grp && b < grp + 13) word |= (uint32_t)__ldg(b) << (8 * bi);
             }
             raw.cw[q] = word;
           }
