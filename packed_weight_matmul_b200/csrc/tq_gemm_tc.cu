@@ -38,7 +38,8 @@ constexpr int kTileM = 128;
 constexpr int kBlockK = 64;                       // k per stage
 constexpr int kDecoderWarps = 8;
 constexpr int kThreads = 32 * (1 + kDecoderWarps);
-constexpr int kStages = 4;
+constexpr int kStages = 3;
+constexpr int kCodeDepth = 6;                     // code blocks per thread ring
 constexpr int kSubTileA = kTileM * 32;            // one k16 step of A: 4 KB
 constexpr int kATile = 4 * kSubTileA;             // 64 k of A (hi or lo): 16 KB
 constexpr int kLutStride = 128;                   // 32 lane copies x 4 B
@@ -59,8 +60,32 @@ struct TcParams {
   int stage_bytes;  // A hi + A lo + x tile
   int x_off;        // x tile offset inside a stage
   int ring_off, lut_off, bar_off, tmem_slot_off;
+  int code_off, code_slot;  // code ring: kCodeDepth slots of 128 rows x 64 B
   size_t smem;
 };
+
+// Asynchronous global -> shared copies; `n` < size bytes are read, the rest
+// of the destination is zero-filled.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, int n) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst),
+               "l"(src), "r"(n)
+               : "memory");
+}
+
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src, int n) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst),
+               "l"(src), "r"(n)
+               : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 
 __device__ __forceinline__ uint32_t bf16_bits_rn(float v) {
   return __bfloat16_as_ushort(__float2bfloat16_rn(v));
@@ -224,77 +249,89 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane8 = (uint32_t)lane * 8u;
     const uint32_t lut_base = sbase + P.lut_off;
     const int64_t gpr = K / 64;  // Format A groups per row (G = 64)
-    // Raw codes of one block, fetched a block ahead of their use.
-    struct Raw {
-      uint32_t cw[8];     // Format B: 32 codes; Format A: 16-byte window
-      uint32_t shift;     // Format A: byte offset of the group in the window
-      uint32_t scale;     // Format A: fp16 scale bits
-    };
+    auto plane_of = [&](int it) { return (it_begin + it) / kblocks; };
+    // Codes stream into a per-thread ring of kCodeDepth blocks in shared
+    // memory with cp.async (each thread reads back only the bytes its own
+    // copies wrote), so kCodeDepth - 1 blocks of every row are in flight.
     const int64_t plane_bytes = w.n * gpr * 13;  // Format A code bytes per plane
-    auto fetch = [&](int it, Raw &raw) {
+    const uint32_t code_ring = sbase + P.code_off + r * 64 + h * 32;
+    uint32_t sc[kCodeDepth];                      // Format A scales, in order
 #pragma unroll
-      for (int q = 0; q < 8; ++q) raw.cw[q] = 0x79797979u;  // code 121: weight 0
-      raw.shift = 0;
-      raw.scale = 0;
-      if (it >= iters || !row_ok) return;
+    for (int q = 0; q < kCodeDepth; ++q) sc[q] = 0;
+    auto issue = [&](int it) -> uint32_t {      // returns the block's scale
+      const uint32_t dst = code_ring + (uint32_t)(it % kCodeDepth) * P.code_slot;
+      if (it >= iters) return 0;
       const int gi_it = it_begin + it;
       const int plane = gi_it / kblocks, kb = gi_it - plane * kblocks;
       if constexpr (FMT == TQ_FMT_B) {
         const int64_t kk = (int64_t)kb * kBlockK + 32 * h;
-        const uint8_t *p = w.codes + grow * K + kk;
-        if (kk < K) {
-          const uint4 a = *reinterpret_cast<const uint4 *>(p);
-          raw.cw[0] = a.x; raw.cw[1] = a.y; raw.cw[2] = a.z; raw.cw[3] = a.w;
-        }
-        if (kk + 16 < K) {
-          const uint4 b = *reinterpret_cast<const uint4 *>(p + 16);
-          raw.cw[4] = b.x; raw.cw[5] = b.y; raw.cw[6] = b.z; raw.cw[7] = b.w;
-        }
+        const uint8_t *p = w.codes + (row_ok ? grow : 0) * K + kk;
+        cp_async16(dst, row_ok && kk < K ? p : w.codes, row_ok && kk < K ? 16 : 0);
+        cp_async16(dst + 16, row_ok && kk + 16 < K ? p + 16 : w.codes,
+                   row_ok && kk + 16 < K ? 16 : 0);
+        return 0;
       } else {
+        if (!row_ok) return 0;
         const int64_t gi = grow * gpr + kb;
         const uint8_t *plane_base = w.codes + plane * w.codes_plane_stride;
         const uint8_t *grp = plane_base + gi * 13;
+        const uint8_t *end = plane_base + plane_bytes;
         // 4-byte aligned window on the absolute address (a plane may start
-        // at any byte); it never starts before the 16-byte aligned buffer
-        // and is used only when it ends inside this plane's data.
+        // at any byte); copies stop at the end of this plane's data.
         const uint8_t *win = reinterpret_cast<const uint8_t *>(
             reinterpret_cast<uintptr_t>(grp) & ~(uintptr_t)3);
-        raw.shift = (uint32_t)(grp - win);
-        if (win + 16 <= plane_base + plane_bytes) {
-          const uint32_t *p4 = reinterpret_cast<const uint32_t *>(win);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) raw.cw[q] = __ldg(p4 + q);
-        } else {  // last group of the plane: byte loads, never past its end
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint32_t word = 0;
-#pragma unroll
-            for (int bi = 0; bi < 4; ++bi) {
-              const uint8_t *b = win + 4 * q + bi;
-              if (b >= grp && b < grp + 13) word |= (uint32_t)__ldg(b) << (8 * bi);
-            }
-            raw.cw[q] = word;
-          }
+        for (int q = 0; q < 4; ++q) {
+          const uint8_t *src = win + 4 * q;
+          const int64_t left = end - src;
+          const int n = left >= 4 ? 4 : (left > 0 ? (int)left : 0);
+          cp_async4(dst + 4 * q, n > 0 ? src : w.codes, n);
         }
-        raw.scale = __ldg(w.scales + plane * w.scales_plane_stride + gi);
+        return __ldg(w.scales + plane * w.scales_plane_stride + gi);
       }
     };
-    Raw cur, nxt;
-    fetch(0, cur);
+#pragma unroll
+    for (int q = 0; q < kCodeDepth - 1; ++q) {
+      sc[q] = issue(q);
+      cp_async_commit();
+    }
     for (int it = 0; it < iters && !abort_flag; ++it) {
       const int s = it % kStages;
       const int kb = (it_begin + it) % kblocks;
       const int64_t k0 = (int64_t)kb * kBlockK;
-      fetch(it + 1, nxt);  // next block's codes load during this one
+      sc[kCodeDepth - 1] = issue(it + kCodeDepth - 1);
+      cp_async_commit();
+      cp_async_wait<kCodeDepth - 1>();  // this block's codes have landed
+      const uint32_t src = code_ring + (uint32_t)(it % kCodeDepth) * P.code_slot;
       uint32_t cw[8];
+      {
+        uint4 a, b2;
+        asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                     : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w) : "r"(src));
+        asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                     : "=r"(b2.x), "=r"(b2.y), "=r"(b2.z), "=r"(b2.w)
+                     : "r"(src + 16));
+        cw[0] = a.x; cw[1] = a.y; cw[2] = a.z; cw[3] = a.w;
+        cw[4] = b2.x; cw[5] = b2.y; cw[6] = b2.z; cw[7] = b2.w;
+      }
+      if constexpr (FMT == TQ_FMT_B) {
+        if (!row_ok) {
 #pragma unroll
-      for (int q = 0; q < 8; ++q) cw[q] = cur.cw[q];
+          for (int q = 0; q < 8; ++q) cw[q] = 0x79797979u;  // weight 0
+        }
+      }
+      const uint32_t cur_scale = sc[0];
+#pragma unroll
+      for (int q = 0; q + 1 < kCodeDepth; ++q) sc[q] = sc[q + 1];
       uint64_t nz = 0, neg = 0;
       uint32_t s_hi = 0, s_lo = 0;
       if constexpr (FMT == TQ_FMT_A) {
         if (row_ok) {
           uint32_t v[4];
-          const uint32_t sh = 8 * cur.shift;
+          const uint32_t sh =
+              8u * (uint32_t)(reinterpret_cast<uintptr_t>(
+                                  w.codes + plane_of(it) * w.codes_plane_stride +
+                                  (grow * gpr + kb) * 13) & 3);
 #pragma unroll
           for (int q = 0; q < 4; ++q)
             v[q] = __funnelshift_r(cw[q], q < 3 ? cw[q + 1] : 0u, sh);
@@ -306,7 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             nz |= (uint64_t)(e & 31u) << (5 * m);
             neg |= (uint64_t)((e >> 5) & 31u) << (5 * m);
           }
-          const float sf = __half2float(__ushort_as_half((uint16_t)cur.scale));
+          const float sf = __half2float(__ushort_as_half((uint16_t)cur_scale));
           s_hi = bf16_bits_rn(sf);
           s_lo = bf16_bits_rn(sf - __uint_as_float(s_hi << 16));
         }
@@ -342,8 +379,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_async_shared();
       __syncwarp();
       if (lane == 0) mbar_arrive(full0 + 8 * s);
-      cur = nxt;
     }
+    cp_async_wait<0>();
     // ---- epilogue: warps of the first half read their TMEM lane quarter ----
     if (h == 0) {
       const bool ok = iters == 0 || mbar_wait(acc_bar, 0);
@@ -413,7 +450,9 @@ TcParams plan_tc(int fmt, int64_t batch) {
   P.stage_bytes = 2 * kATile + P.n_pad * kBlockK * 2;
   P.x_off = 2 * kATile;
   P.ring_off = 0;
-  P.lut_off = kStages * P.stage_bytes;
+  P.code_slot = kTileM * 64;
+  P.code_off = kStages * P.stage_bytes;
+  P.lut_off = P.code_off + kCodeDepth * P.code_slot;
   const int table = fmt == TQ_FMT_B ? kLutBytes : 512;
   P.bar_off = P.lut_off + table;
   P.tmem_slot_off = P.bar_off + (2 * kStages + 1) * 8 + 8;
