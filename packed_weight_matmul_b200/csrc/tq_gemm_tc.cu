@@ -295,6 +295,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       sc[q] = issue(q);
       cp_async_commit();
     }
+    // This thread's (at most two) 16-byte x chunks of block it; zero past
+    // the batch, past K and past the slice.
+    auto load_x = [&](int it, uint4 (&v)[2]) {
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        v[q] = make_uint4(0, 0, 0, 0);
+        const int id = wid * 32 + lane + q * kDecoderWarps * 32;
+        const int n = id >> 3, c = id & 7;
+        if (it < iters && id < N * 8 && n < batch) {
+          const int64_t kk = (int64_t)((it_begin + it) % kblocks) * kBlockK + 8 * c;
+          if (kk < K) v[q] = *reinterpret_cast<const uint4 *>(x + (int64_t)n * ldx + kk);
+        }
+      }
+    };
+    uint4 xr0[2], xr1[2];
+    load_x(0, xr0);
+    load_x(1, xr1);
     for (int it = 0; it < iters && !abort_flag; ++it) {
       const int s = it % kStages;
       const int kb = (it_begin + it) % kblocks;
@@ -367,15 +384,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         *reinterpret_cast<uint4 *>(st + kATile + off) =
             make_uint4(lo[0], lo[1], lo[2], lo[3]);
       }
-      // x tile: N rows x 64 k, 16 bytes per chunk, zero past batch and K
-      for (int id = wid * 32 + lane; id < N * 8; id += kDecoderWarps * 32) {
-        const int n = id >> 3, c = id & 7;
-        const int64_t kk = k0 + 8 * c;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (n < batch && kk < K)
-          v = *reinterpret_cast<const uint4 *>(x + (int64_t)n * ldx + kk);
-        *reinterpret_cast<uint4 *>(st + P.x_off + tile_off(n, 8 * c, N)) = v;
+      // x tile: N rows x 64 k, 16 bytes per chunk (fetched two blocks ahead)
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const int id = wid * 32 + lane + q * kDecoderWarps * 32;
+        if (id < N * 8)
+          *reinterpret_cast<uint4 *>(st + P.x_off +
+                                     tile_off(id >> 3, 8 * (id & 7), N)) = xr0[q];
+        xr0[q] = xr1[q];
       }
+      load_x(it + 2, xr1);
       fence_async_shared();
       __syncwarp();
       if (lane == 0) mbar_arrive(full0 + 8 * s);
