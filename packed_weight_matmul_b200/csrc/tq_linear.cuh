@@ -15,18 +15,6 @@ bool gemv_b_supported(const WeightsView &w, int64_t batch);
 cudaError_t gemv_b(const WeightsView &w, const __nv_bfloat16 *x, int64_t batch,
                    int64_t ldx, float *y, int64_t ldy, cudaStream_t stream);
 
-// Format B, batch 1..2: row-parallel lanes, x staged in shared memory.
-bool gemv_b_rows_supported(const WeightsView &w, int64_t batch);
-cudaError_t gemv_b_rows(const WeightsView &w, const __nv_bfloat16 *x,
-                        int64_t batch, int64_t ldx, float *y, int64_t ldy,
-                        cudaStream_t stream);
-
-// Format B, batch 1..2: rows streamed through shared memory by bulk copies.
-bool gemv_b_stream_supported(const WeightsView &w, int64_t batch);
-cudaError_t gemv_b_stream(const WeightsView &w, const __nv_bfloat16 *x,
-                          int64_t batch, int64_t ldx, float *y, int64_t ldy,
-                          cudaStream_t stream);
-
 // Batches that are a real contraction: tcgen05 MMAs on decoded bf16 hi/lo
 // operands, accumulator in tensor memory.
 bool gemm_tc_supported(const WeightsView &w, int64_t batch);
