@@ -11,21 +11,23 @@
 //     address, a warp's 32 lookups hit 32 distinct banks, and all 256 byte
 //     values are present, so an invalid code reads its NaN entry.
 //   - Two neighbouring weights are multiplied by their two x values with one
-//     packed fp32x2 FMA (even and odd k accumulate separately and are added
-//     at the end of a unit).
-//   - Work unit: R rows x one k-chunk of 32 lanes x KPL codes (16-byte or
-//     8-byte loads per lane and row, a fully coalesced 512- or 256-byte run
-//     per row). A CTA (one per SM) owns an even share of the rows; its units
-//     are ordered chunk-major and cut into equal contiguous ranges, one per
-//     warp, so every warp does the same amount of work (+-1 unit) and keeps
-//     the chunk's x in registers across the row groups it walks.
-//   - Codes of the next D-1 units are in flight while a unit is computed (a
-//     register ring, 128-bit loads that bypass L1); the x of the next chunk
-//     is fetched while the current chunk is in use.
-//   - A unit's R*B sums are reduced across lanes by a transposing butterfly
-//     and written to a per-(chunk, row) slot in shared memory; the slots of a
-//     row are added in chunk order at the end, so the result does not depend
-//     on timing.
+//     packed fp32x2 FMA (even and odd k accumulate separately).
+//   - Work unit: R rows x one k-chunk of 512 codes (16 per lane, a fully
+//     coalesced 512-byte run per row). A CTA (one per SM) owns an even share
+//     of the rows; its units are ordered row-group major and cut into equal
+//     contiguous ranges, one per warp, so every warp does the same amount of
+//     work (+-1 unit) and streams along its rows.
+//   - HBM needs tens of KB in flight per SM. The codes therefore stream
+//     through a per-warp ring of D unit slots in shared memory, filled by
+//     asynchronous 16-byte copies (each lane copies, and later reads back,
+//     only its own bytes, so no barrier is involved); D-1 units are in
+//     flight while one is computed, without holding registers. The rings
+//     live in the shared memory around the code book. x is read through
+//     the caches (L2, and L1 where it fits), one unit ahead.
+//   - Sums stay in registers along a row segment; at its end the R*B values
+//     are reduced across lanes by a transposing butterfly and stored in the
+//     slot of the segment's first chunk. The slots of a row are added in a
+//     fixed order at the end, so the result does not depend on timing.
 #include "tq_common.cuh"
 #include "tq_linear.cuh"
 
@@ -36,28 +38,59 @@ constexpr uint32_t kLutAddr = 0x10000u;  // shared-window address of the book
 constexpr uint32_t kLutStride = 256;     // bytes per entry (32 lane copies)
 constexpr uint32_t kRedAddr = 0x20000u;  // partial sums follow the book
 constexpr int kSmemMax = 227 * 1024;     // dynamic shared memory per CTA
-// The request covers [0, kRedAddr + red) whatever the window base is.
-constexpr int kRedMaxBytes = kSmemMax - (int)kRedAddr;
+// Rings below the code book start at or below this shared-window address
+// (the dynamic window starts right after the 1 KB reserved per CTA).
+constexpr uint32_t kRingLoAddr = 0x1000u;
+constexpr int KPL = 16;             // codes per lane and row
+constexpr int KC = 32 * KPL;        // codes per chunk
+constexpr uint32_t kRowBytes = KC;  // one row of a unit slot
 
-__device__ __forceinline__ uint4 ld_stream16(const void *p) {
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src,
+                                           uint32_t n) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst),
+               "l"(src), "r"(n)
+               : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// x: read-only and shared by every row (cached loads). Volatile so that it
+// stays where it is issued, a unit ahead of its use.
+__device__ __forceinline__ uint4 ld_x16(const void *p) {
   uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "l"(p));
   return v;
 }
 
-__device__ __forceinline__ uint2 ld_stream8(const void *p) {
-  uint2 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
-               : "=r"(v.x), "=r"(v.y)
-               : "l"(p));
+__device__ __forceinline__ uint4 lds_v4(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(a)
+               : "memory");
   return v;
 }
 
+// Code-book lookup. Not volatile, so the compiler may schedule it freely; it
+// is ordered after the code book is built through its address operand.
 __device__ __forceinline__ float lds_f32(uint32_t a) {
   float v;
-  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
+  asm("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
+  return v;
+}
+
+__device__ __forceinline__ float lds_f32_volatile(uint32_t a) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory");
   return v;
 }
 
@@ -100,144 +133,171 @@ constexpr int pow2_ceil(int v) {
   return p;
 }
 
-// Position of a work unit: chunk c, row group g, and the byte offset of this
-// lane's codes for the group's first row.
+// Position of a work unit: row group g and chunk c.
 struct UnitPos {
-  int c, g;
-  int64_t off;
+  int g, c;
 };
 
-template <int B, int KPL, int R, int D, int NT>
+__device__ __forceinline__ void advance(UnitPos &q, int nchunks) {
+  if (++q.c == nchunks) {
+    q.c = 0;
+    ++q.g;
+  }
+}
+
+// hi_ring: shared-window address of the rings placed above the partial sums.
+template <int B, int R, int D, int NT>
 __global__ void __launch_bounds__(NT, 1)
     gemv_b_kernel(const uint8_t *__restrict__ codes, int64_t n, int64_t k,
                   const float *__restrict__ lut,
                   const uint16_t *__restrict__ rho, int rps,
                   const __nv_bfloat16 *__restrict__ x, int64_t ldx,
-                  float *__restrict__ y, int64_t ldy, int rows_max) {
-  constexpr int KC = 32 * KPL;         // k per chunk
+                  float *__restrict__ y, int64_t ldy, int rows_max,
+                  uint32_t hi_ring) {
   constexpr int NW = KPL / 4;          // code words per lane and row
-  constexpr int NX = KPL / 2;          // x pairs per lane and batch row
-  constexpr int M = pow2_ceil(R * B);  // values reduced per unit
+  constexpr int NX = KPL / 2;          // x words (bf16 pairs) per lane and row
+  constexpr int M = pow2_ceil(R * B);  // values reduced per row segment
   constexpr int kWarps = NT / 32;
+  constexpr uint32_t kSlot = R * kRowBytes;  // one unit's codes
+  constexpr uint32_t kRing = D * kSlot;      // one warp's ring
   extern __shared__ __align__(16) uint8_t smem[];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t row_lo = (int64_t)blockIdx.x * n / gridDim.x;
   const int rows = (int)((int64_t)(blockIdx.x + 1) * n / gridDim.x - row_lo);
 
-  // The code book must start exactly at kLutAddr; the request size makes the
-  // window reach kRedAddr + partial sums when the base is at most kLutAddr.
+  // The layout assumes the dynamic window starts at or below kRingLoAddr
+  // (then the request covers the code book, the partial sums and the rings).
   const uint32_t base = (uint32_t)__cvta_generic_to_shared(smem);
-  if (base > kLutAddr) {
+  if (base > kRingLoAddr) {
     for (int i = threadIdx.x; i < rows * B; i += NT) {
       const int r = i / B, b = i - r * B;
       y[(int64_t)b * ldy + row_lo + r] = __int_as_float(0x7FC00000);
     }
     return;
   }
+  const uint32_t lo_ring = (base + 127u) & ~127u;
+  const int lo_warps = (int)((kLutAddr - lo_ring) / kRing);
+  const uint32_t ring = warp < lo_warps
+                            ? lo_ring + (uint32_t)warp * kRing
+                            : hi_ring + (uint32_t)(warp - lo_warps) * kRing;
+  const uint32_t ring_end = ring + kRing;
+  const uint32_t lane16 = (uint32_t)lane * 16u;
 
   const int ng = (rows + R - 1) / R;
   const int nchunks = (int)((k + KC - 1) / KC);
-  const int units = ng * nchunks;
+  const int units = ng * nchunks;  // row-group major: u = g * nchunks + c
   const int u_begin = (int)((int64_t)units * warp / kWarps);
   const int u_end = (int)((int64_t)units * (warp + 1) / kWarps);
   const int64_t kstride = k;
   const int64_t group_step = (int64_t)R * kstride;
   const uint8_t *crow = codes + row_lo * kstride + lane * KPL;
+  const __nv_bfloat16 *xl = x + lane * KPL;
+  // lanes past k in the last chunk hold nothing
+  const bool last_ok = (int64_t)(nchunks - 1) * KC + lane * KPL < k;
 
-  UnitPos ld;  // next unit whose codes are loaded
-  ld.c = u_begin / ng;
-  ld.g = u_begin - ld.c * ng;
-  ld.off = (int64_t)ld.g * group_step + (int64_t)ld.c * KC;
+  UnitPos ld;  // next unit whose codes are copied
+  ld.g = u_begin / nchunks;
+  ld.c = u_begin - ld.g * nchunks;
+  const uint8_t *ld_p = crow + (int64_t)ld.g * group_step + (int64_t)ld.c * KC;
   int u_ld = u_begin;
+  uint32_t ld_slot = ring;
   UnitPos cur = ld;
 
-  auto advance = [&](UnitPos &p) {
-    if (++p.g == ng) {
-      p.g = 0;
-      ++p.c;
-      p.off = (int64_t)p.c * KC;
-    } else {
-      p.off += group_step;
-    }
-  };
-  auto lane_in_k = [&](int c) { return (int64_t)c * KC + lane * KPL < k; };
-
-  // Codes of unit u_ld into slot cw, 121 (weight 0) where nothing is loaded.
-  auto issue = [&](uint32_t (&cw)[R][NW]) {
-    const bool ok = u_ld < u_end && lane_in_k(ld.c);
+  // Copy unit u_ld's codes into the next ring slot (one commit group per
+  // unit, empty past the range). Rows past the CTA's rows and lanes past k
+  // are zero-filled; their products are never used.
+  auto issue = [&]() {
+    if (u_ld < u_end) {
+      const uint32_t dst = ld_slot + lane16;
+      const bool full =
+          (ld.g + 1) * R <= rows && (int64_t)(ld.c + 1) * KC <= k;  // uniform
+      if (full) {
 #pragma unroll
-    for (int r = 0; r < R; ++r) {
-      const bool okr = ok && ld.g * R + r < rows;
-      const uint8_t *p = crow + ld.off + r * kstride;
-      if constexpr (KPL == 16) {
-        uint4 v = make_uint4(0x79797979u, 0x79797979u, 0x79797979u,
-                             0x79797979u);
-        if (okr) v = ld_stream16(p);
-        cw[r][0] = v.x; cw[r][1] = v.y; cw[r][2] = v.z; cw[r][3] = v.w;
+        for (int r = 0; r < R; ++r)
+          cp_async16(dst + r * kRowBytes, ld_p + r * kstride, 16u);
       } else {
-        uint2 v = make_uint2(0x79797979u, 0x79797979u);
-        if (okr) v = ld_stream8(p);
-        cw[r][0] = v.x; cw[r][1] = v.y;
+        const bool ok = ld.c + 1 < nchunks || last_ok;
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          const bool okr = ok && ld.g * R + r < rows;
+          cp_async16(dst + r * kRowBytes, okr ? ld_p + r * kstride : codes,
+                     okr ? 16u : 0u);
+        }
       }
+      advance(ld, nchunks);
+      ld_p = ld.c == 0 ? crow + (int64_t)ld.g * group_step : ld_p + KC;
     }
-    if (u_ld < u_end) advance(ld);
+    cp_async_commit();
+    ld_slot = ld_slot + kSlot == ring_end ? ring : ld_slot + kSlot;
     ++u_ld;
   };
 
-  // Raw bf16 x words of chunk c for this lane (zero outside k).
-  uint32_t xr[B][NX];
+  // Raw bf16 x of chunk c for this lane (zero past k).
+  uint32_t xw[B][NX];
   auto load_x = [&](int c) {
-    const bool ok = c < nchunks && lane_in_k(c);
-    const int64_t kb = (int64_t)c * KC + lane * KPL;
+    const bool ok = c + 1 < nchunks || last_ok;
+    const __nv_bfloat16 *xp = xl + (int64_t)c * KC;
 #pragma unroll
-    for (int b = 0; b < B; ++b) {
+    for (int b = 0; b < B; ++b)
 #pragma unroll
       for (int q = 0; q < NX; q += 4) {
         uint4 v = make_uint4(0, 0, 0, 0);
-        if (ok) v = *reinterpret_cast<const uint4 *>(x + b * ldx + kb + 2 * q);
-        xr[b][q] = v.x;
-        xr[b][q + 1] = v.y;
-        xr[b][q + 2] = v.z;
-        xr[b][q + 3] = v.w;
+        if (ok) v = ld_x16(xp + b * ldx + 2 * q);
+        xw[b][q] = v.x;
+        xw[b][q + 1] = v.y;
+        xw[b][q + 2] = v.z;
+        xw[b][q + 3] = v.w;
       }
-    }
   };
 
-  // Start the first loads, then build the code book while they fly.
-  uint32_t cw[D][R][NW];
+  // Start the first copies, then clear the partial sums and build the code
+  // book while they fly.
 #pragma unroll
-  for (int d = 0; d < D; ++d) issue(cw[d]);
+  for (int d = 0; d < D - 1; ++d) issue();
   load_x(cur.c);
+  const int red_words = nchunks * rows_max * B;
+  for (int i = threadIdx.x; i < red_words; i += NT)
+    sts_f32(kRedAddr + 4u * (uint32_t)i, 0.0f);
   for (int i = threadIdx.x; i < 256 * 8; i += NT) {
     const int e = i >> 3, j = i & 7;
     sts_v4(kLutAddr + e * kLutStride + j * 16, __ldg(lut + e));
   }
   __syncthreads();
+  // Defined after the barrier (volatile), so no table lookup can be hoisted
+  // above it.
+  uint32_t lane_lut;
+  asm volatile("mov.b32 %0, %1;" : "=r"(lane_lut) : "r"(kLutAddr | (lane << 2)));
 
-  const uint32_t lane_lut = kLutAddr | ((uint32_t)lane << 2);
-  float2 xv[B][NX];
-  int xc = -1;  // chunk whose x is in xv
-  bool k_ok = false;
+  float2 acc[R][B];
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int b = 0; b < B; ++b) acc[r][b] = make_float2(0.0f, 0.0f);
+  int c_seg = cur.c;  // first chunk of the current row segment
+  uint32_t cur_slot = ring;
 
-  auto process = [&](const uint32_t (&cw)[R][NW]) {
-    if (cur.c != xc) {  // entering a new chunk: take its x, fetch the next
-      xc = cur.c;
-      k_ok = lane_in_k(xc);
+  for (int u = u_begin; u < u_end; ++u) {
+    issue();                 // unit u + D - 1
+    cp_async_wait<D - 1>();  // unit u has landed
+    uint32_t cw[R][NW];
 #pragma unroll
-      for (int b = 0; b < B; ++b)
-#pragma unroll
-        for (int q = 0; q < NX; ++q)
-          xv[b][q] = make_float2(__uint_as_float(xr[b][q] << 16),
-                                 __uint_as_float(xr[b][q] & 0xFFFF0000u));
-      load_x(xc + 1);
+    for (int r = 0; r < R; ++r) {
+      const uint4 v = lds_v4(cur_slot + r * kRowBytes + lane16);
+      cw[r][0] = v.x; cw[r][1] = v.y; cw[r][2] = v.z; cw[r][3] = v.w;
     }
-    float2 acc[R][B];
+    cur_slot = cur_slot + kSlot == ring_end ? ring : cur_slot + kSlot;
+
+    float2 xv[B][NX];
 #pragma unroll
-    for (int r = 0; r < R; ++r)
+    for (int b = 0; b < B; ++b)
 #pragma unroll
-      for (int b = 0; b < B; ++b) acc[r][b] = make_float2(0.0f, 0.0f);
-    if (k_ok) {
+      for (int q = 0; q < NX; ++q)
+        xv[b][q] = make_float2(__uint_as_float(xw[b][q] << 16),
+                               __uint_as_float(xw[b][q] & 0xFFFF0000u));
+    if (u + 1 < u_end) load_x(cur.c + 1 == nchunks ? 0 : cur.c + 1);
+
+    if (cur.c + 1 < nchunks || last_ok) {
 #pragma unroll
       for (int r = 0; r < R; ++r)
 #pragma unroll
@@ -254,74 +314,88 @@ __global__ void __launch_bounds__(NT, 1)
               acc[r][b] = __ffma2_rn(wv, xv[b][2 * q + h], acc[r][b]);
           }
     }
-    float v[M];
-#pragma unroll
-    for (int r = 0; r < R; ++r)
-#pragma unroll
-      for (int b = 0; b < B; ++b) v[r * B + b] = acc[r][b].x + acc[r][b].y;
-#pragma unroll
-    for (int q = R * B; q < M; ++q) v[q] = 0.0f;
-    const float s = butterfly_reduce<M>(v, lane);
-    constexpr int kLow = 32 / M;  // lanes holding the same reduced value
-    const int idx = lane / kLow;
-    if ((lane % kLow) == 0 && idx < R * B) {
-      const int r = idx / B, b = idx - (idx / B) * B;
-      const int row = cur.g * R + r;
-      if (row < rows)
-        sts_f32(kRedAddr + (uint32_t)(((cur.c * rows_max + row) * B + b) * 4),
-                s);
-    }
-    advance(cur);
-  };
 
-  for (int u = u_begin; u < u_end; u += D) {
+    if (u + 1 == u_end || cur.c + 1 == nchunks) {
+      // End of a row segment: reduce across lanes and store the sums in the
+      // slot of the segment's first chunk (distinct for every warp touching
+      // the rows).
+      float v[M];
 #pragma unroll
-    for (int d = 0; d < D; ++d) {
-      if (u + d < u_end) {
-        process(cw[d]);
-        issue(cw[d]);  // unit u + d + D
+      for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int b = 0; b < B; ++b) {
+          v[r * B + b] = acc[r][b].x + acc[r][b].y;
+          acc[r][b] = make_float2(0.0f, 0.0f);
+        }
+#pragma unroll
+      for (int q = R * B; q < M; ++q) v[q] = 0.0f;
+      const float s = butterfly_reduce<M>(v, lane);
+      constexpr int kLow = 32 / M;  // lanes holding the same reduced value
+      const int idx = lane / kLow;
+      if ((lane % kLow) == 0 && idx < R * B) {
+        const int r = idx / B, b = idx - (idx / B) * B;
+        const int row = cur.g * R + r;
+        if (row < rows)
+          sts_f32(
+              kRedAddr + (uint32_t)(((c_seg * rows_max + row) * B + b) * 4),
+              s);
       }
+      c_seg = 0;  // the next unit starts a row group at chunk 0
     }
+    advance(cur, nchunks);
   }
+  cp_async_wait<0>();
   __syncthreads();
 
-  for (int i = threadIdx.x; i < rows * B; i += NT) {
-    const int r = i / B, b = i - r * B;
+  // Sum each row's chunk slots in a fixed order: lane-strided, then across
+  // the warp.
+  for (int o = warp; o < rows * B; o += kWarps) {
+    const int r = o / B, b = o - r * B;
     float s = 0.0f;
-    for (int c = 0; c < nchunks; ++c)
-      s += lds_f32(kRedAddr + (uint32_t)(((c * rows_max + r) * B + b) * 4));
-    const int64_t row = row_lo + r;
-    const float scale =
-        rho ? __half2float(__ushort_as_half(rho[row / rps])) : 1.0f;
-    y[(int64_t)b * ldy + row] = scale * s;
+    for (int c = lane; c < nchunks; c += 32)
+      s += lds_f32_volatile(
+          kRedAddr + (uint32_t)(((c * rows_max + r) * B + b) * 4));
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, m);
+    if (lane == 0) {
+      const int64_t row = row_lo + r;
+      const float scale =
+          rho ? __half2float(__ushort_as_half(rho[row / rps])) : 1.0f;
+      y[(int64_t)b * ldy + row] = scale * s;
+    }
   }
 }
 
-// Tile parameters of one launch.
-struct GemvCfg {
-  int kpl, r, d, nt;
-};
-
-template <int B, int KPL, int R, int D, int NT>
+template <int B, int R, int D, int NT>
 cudaError_t launch_cfg(const WeightsView &w, const __nv_bfloat16 *x,
                        int64_t ldx, float *y, int64_t ldy, int sms,
                        cudaStream_t stream) {
-  constexpr int KC = 32 * KPL;
+  constexpr int kWarps = NT / 32;
+  constexpr uint32_t kRing = D * R * kRowBytes;
+  // Rings that fit below the code book even with the window at kRingLoAddr;
+  // the others go above the partial sums.
+  constexpr int lo_min = (int)((kLutAddr - kRingLoAddr) / kRing);
+  constexpr int hi_warps = kWarps > lo_min ? kWarps - lo_min : 0;
   const int64_t nchunks = (w.k + KC - 1) / KC;
   int64_t ctas = sms < w.n ? sms : w.n;
   // the partial sums (one slot per chunk, row and batch row) must fit
-  const int64_t rows_cap = kRedMaxBytes / (nchunks * B * 4);
+  // between the code book and the upper rings
+  const int64_t red_max =
+      (int64_t)kSmemMax - kRedAddr - (int64_t)hi_warps * kRing - 128;
+  const int64_t rows_cap = red_max / (nchunks * B * 4);
   if (rows_cap < 1) return cudaErrorInvalidValue;
   if ((w.n + ctas - 1) / ctas > rows_cap) ctas = (w.n + rows_cap - 1) / rows_cap;
   const int rows_max = (int)((w.n + ctas - 1) / ctas);
-  const size_t smem = kRedAddr + (size_t)nchunks * rows_max * B * 4;
-  auto kern = gemv_b_kernel<B, KPL, R, D, NT>;
+  const uint32_t red_bytes = (uint32_t)(nchunks * rows_max * B * 4);
+  const uint32_t hi_ring = (kRedAddr + red_bytes + 127u) & ~127u;
+  const size_t smem = hi_ring + (size_t)hi_warps * kRing;
+  auto kern = gemv_b_kernel<B, R, D, NT>;
   cudaError_t e = cudaFuncSetAttribute(
       kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   kern<<<(unsigned)ctas, NT, smem, stream>>>(w.codes, w.n, w.k, w.lut,
                                               w.scales, w.rps, x, ldx, y, ldy,
-                                              rows_max);
+                                              rows_max, hi_ring);
   return cudaGetLastError();
 }
 
@@ -330,20 +404,6 @@ int device_sms() {
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   return sms;
-}
-
-// Row-group height for a shape: the largest R whose units still split
-// evenly over the warps (at most ~12 % lost to the last partial unit).
-int pick_rows(int64_t n, int64_t k, int kpl, int warps, int sms) {
-  const int64_t nchunks = (k + 32 * kpl - 1) / (32 * kpl);
-  const int64_t rows = (n + sms - 1) / sms;
-  for (int r = 4; r >= 2; r /= 2) {
-    const int64_t units = (rows + r - 1) / r * nchunks;
-    const int64_t per_warp = (units + warps - 1) / warps;
-    const double eff = (double)rows * nchunks / ((double)per_warp * warps * r);
-    if (eff >= 0.88) return r;
-  }
-  return 2;
 }
 
 }  // namespace
@@ -356,16 +416,10 @@ cudaError_t gemv_b(const WeightsView &w, const __nv_bfloat16 *x, int64_t batch,
                    int64_t ldx, float *y, int64_t ldy, cudaStream_t stream) {
   const int sms = device_sms();
   switch (batch) {
-    case 1:
-      if (pick_rows(w.n, w.k, 16, 16, sms) == 4)
-        return launch_cfg<1, 16, 4, 2, 512>(w, x, ldx, y, ldy, sms, stream);
-      return launch_cfg<1, 16, 2, 3, 512>(w, x, ldx, y, ldy, sms, stream);
-    case 2:
-      return launch_cfg<2, 16, 2, 2, 512>(w, x, ldx, y, ldy, sms, stream);
-    case 3:
-      return launch_cfg<3, 8, 2, 3, 512>(w, x, ldx, y, ldy, sms, stream);
-    default:
-      return launch_cfg<4, 8, 2, 3, 512>(w, x, ldx, y, ldy, sms, stream);
+    case 1: return launch_cfg<1, 4, 3, 768>(w, x, ldx, y, ldy, sms, stream);
+    case 2: return launch_cfg<2, 4, 4, 512>(w, x, ldx, y, ldy, sms, stream);
+    case 3: return launch_cfg<3, 2, 4, 512>(w, x, ldx, y, ldy, sms, stream);
+    default: return launch_cfg<4, 2, 4, 512>(w, x, ldx, y, ldy, sms, stream);
   }
 }
 
