@@ -8,6 +8,7 @@ cudaError_t launch_linear(const WeightsView &w, const __nv_bfloat16 *x,
                           cudaStream_t stream) {
   if (gemv_b_supported(w, batch))
     return gemv_b(w, x, batch, ldx, y, ldy, stream);
+  if (gemv_a_supported(w, batch)) return gemv_a(w, x, y, stream);
   const int64_t tc_min_batch = w.format == TQ_FMT_B ? 5 : 2;
   if (batch >= tc_min_batch && gemm_tc_supported(w, batch))
     return gemm_tc(w, x, batch, ldx, y, ldy, stream);

@@ -15,6 +15,12 @@ bool gemv_b_supported(const WeightsView &w, int64_t batch);
 cudaError_t gemv_b(const WeightsView &w, const __nv_bfloat16 *x, int64_t batch,
                    int64_t ldx, float *y, int64_t ldy, cudaStream_t stream);
 
+// Format A, batch 1, G = 64: activation tables (243 partial sums of x per
+// code byte position), one table load per code byte.
+bool gemv_a_supported(const WeightsView &w, int64_t batch);
+cudaError_t gemv_a(const WeightsView &w, const __nv_bfloat16 *x, float *y,
+                   cudaStream_t stream);
+
 // Batches that are a real contraction: tcgen05 MMAs on decoded bf16 hi/lo
 // operands, accumulator in tensor memory.
 bool gemm_tc_supported(const WeightsView &w, int64_t batch);
