@@ -55,21 +55,28 @@ def peaks():
 # ---- distributed plumbing (replicas only) -------------------------------------
 
 def dist_setup():
+    """One process per GPU (torchrun env). NCCL when there is a GPU; gloo on a
+    host without one (the reference arm and the CPU tests of this path)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
-        torch.distributed.init_process_group(
-            "nccl", timeout=datetime.timedelta(seconds=120),
-            device_id=torch.device("cuda", local))
+        timeout = datetime.timedelta(seconds=120)
+        if torch.cuda.is_available():
+            torch.distributed.init_process_group(
+                "nccl", timeout=timeout, device_id=torch.device("cuda", local))
+        else:
+            torch.distributed.init_process_group("gloo", timeout=timeout)
     return world, rank, local
 
 
 def dist_max(v: float, world: int) -> float:
+    """Max of v over the ranks (the slowest rank's time)."""
     if world == 1:
         return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
 
@@ -185,7 +192,7 @@ class Workload:
     """A workload: device inputs, the graphs of one step, the host copies of
     the end-to-end leg and the oracle sample of the CPU legs."""
     name = ""
-    SOURCES = ("tq_linear.cu", "tq_gemv_b.cu", "tq_gemm_tc.cu",
+    SOURCES = ("tq_linear.cu", "tq_gemv_a.cu", "tq_gemv_b.cu", "tq_gemm_tc.cu",
                "tq_linear_simple.cu")
 
     def h2d(self):
@@ -587,7 +594,7 @@ def run_reference(args, world, rank):
     t0 = time.perf_counter()
     wl.oracle_pass(16)
     per_row = (time.perf_counter() - t0) / 16
-    budget = 90.0 / max(1, args.steps + args.warmup)
+    budget = args.ref_seconds / max(1, args.steps + args.warmup)
     rows = int(max(1, min(wl.MAX_ROWS, budget / max(per_row, 1e-9))))
     for _ in range(args.warmup):
         wl.oracle_pass(rows)
@@ -728,6 +735,8 @@ def main():
                     help="batch of the decode_step workload")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-seconds", type=float, default=90.0,
+                    help="host time the reference arm spends in total")
     args = ap.parse_args()
     world, rank, local = dist_setup()
     try:
