@@ -6,24 +6,28 @@
 //   Format B: y[b][n] = rho[n / rps] * sum_k LUT[code[n][k]] x[b][k]
 //             (alphaneural.io page, sections 3.2, 3.3 and 4.2)
 //
-// One CTA computes a 128-row tile of y^T over the whole of K for N = batch
-// rounded up to 16 (<= 64), accumulating in tensor memory (128 lanes x N
-// fp32 columns). Per 64-wide K block (and per plane):
-//   - 8 decoder warps (two per TMEM lane quarter) turn the codes of their
-//     rows into bf16 operands, written straight into shared memory in the
-//     K-major canonical layout, and stage the x tile beside them. Each weight
-//     w is split into w_hi = bf16(w) and w_lo = bf16(w - w_hi): two MMAs
-//     (hi, then lo) give products exact to ~2^-16 relative, well inside the
-//     2e-3 tolerance, with bf16 x used as is. For Format A, s*t splits
-//     exactly (an fp16 scale has 11 significant bits: 8 in s_hi, 3 in s_lo).
-//   - One thread issues the 2 x 4 MMAs (M=128, N, K=16) of the block and
-//     commits them to the stage's mbarrier, which frees the stage for the
-//     decoders. The codes are never written out as a bf16 matrix.
+// One CTA computes a 128-row tile of y^T over the whole of K (or a cluster
+// slice of it) for N = batch rounded up to 16 (<= 64), accumulating in tensor
+// memory (128 lanes x N fp32 columns). Per 64-wide K block (and per plane):
+//   - 8 decoder warps (two per TMEM lane quarter; a thread owns one row and
+//     half of the block's k) turn the codes of their rows into bf16 operands
+//     and write them straight into tensor memory with tcgen05.st: the A
+//     operand never passes through shared memory, whose bandwidth then only
+//     carries the code-book lookups. Each weight w is split into
+//     w_hi = bf16(w) and w_lo = bf16(w - w_hi): two MMAs (hi, then lo) give
+//     products exact to ~2^-16 relative, well inside the 2e-3 tolerance, with
+//     bf16 x used as is. For Format A, s*t splits exactly (an fp16 scale has
+//     11 significant bits: 8 in s_hi, 3 in s_lo). The x tile is staged in
+//     shared memory (operand B, K-major canonical layout).
+//   - One thread issues the 2 x 4 MMAs (M=128, N, K=16; A from tensor
+//     memory, B from shared memory) of the block and commits them to the
+//     stage's mbarrier, which frees the stage for the decoders. Tensor memory
+//     holds the accumulator and 6 A stages of 64 columns (32 hi + 32 lo).
 //   - After the last block the accumulator is read back with tcgen05.ld,
 //     rho applied (Format B) and y stored.
 // Waits are bounded; on a time-out the CTA writes NaN to its outputs, gives
 // in-flight MMAs a bounded chance to finish, frees its tensor memory and
-// exits.
+// exits. Decisions in front of warp-wide tcgen05 instructions are uniform.
 #include <cooperative_groups.h>
 
 #include "tq_common.cuh"
@@ -38,10 +42,11 @@ constexpr int kTileM = 128;
 constexpr int kBlockK = 64;                       // k per stage
 constexpr int kDecoderWarps = 8;
 constexpr int kThreads = 32 * (1 + kDecoderWarps);
-constexpr int kStages = 3;
+constexpr int kStages = 6;                        // A in TMEM, x in smem
 constexpr int kCodeDepth = 6;                     // code blocks per thread ring
-constexpr int kSubTileA = kTileM * 32;            // one k16 step of A: 4 KB
-constexpr int kATile = 4 * kSubTileA;             // 64 k of A (hi or lo): 16 KB
+constexpr uint32_t kTmemCols = 512;               // the whole tensor memory
+constexpr uint32_t kAccCols = 64;                 // accumulator: N <= 64
+constexpr uint32_t kStageCols = 64;               // A stage: 32 hi + 32 lo
 constexpr int kLutStride = 128;                   // 32 lane copies x 4 B
 constexpr int kLutBytes = 256 * kLutStride;       // 32 KB
 constexpr int kMaxN = 64;
@@ -57,7 +62,7 @@ __device__ __forceinline__ uint32_t tile_off(int r, int k, int rows) {
 struct TcParams {
   int ks_count;     // CTAs per cluster, each taking a slice of K
   int n_pad;        // N of the MMA (batch rounded up to 16)
-  int stage_bytes;  // A hi + A lo + x tile
+  int stage_bytes;  // x tile
   int x_off;        // x tile offset inside a stage
   int ring_off, lut_off, bar_off, tmem_slot_off;
   int code_off, code_slot;  // code ring: kCodeDepth slots of 128 rows x 64 B
@@ -174,7 +179,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(acc_bar, 1);
     mbar_init_fence();
   }
-  if (warp == 0) tmem_alloc(sbase + P.tmem_slot_off, 64);
+  if (warp == 0) tmem_alloc(sbase + P.tmem_slot_off, kTmemCols);
   // Lookup tables.
   if constexpr (FMT == TQ_FMT_B) {
     // entry e, lane copy l at e*128 + 4*l: bf16(w) | bf16(w - bf16(w)) << 16
@@ -224,15 +229,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after_sync();
         const uint32_t st = ring + s * P.stage_bytes;
+        const uint32_t a_st = tmem + kAccCols + (uint32_t)s * kStageCols;
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
-          const uint64_t ah = smem_desc_kmajor(st + ks * kSubTileA, 128, 256);
-          const uint64_t al =
-              smem_desc_kmajor(st + kATile + ks * kSubTileA, 128, 256);
           const uint64_t bx =
               smem_desc_kmajor(st + P.x_off + ks * N * 32, 128, 256);
-          mma_bf16(tmem, ah, bx, idesc, (it > 0 || ks > 0) ? 1u : 0u);
-          mma_bf16(tmem, al, bx, idesc, 1u);
+          // k16 step ks: 8 columns of the hi half, then of the lo half
+          mma_bf16_ts(tmem, a_st + 8 * ks, bx, idesc,
+                      (it > 0 || ks > 0) ? 1u : 0u);
+          mma_bf16_ts(tmem, a_st + 32 + 8 * ks, bx, idesc, 1u);
         }
         mma_commit(empty0 + 8 * s);  // frees the stage when these finish
       }
@@ -312,10 +317,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint4 xr0[2], xr1[2];
     load_x(0, xr0);
     load_x(1, xr1);
-    for (int it = 0; it < iters && !abort_flag; ++it) {
+    // Every decision before a warp-wide (.sync.aligned) instruction is made
+    // uniform across the warp.
+    for (int it = 0; it < iters && !__any_sync(0xFFFFFFFFu, abort_flag != 0);
+         ++it) {
       const int s = it % kStages;
       const int kb = (it_begin + it) % kblocks;
-      const int64_t k0 = (int64_t)kb * kBlockK;
       sc[kCodeDepth - 1] = issue(it + kCodeDepth - 1);
       cp_async_commit();
       cp_async_wait<kCodeDepth - 1>();  // this block's codes have landed
@@ -365,25 +372,38 @@ __global__ void __launch_bounds__(kThreads, 1)
           s_lo = bf16_bits_rn(sf - __uint_as_float(s_hi << 16));
         }
       }
-      if (it >= kStages &&
-          !mbar_wait(empty0 + 8 * s, ((it / kStages) - 1) & 1)) {
-        abort_flag = 1;
-        break;
-      }
-      uint8_t *st = smem + P.ring_off + s * P.stage_bytes;
+      // decode this thread's 32 k of its row: 16 hi and 16 lo bf16 pairs
+      uint32_t hi[16], lo[16];
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
         const int c = 4 * h + cc;  // 8-k chunk of the block
-        uint32_t hi[4], lo[4];
+        uint32_t h4[4], l4[4];
         if constexpr (FMT == TQ_FMT_B)
-          decode8_b(cw[2 * cc], cw[2 * cc + 1], lut_base, lane8, hi, lo);
+          decode8_b(cw[2 * cc], cw[2 * cc + 1], lut_base, lane8, h4, l4);
         else
-          decode8_a(nz, neg, c, s_hi, s_lo, hi, lo);
-        const uint32_t off = tile_off(r, 8 * c, kTileM);
-        *reinterpret_cast<uint4 *>(st + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4 *>(st + kATile + off) =
-            make_uint4(lo[0], lo[1], lo[2], lo[3]);
+          decode8_a(nz, neg, c, s_hi, s_lo, h4, l4);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          hi[4 * cc + q] = h4[q];
+          lo[4 * cc + q] = l4[q];
+        }
       }
+      if (it >= kStages) {
+        const bool ok = mbar_wait(empty0 + 8 * s, ((it / kStages) - 1) & 1);
+        if (!__all_sync(0xFFFFFFFFu, ok)) {
+          abort_flag = 1;
+          break;
+        }
+      }
+      tc_fence_after_sync();  // the stage's MMAs are done reading it
+      {
+        const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + kAccCols +
+                            (uint32_t)s * kStageCols + 16u * (uint32_t)h;
+        tmem_st16(ta, hi);
+        tmem_st16(ta + 32, lo);
+        tmem_st_wait();
+      }
+      uint8_t *st = smem + P.ring_off + s * P.stage_bytes;
       // x tile: N rows x 64 k, 16 bytes per chunk (fetched two blocks ahead)
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
@@ -394,7 +414,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         xr0[q] = xr1[q];
       }
       load_x(it + 2, xr1);
-      fence_async_shared();
+      fence_async_shared();   // x tile -> async proxy (MMA operand B)
+      tc_fence_before_sync();  // A stores -> ordered before the arrive
       __syncwarp();
       if (lane == 0) mbar_arrive(full0 + 8 * s);
     }
@@ -457,7 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (warp == 0) {
     tc_fence_after_sync();
-    tmem_dealloc(tmem, 64);
+    tmem_dealloc(tmem, kTmemCols);
   }
 }
 
@@ -465,8 +486,8 @@ TcParams plan_tc(int fmt, int64_t batch) {
   TcParams P{};
   const int64_t b = batch < kMaxN ? batch : kMaxN;
   P.n_pad = (int)((b + 15) / 16 * 16);
-  P.stage_bytes = 2 * kATile + P.n_pad * kBlockK * 2;
-  P.x_off = 2 * kATile;
+  P.stage_bytes = P.n_pad * kBlockK * 2;
+  P.x_off = 0;
   P.ring_off = 0;
   P.code_slot = kTileM * 64;
   P.code_off = kStages * P.stage_bytes;
@@ -475,6 +496,8 @@ TcParams plan_tc(int fmt, int64_t batch) {
   P.bar_off = P.lut_off + table;
   P.tmem_slot_off = P.bar_off + (2 * kStages + 1) * 8 + 8;
   P.smem = (size_t)P.tmem_slot_off + 16;
+  // one CTA per SM: each allocates the whole tensor memory
+  if (P.smem < 120 * 1024) P.smem = 120 * 1024;
   return P;
 }
 
