@@ -39,9 +39,21 @@ namespace tq {
 namespace {
 
 constexpr int kTileM = 128;
+constexpr int kMaxN = 64;
 constexpr int kBlockK = 64;                       // k per stage
-constexpr int kDecoderWarps = 8;
-constexpr int kThreads = 32 * (1 + kDecoderWarps);
+// Decoder warps per CTA (a multiple of 4: the TMEM lane quarters). Format B
+// decodes are short (a lookup per weight), so 16 warps, 16 k per thread, keep
+// more loads in flight; a Format A thread rebuilds its group's trit masks,
+// so 8 warps (32 k per thread) share that work better.
+template <int FMT>
+struct TcCfg {
+  static constexpr int kDecoderWarps = FMT == TQ_FMT_B ? 16 : 8;
+  static constexpr int kKParts = kDecoderWarps / 4;  // k parts of a block
+  static constexpr int kKPT = kBlockK / kKParts;     // k per decoder thread
+  static constexpr int kXPerThread =
+      (kMaxN * 8 + kDecoderWarps * 32 - 1) / (kDecoderWarps * 32);
+  static constexpr int kThreads = 32 * (1 + kDecoderWarps);
+};
 constexpr int kStages = 6;                        // A in TMEM, x in smem
 constexpr int kCodeDepth = 6;                     // code blocks per thread ring
 constexpr uint32_t kTmemCols = 512;               // the whole tensor memory
@@ -49,7 +61,6 @@ constexpr uint32_t kAccCols = 64;                 // accumulator: N <= 64
 constexpr uint32_t kStageCols = 64;               // A stage: 32 hi + 32 lo
 constexpr int kLutStride = 128;                   // 32 lane copies x 4 B
 constexpr int kLutBytes = 256 * kLutStride;       // 32 KB
-constexpr int kMaxN = 64;
 
 // Offset of element (row r, k in [0,64)) inside an A (or x) K-block tile:
 // four k16 sub-tiles of rows*32 bytes, each in the canonical K-major layout
@@ -90,6 +101,18 @@ __device__ __forceinline__ void cp_async_commit() {
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Warp-wide store of N (8 or 16) consecutive TMEM columns.
+template <int N>
+__device__ __forceinline__ void tmem_st_cols(uint32_t ta,
+                                             const uint32_t (&v)[N]) {
+  if constexpr (N == 16) {
+    tmem_st16(ta, v);
+  } else {
+    static_assert(N == 8, "8 or 16 columns");
+    tmem_st8(ta, v);
+  }
 }
 
 __device__ __forceinline__ uint32_t bf16_bits_rn(float v) {
@@ -142,10 +165,13 @@ __device__ __forceinline__ void decode8_a(uint64_t nz, uint64_t neg, int c,
 }
 
 template <int FMT>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(TcCfg<FMT>::kThreads, 1)
     gemm_tc_kernel(WeightsView w, const __nv_bfloat16 *__restrict__ x,
                    int64_t batch, int64_t ldx, float *__restrict__ y,
                    int64_t ldy, TcParams P) {
+  constexpr int kDecoderWarps = TcCfg<FMT>::kDecoderWarps;
+  constexpr int kKPT = TcCfg<FMT>::kKPT;
+  constexpr int kXPerThread = TcCfg<FMT>::kXPerThread;
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
   const uint32_t ring = sbase + P.ring_off;
@@ -247,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- decoders ----
     const int wid = warp - 1;
     const int quarter = warp & 3;  // TMEM lanes this warp may access
-    const int h = wid >> 2;        // which half of the 64 k of a block
+    const int kp = wid >> 2;       // which part of the 64 k of a block
     const int r = quarter * 32 + lane;
     const int64_t grow = row0 + r;
     const bool row_ok = grow < w.n;
@@ -259,7 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // memory with cp.async (each thread reads back only the bytes its own
     // copies wrote), so kCodeDepth - 1 blocks of every row are in flight.
     const int64_t plane_bytes = w.n * gpr * 13;  // Format A code bytes per plane
-    const uint32_t code_ring = sbase + P.code_off + r * 64 + h * 32;
+    const uint32_t code_ring = sbase + P.code_off + r * 64 + kp * kKPT;
     uint32_t sc[kCodeDepth];                      // Format A scales, in order
 #pragma unroll
     for (int q = 0; q < kCodeDepth; ++q) sc[q] = 0;
@@ -269,11 +295,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int gi_it = it_begin + it;
       const int plane = gi_it / kblocks, kb = gi_it - plane * kblocks;
       if constexpr (FMT == TQ_FMT_B) {
-        const int64_t kk = (int64_t)kb * kBlockK + 32 * h;
+        const int64_t kk = (int64_t)kb * kBlockK + kKPT * kp;
         const uint8_t *p = w.codes + (row_ok ? grow : 0) * K + kk;
-        cp_async16(dst, row_ok && kk < K ? p : w.codes, row_ok && kk < K ? 16 : 0);
-        cp_async16(dst + 16, row_ok && kk + 16 < K ? p + 16 : w.codes,
-                   row_ok && kk + 16 < K ? 16 : 0);
+#pragma unroll
+        for (int j = 0; j < kKPT / 16; ++j) {
+          const bool ok = row_ok && kk + 16 * j < K;
+          cp_async16(dst + 16 * j, ok ? p + 16 * j : w.codes, ok ? 16 : 0);
+        }
         return 0;
       } else {
         if (!row_ok) return 0;
@@ -302,9 +330,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // This thread's (at most two) 16-byte x chunks of block it; zero past
     // the batch, past K and past the slice.
-    auto load_x = [&](int it, uint4 (&v)[2]) {
+    auto load_x = [&](int it, uint4 (&v)[kXPerThread]) {
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
+      for (int q = 0; q < kXPerThread; ++q) {
         v[q] = make_uint4(0, 0, 0, 0);
         const int id = wid * 32 + lane + q * kDecoderWarps * 32;
         const int n = id >> 3, c = id & 7;
@@ -314,7 +342,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     };
-    uint4 xr0[2], xr1[2];
+    uint4 xr0[kXPerThread], xr1[kXPerThread];
     load_x(0, xr0);
     load_x(1, xr1);
     // Every decision before a warp-wide (.sync.aligned) instruction is made
@@ -327,21 +355,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       cp_async_commit();
       cp_async_wait<kCodeDepth - 1>();  // this block's codes have landed
       const uint32_t src = code_ring + (uint32_t)(it % kCodeDepth) * P.code_slot;
-      uint32_t cw[8];
-      {
-        uint4 a, b2;
+      uint32_t cw[kKPT / 4 > 4 ? kKPT / 4 : 4];
+#pragma unroll
+      for (int j = 0; j < (kKPT / 16 > 1 ? kKPT / 16 : 1); ++j) {
+        uint4 a;
         asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
-                     : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w) : "r"(src));
-        asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
-                     : "=r"(b2.x), "=r"(b2.y), "=r"(b2.z), "=r"(b2.w)
-                     : "r"(src + 16));
-        cw[0] = a.x; cw[1] = a.y; cw[2] = a.z; cw[3] = a.w;
-        cw[4] = b2.x; cw[5] = b2.y; cw[6] = b2.z; cw[7] = b2.w;
+                     : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w)
+                     : "r"(src + 16 * j));
+        cw[4 * j] = a.x; cw[4 * j + 1] = a.y; cw[4 * j + 2] = a.z;
+        cw[4 * j + 3] = a.w;
       }
       if constexpr (FMT == TQ_FMT_B) {
         if (!row_ok) {
 #pragma unroll
-          for (int q = 0; q < 8; ++q) cw[q] = 0x79797979u;  // weight 0
+          for (int q = 0; q < kKPT / 4; ++q) cw[q] = 0x79797979u;  // weight 0
         }
       }
       const uint32_t cur_scale = sc[0];
@@ -361,22 +388,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             v[q] = __funnelshift_r(cw[q], q < 3 ? cw[q + 1] : 0u, sh);
           const uint16_t *tab =
               reinterpret_cast<const uint16_t *>(smem + P.lut_off);
+          // only the bytes that hold this thread's kKPT trits
+          constexpr int kBytes = (kKPT + 8) / 5;  // bytes any kKPT-window spans
+          const int m_lo = (kKPT * kp) / 5;
 #pragma unroll
-          for (int m = 0; m < 13; ++m) {
-            const uint32_t e = tab[(v[m >> 2] >> (8 * (m & 3))) & 0xFFu];
-            nz |= (uint64_t)(e & 31u) << (5 * m);
-            neg |= (uint64_t)((e >> 5) & 31u) << (5 * m);
+          for (int j = 0; j < kBytes; ++j) {
+            const int m = m_lo + j;
+            if (m < 13) {
+              const int wi = m >> 2;  // selected without indexing (no stack)
+              const uint32_t wv = wi == 0 ? v[0] : wi == 1 ? v[1] : wi == 2 ? v[2] : v[3];
+              const uint32_t e = tab[(wv >> (8 * (m & 3))) & 0xFFu];
+              nz |= (uint64_t)(e & 31u) << (5 * m);
+              neg |= (uint64_t)((e >> 5) & 31u) << (5 * m);
+            }
           }
           const float sf = __half2float(__ushort_as_half((uint16_t)cur_scale));
           s_hi = bf16_bits_rn(sf);
           s_lo = bf16_bits_rn(sf - __uint_as_float(s_hi << 16));
         }
       }
-      // decode this thread's 32 k of its row: 16 hi and 16 lo bf16 pairs
-      uint32_t hi[16], lo[16];
+      // decode this thread's kKPT k of its row: kKPT/2 hi and lo bf16 pairs
+      uint32_t hi[kKPT / 2], lo[kKPT / 2];
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        const int c = 4 * h + cc;  // 8-k chunk of the block
+      for (int cc = 0; cc < kKPT / 8; ++cc) {
+        const int c = (kKPT / 8) * kp + cc;  // 8-k chunk of the block
         uint32_t h4[4], l4[4];
         if constexpr (FMT == TQ_FMT_B)
           decode8_b(cw[2 * cc], cw[2 * cc + 1], lut_base, lane8, h4, l4);
@@ -398,15 +433,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after_sync();  // the stage's MMAs are done reading it
       {
         const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + kAccCols +
-                            (uint32_t)s * kStageCols + 16u * (uint32_t)h;
-        tmem_st16(ta, hi);
-        tmem_st16(ta + 32, lo);
+                            (uint32_t)s * kStageCols +
+                            (uint32_t)(kKPT / 2) * (uint32_t)kp;
+        tmem_st_cols(ta, hi);
+        tmem_st_cols(ta + 32, lo);
         tmem_st_wait();
       }
       uint8_t *st = smem + P.ring_off + s * P.stage_bytes;
       // x tile: N rows x 64 k, 16 bytes per chunk (fetched two blocks ahead)
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
+      for (int q = 0; q < kXPerThread; ++q) {
         const int id = wid * 32 + lane + q * kDecoderWarps * 32;
         if (id < N * 8)
           *reinterpret_cast<uint4 *>(st + P.x_off +
@@ -421,7 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     cp_async_wait<0>();
     // ---- epilogue: warps of the first half read their TMEM lane quarter ----
-    if (h == 0) {
+    if (kp == 0) {
       const bool ok = iters == 0 || mbar_wait(acc_bar, 0);
       if (!ok) abort_flag = 1;
       tc_fence_after_sync();
@@ -536,7 +572,7 @@ cudaError_t launch_tc(const WeightsView &w, const __nv_bfloat16 *x,
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(tiles * P.ks_count), 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(TcCfg<FMT>::kThreads, 1, 1);
   cfg.dynamicSmemBytes = P.smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
