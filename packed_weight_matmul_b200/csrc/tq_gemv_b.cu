@@ -145,8 +145,19 @@ __device__ __forceinline__ void advance(UnitPos &q, int nchunks) {
   }
 }
 
+__device__ __forceinline__ void advance_cm(UnitPos &q, int ng) {
+  if (++q.g == ng) {
+    q.g = 0;
+    ++q.c;
+  }
+}
+
 // hi_ring: shared-window address of the rings placed above the partial sums.
-template <int B, int R, int D, int NT>
+// CM (chunk-major): units ordered chunk first, so a warp keeps one chunk's x
+// (converted once) in registers across the row groups it walks and reduces
+// every unit; used for 3-4 batch rows, where converting x per unit would cost
+// more than the reductions. Otherwise row-group major with row segments.
+template <int B, int R, int D, int NT, bool CM>
 __global__ void __launch_bounds__(NT, 1)
     gemv_b_kernel(const uint8_t *__restrict__ codes, int64_t n, int64_t k,
                   const float *__restrict__ lut,
@@ -186,7 +197,7 @@ __global__ void __launch_bounds__(NT, 1)
 
   const int ng = (rows + R - 1) / R;
   const int nchunks = (int)((k + KC - 1) / KC);
-  const int units = ng * nchunks;  // row-group major: u = g * nchunks + c
+  const int units = ng * nchunks;  // u = g * nchunks + c (CM: c * ng + g)
   const int u_begin = (int)((int64_t)units * warp / kWarps);
   const int u_end = (int)((int64_t)units * (warp + 1) / kWarps);
   const int64_t kstride = k;
@@ -197,8 +208,13 @@ __global__ void __launch_bounds__(NT, 1)
   const bool last_ok = (int64_t)(nchunks - 1) * KC + lane * KPL < k;
 
   UnitPos ld;  // next unit whose codes are copied
-  ld.g = u_begin / nchunks;
-  ld.c = u_begin - ld.g * nchunks;
+  if constexpr (CM) {
+    ld.c = u_begin / ng;
+    ld.g = u_begin - ld.c * ng;
+  } else {
+    ld.g = u_begin / nchunks;
+    ld.c = u_begin - ld.g * nchunks;
+  }
   const uint8_t *ld_p = crow + (int64_t)ld.g * group_step + (int64_t)ld.c * KC;
   int u_ld = u_begin;
   uint32_t ld_slot = ring;
@@ -225,8 +241,13 @@ __global__ void __launch_bounds__(NT, 1)
                      okr ? 16u : 0u);
         }
       }
-      advance(ld, nchunks);
-      ld_p = ld.c == 0 ? crow + (int64_t)ld.g * group_step : ld_p + KC;
+      if constexpr (CM) {
+        advance_cm(ld, ng);
+        ld_p = ld.g == 0 ? crow + (int64_t)ld.c * KC : ld_p + group_step;
+      } else {
+        advance(ld, nchunks);
+        ld_p = ld.c == 0 ? crow + (int64_t)ld.g * group_step : ld_p + KC;
+      }
     }
     cp_async_commit();
     ld_slot = ld_slot + kSlot == ring_end ? ring : ld_slot + kSlot;
@@ -255,7 +276,7 @@ __global__ void __launch_bounds__(NT, 1)
   // book while they fly.
 #pragma unroll
   for (int d = 0; d < D - 1; ++d) issue();
-  load_x(cur.c);
+  if constexpr (!CM) load_x(cur.c);
   const int red_words = nchunks * rows_max * B;
   for (int i = threadIdx.x; i < red_words; i += NT)
     sts_f32(kRedAddr + 4u * (uint32_t)i, 0.0f);
@@ -276,6 +297,8 @@ __global__ void __launch_bounds__(NT, 1)
     for (int b = 0; b < B; ++b) acc[r][b] = make_float2(0.0f, 0.0f);
   int c_seg = cur.c;  // first chunk of the current row segment
   uint32_t cur_slot = ring;
+  float2 xv[B][NX];  // x of the current chunk (CM: kept across units)
+  int xc = -1;       // chunk whose x is in xv (CM)
 
   for (int u = u_begin; u < u_end; ++u) {
     issue();                 // unit u + D - 1
@@ -288,14 +311,24 @@ __global__ void __launch_bounds__(NT, 1)
     }
     cur_slot = cur_slot + kSlot == ring_end ? ring : cur_slot + kSlot;
 
-    float2 xv[B][NX];
+    auto convert_x = [&]() {
 #pragma unroll
-    for (int b = 0; b < B; ++b)
+      for (int b = 0; b < B; ++b)
 #pragma unroll
-      for (int q = 0; q < NX; ++q)
-        xv[b][q] = make_float2(__uint_as_float(xw[b][q] << 16),
-                               __uint_as_float(xw[b][q] & 0xFFFF0000u));
-    if (u + 1 < u_end) load_x(cur.c + 1 == nchunks ? 0 : cur.c + 1);
+        for (int q = 0; q < NX; ++q)
+          xv[b][q] = make_float2(__uint_as_float(xw[b][q] << 16),
+                                 __uint_as_float(xw[b][q] & 0xFFFF0000u));
+    };
+    if constexpr (CM) {
+      if (cur.c != xc) {  // entering a chunk: fetch and convert its x once
+        xc = cur.c;
+        load_x(xc);
+        convert_x();
+      }
+    } else {
+      convert_x();
+      if (u + 1 < u_end) load_x(cur.c + 1 == nchunks ? 0 : cur.c + 1);
+    }
 
     if (cur.c + 1 < nchunks || last_ok) {
 #pragma unroll
@@ -315,7 +348,8 @@ __global__ void __launch_bounds__(NT, 1)
           }
     }
 
-    if (u + 1 == u_end || cur.c + 1 == nchunks) {
+    if (CM || u + 1 == u_end || cur.c + 1 == nchunks) {
+      if constexpr (CM) c_seg = cur.c;  // every unit is its own segment
       // End of a row segment: reduce across lanes and store the sums in the
       // slot of the segment's first chunk (distinct for every warp touching
       // the rows).
@@ -342,7 +376,11 @@ __global__ void __launch_bounds__(NT, 1)
       }
       c_seg = 0;  // the next unit starts a row group at chunk 0
     }
-    advance(cur, nchunks);
+    if constexpr (CM) {
+      advance_cm(cur, ng);
+    } else {
+      advance(cur, nchunks);
+    }
   }
   cp_async_wait<0>();
   __syncthreads();
@@ -366,7 +404,7 @@ __global__ void __launch_bounds__(NT, 1)
   }
 }
 
-template <int B, int R, int D, int NT>
+template <int B, int R, int D, int NT, bool CM = false>
 cudaError_t launch_cfg(const WeightsView &w, const __nv_bfloat16 *x,
                        int64_t ldx, float *y, int64_t ldy, int sms,
                        cudaStream_t stream) {
@@ -389,7 +427,7 @@ cudaError_t launch_cfg(const WeightsView &w, const __nv_bfloat16 *x,
   const uint32_t red_bytes = (uint32_t)(nchunks * rows_max * B * 4);
   const uint32_t hi_ring = (kRedAddr + red_bytes + 127u) & ~127u;
   const size_t smem = hi_ring + (size_t)hi_warps * kRing;
-  auto kern = gemv_b_kernel<B, R, D, NT>;
+  auto kern = gemv_b_kernel<B, R, D, NT, CM>;
   cudaError_t e = cudaFuncSetAttribute(
       kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -418,8 +456,8 @@ cudaError_t gemv_b(const WeightsView &w, const __nv_bfloat16 *x, int64_t batch,
   switch (batch) {
     case 1: return launch_cfg<1, 4, 3, 768>(w, x, ldx, y, ldy, sms, stream);
     case 2: return launch_cfg<2, 4, 4, 512>(w, x, ldx, y, ldy, sms, stream);
-    case 3: return launch_cfg<3, 2, 4, 512>(w, x, ldx, y, ldy, sms, stream);
-    default: return launch_cfg<4, 2, 4, 512>(w, x, ldx, y, ldy, sms, stream);
+    case 3: return launch_cfg<3, 2, 4, 512, true>(w, x, ldx, y, ldy, sms, stream);
+    default: return launch_cfg<4, 2, 4, 512, true>(w, x, ldx, y, ldy, sms, stream);
   }
 }
 
