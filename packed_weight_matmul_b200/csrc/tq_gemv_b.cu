@@ -155,8 +155,9 @@ __device__ __forceinline__ void advance_cm(UnitPos &q, int ng) {
 // hi_ring: shared-window address of the rings placed above the partial sums.
 // CM (chunk-major): units ordered chunk first, so a warp keeps one chunk's x
 // (converted once) in registers across the row groups it walks and reduces
-// every unit; used for 3-4 batch rows, where converting x per unit would cost
-// more than the reductions. Otherwise row-group major with row segments.
+// every unit (the dispatched order: converting x per unit costs more than the
+// reductions). Otherwise row-group major: sums stay in registers along a row
+// segment and are reduced once per segment.
 template <int B, int R, int D, int NT, bool CM>
 __global__ void __launch_bounds__(NT, 1)
     gemv_b_kernel(const uint8_t *__restrict__ codes, int64_t n, int64_t k,
@@ -454,8 +455,8 @@ cudaError_t gemv_b(const WeightsView &w, const __nv_bfloat16 *x, int64_t batch,
                    int64_t ldx, float *y, int64_t ldy, cudaStream_t stream) {
   const int sms = device_sms();
   switch (batch) {
-    case 1: return launch_cfg<1, 4, 3, 768>(w, x, ldx, y, ldy, sms, stream);
-    case 2: return launch_cfg<2, 4, 4, 512>(w, x, ldx, y, ldy, sms, stream);
+    case 1: return launch_cfg<1, 8, 2, 512, true>(w, x, ldx, y, ldy, sms, stream);
+    case 2: return launch_cfg<2, 4, 4, 512, true>(w, x, ldx, y, ldy, sms, stream);
     case 3: return launch_cfg<3, 2, 4, 512, true>(w, x, ldx, y, ldy, sms, stream);
     default: return launch_cfg<4, 2, 4, 512, true>(w, x, ldx, y, ldy, sms, stream);
   }
