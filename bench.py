@@ -152,7 +152,8 @@ def kernel_hash(files):
 
 def ncu_traffic(kernel_label, files, units):
     """dram bytes per launch from the committed ncu summary, or None when the
-    kernel source changed since the capture."""
+    sources the captured kernel is built from (the entry's "files", else the
+    workload's) changed since the capture."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
@@ -160,7 +161,7 @@ def ncu_traffic(kernel_label, files, units):
     except (OSError, ValueError):
         return None
     e = table.get(kernel_label)
-    if not e or e.get("source_hash") != kernel_hash(files):
+    if not e or e.get("source_hash") != kernel_hash(e.get("files", files)):
         return None
     return e["dram_bytes_per_unit"] * units
 

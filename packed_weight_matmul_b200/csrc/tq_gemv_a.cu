@@ -179,35 +179,54 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < kSteps; ++i) st_on[i] = lane_on && 2 * i + lg < gw;
     const bool sc_on = lane < gw;
 
-    for (int pl = 0; pl < w.planes; ++pl) {
+    // In a full window every lane loads unconditionally: lanes 26-31 read
+    // lane 0's byte (their table column is all zeros), lanes past the
+    // window's groups read the last group's scale (never used).
+    const bool full_win = gw == kWinGroups;
+    const int loff = lane < kLanes ? lane : 0;
+    const int soff = lane < gw ? lane : gw - 1;
+    for (int pl = 0; pl < w.planes && r_n > 0; ++pl) {
       // this lane's code byte of step 0 and its scale, row r_lo
-      const uint8_t *c0 = w.codes + pl * w.codes_plane_stride +
-                          ((row_lo + r_lo) * P.ng + w0) * kNB + lane;
-      const uint16_t *s0 = w.scales + pl * w.scales_plane_stride +
-                           (row_lo + r_lo) * P.ng + w0 + lane;
-      const uint8_t *ldc = c0, *pfc = c0;
-      const uint16_t *lds_ = s0, *pfs = s0;
-      const bool pf_lane = lane < 2;
-      const int pf_off = lane == 0 ? 0 : kNB * gw - 2;  // window's last byte
+      const uint8_t *rb = w.codes + pl * w.codes_plane_stride +
+                          ((row_lo + r_lo) * P.ng + w0) * kNB;
+      const uint16_t *sb = w.scales + pl * w.scales_plane_stride +
+                           (row_lo + r_lo) * P.ng + w0;
+      const uint8_t *ldc = rb + (full_win ? loff : lane);
+      const uint16_t *lds_ = sb + (full_win ? soff : lane);
+      // the last row's pointers: rows past r_n reload it (values unused)
+      const uint8_t *ldc_last = ldc + (int64_t)(r_n - 1) * c_row;
+      const uint16_t *lds_last = lds_ + (int64_t)(r_n - 1) * P.ng;
+      // all lanes prefetch: lane 1 the line of the window's last byte, the
+      // others its first line (same address: one request), and the scales
+      const uint8_t *pfc = rb + (lane == 1 ? kNB * gw - 1 : 0);
+      const uint16_t *pfs = sb;
       int pf_r = 0;
       for (; pf_r < kL2Ahead && pf_r < r_n; ++pf_r) {
-        if (pf_lane) prefetch_l2(pfc + pf_off);
-        if (lane == 0) prefetch_l2(pfs);
+        prefetch_l2(pfc);
+        prefetch_l2(pfs);
         pfc += c_row;
         pfs += P.ng;
       }
       uint32_t vb[kRing][kSteps];  // code bytes of the ring's rows
       uint32_t sr[kRing];          // raw fp16 scale (lanes 0..gw-1)
+      auto load_row = [&](int d, bool ok) {
+        if (full_win) {
+          const uint8_t *c = ok ? ldc : ldc_last;
+          const uint16_t *sp = ok ? lds_ : lds_last;
 #pragma unroll
-      for (int d = 0; d < kRing; ++d) {
-        const bool ok = d < r_n;
+          for (int i = 0; i < kSteps; ++i) vb[d][i] = ld_u8(c + kLanes * i);
+          sr[d] = ld_u16(sp);
+        } else {
 #pragma unroll
-        for (int i = 0; i < kSteps; ++i)
-          vb[d][i] = ok && st_on[i] ? ld_u8(ldc + kLanes * i) : 0u;
-        sr[d] = ok && sc_on ? ld_u16(lds_) : 0u;
+          for (int i = 0; i < kSteps; ++i)
+            vb[d][i] = ok && st_on[i] ? ld_u8(ldc + kLanes * i) : 0u;
+          sr[d] = ok && sc_on ? ld_u16(lds_) : 0u;
+        }
         ldc += c_row;
         lds_ += P.ng;
-      }
+      };
+#pragma unroll
+      for (int d = 0; d < kRing; ++d) load_row(d, d < r_n);
       for (int r0 = 0; r0 < r_n; r0 += kRing) {
         float v[kRing];
 #pragma unroll
@@ -222,16 +241,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           v[d] = acc;  // rows past r_n compute on zeros; not stored
           // refill the slot with row r0 + d + kRing
-          const bool ok = r0 + d + kRing < r_n;
-#pragma unroll
-          for (int i = 0; i < kSteps; ++i)
-            vb[d][i] = ok && st_on[i] ? ld_u8(ldc + kLanes * i) : 0u;
-          sr[d] = ok && sc_on ? ld_u16(lds_) : 0u;
-          ldc += c_row;
-          lds_ += P.ng;
+          load_row(d, r0 + d + kRing < r_n);
           if (pf_r < r_n) {
-            if (pf_lane) prefetch_l2(pfc + pf_off);
-            if (lane == 0) prefetch_l2(pfs);
+            prefetch_l2(pfc);
+            prefetch_l2(pfs);
           }
           ++pf_r;
           pfc += c_row;
