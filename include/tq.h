@@ -88,8 +88,9 @@ typedef struct {
   int64_t n_rows;          /* N: rows of W (outputs) */
   int64_t k_cols;          /* K: columns of W (inputs). B: multiple of 16 */
   const uint8_t *codes;    /* device, 16-byte aligned; layout above */
-  const uint16_t *scales;  /* device. A: fp16 group scales (required).
-                              B: rho (fp16) or NULL */
+  const uint16_t *scales;  /* device. A: fp16 group scales (required),
+                              16-byte aligned. B: rho (fp16, 2-byte
+                              aligned) or NULL */
   const float *lut;        /* B: device, 256 fp32 (tq_build_lut), 16-byte
                               aligned. A: ignored */
   int64_t codes_plane_stride;  /* A: bytes between planes; 0 = dense */

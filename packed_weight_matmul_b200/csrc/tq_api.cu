@@ -48,7 +48,8 @@ tq_status check_weights(const tq_weights *w, tq::WeightsView *v) {
       return TQ_ERR_SHAPE;
     if (w->codes_plane_stride < 0 || w->scales_plane_stride < 0)
       return TQ_ERR_INVALID_ARG;
-    if (!aligned(w->codes, 16) || !aligned(w->scales, 2))
+    // scales 16-byte aligned: kernels fetch them in aligned 16-byte chunks
+    if (!aligned(w->codes, 16) || !aligned(w->scales, 16))
       return TQ_ERR_ALIGNMENT;
   } else if (w->format == TQ_FMT_B) {
     if (w->planes != 1) return TQ_ERR_INVALID_ARG;

@@ -41,21 +41,30 @@ namespace {
 constexpr int kTileM = 128;
 constexpr int kMaxN = 64;
 constexpr int kBlockK = 64;                       // k per stage
-// Decoder warps per CTA (a multiple of 4: the TMEM lane quarters). Format B
-// decodes are short (a lookup per weight), so 16 warps, 16 k per thread, keep
-// more loads in flight; a Format A thread rebuilds its group's trit masks,
-// so 8 warps (32 k per thread) share that work better.
+// Decoder warps per CTA (a multiple of 4: the TMEM lane quarters): 16, four
+// per scheduler, 16 k per thread. The decode is bound by instruction issue
+// and latency, so every warp the register budget allows is a decoder.
 template <int FMT>
 struct TcCfg {
-  static constexpr int kDecoderWarps = FMT == TQ_FMT_B ? 16 : 8;
+  static constexpr int kDecoderWarps = 16;
   static constexpr int kKParts = kDecoderWarps / 4;  // k parts of a block
   static constexpr int kKPT = kBlockK / kKParts;     // k per decoder thread
+
   static constexpr int kXPerThread =
       (kMaxN * 8 + kDecoderWarps * 32 - 1) / (kDecoderWarps * 32);
   static constexpr int kThreads = 32 * (1 + kDecoderWarps);
 };
 constexpr int kStages = 6;                        // A in TMEM, x in smem
-constexpr int kCodeDepth = 6;                     // code blocks per thread ring
+constexpr int kCodeDepth = 6;                     // x (and B code) ring depth
+// Format A codes arrive in windows of kWinBlocks k-blocks: per row the
+// window's 8 groups (104 code bytes) and 8 scales (16 bytes), fetched as
+// 16-byte aligned chunks (so up to 128 + 32 bytes with the alignment slack)
+// by all decoder threads together, lanes on consecutive chunks of a row.
+constexpr int kWinBlocks = 8;
+constexpr int kWinSlots = 3;                      // windows in the ring
+constexpr int kWinRowCodes = 128;
+constexpr int kWinRowBytes = kWinRowCodes + 32;
+constexpr int kWinChunks = kTileM * kWinRowBytes / 16;  // 16-byte copies
 constexpr uint32_t kTmemCols = 512;               // the whole tensor memory
 constexpr uint32_t kAccCols = 64;                 // accumulator: N <= 64
 constexpr uint32_t kStageCols = 64;               // A stage: 32 hi + 32 lo
@@ -76,7 +85,9 @@ struct TcParams {
   int stage_bytes;  // x tile
   int x_off;        // x tile offset inside a stage
   int ring_off, lut_off, bar_off, tmem_slot_off;
-  int code_off, code_slot;  // code ring: kCodeDepth slots of 128 rows x 64 B
+  int code_off, code_slot;  // B: kCodeDepth slots of 128 rows x 64 B;
+                            // A: kWinSlots windows of 128 rows x 160 B
+  int xring_off;            // x ring: kCodeDepth slots of n_pad rows x 128 B
   size_t smem;
 };
 
@@ -88,12 +99,6 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, int n)
                : "memory");
 }
 
-__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src, int n) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst),
-               "l"(src), "r"(n)
-               : "memory");
-}
-
 __device__ __forceinline__ void cp_async_commit() {
   asm volatile("cp.async.commit_group;" ::: "memory");
 }
@@ -101,6 +106,13 @@ __device__ __forceinline__ void cp_async_commit() {
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Arrives on `bar` once every cp.async this thread issued so far has landed
+// (the barrier's count includes this arrival).
+__device__ __forceinline__ void cp_async_mbar_arrive(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar)
+               : "memory");
 }
 
 // Warp-wide store of N (8 or 16) consecutive TMEM columns.
@@ -139,28 +151,26 @@ __device__ __forceinline__ void decode8_b(uint32_t w0, uint32_t w1,
   }
 }
 
-// Format A: trits 8c..8c+7 of a group given as bit masks (bit j: t_j != 0,
-// t_j < 0) -> 4 hi and 4 lo pairs of s*t.
-__device__ __forceinline__ void decode8_a(uint64_t nz, uint64_t neg, int c,
-                                          uint32_t s_hi, uint32_t s_lo,
+// Format A: trits 8c..8c+7 of the thread's 16, given as 2-bit fields
+// (bit 2j: t_j != 0, bit 2j+1: t_j < 0) -> 4 hi and 4 lo pairs of s*t.
+// s2 = s | s << 16 (hi or lo part of the scale in both halves); pair_tab[f]
+// holds, for the 4 bits f of a pair, the keep mask (0xFFFF per nonzero half)
+// and the sign mask (0x8000 per negative half), so a pair is one
+// (s2 & keep) ^ sign. XOR (not OR) keeps a negative lo part exact.
+__device__ __forceinline__ void decode8_a(uint32_t bits, int c,
+                                          uint32_t s_hi2, uint32_t s_lo2,
+                                          uint32_t pair_tab,
                                           uint32_t (&hi)[4],
                                           uint32_t (&lo)[4]) {
-  const uint32_t z8 = (uint32_t)(nz >> (8 * c)) & 0xFFu;
-  const uint32_t n8 = (uint32_t)(neg >> (8 * c)) & 0xFFu;
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
-    uint32_t h = 0, l = 0;
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int j = 2 * q + e;
-      const uint32_t on = (z8 >> j) & 1u, sg = ((n8 >> j) & 1u) << 15;
-      const uint32_t vh = on ? (s_hi ^ sg) : 0u;
-      const uint32_t vl = on ? (s_lo ^ sg) : 0u;
-      h |= vh << (16 * e);
-      l |= vl << (16 * e);
-    }
-    hi[q] = h;
-    lo[q] = l;
+    const uint32_t f = (bits >> (16 * c + 4 * q)) & 15u;
+    uint32_t keep, sign;
+    asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];"
+                 : "=r"(keep), "=r"(sign)
+                 : "r"(pair_tab + f * 8u));
+    hi[q] = (s_hi2 & keep) ^ sign;
+    lo[q] = (s_lo2 & keep) ^ sign;
   }
 }
 
@@ -178,6 +188,8 @@ __global__ void __launch_bounds__(TcCfg<FMT>::kThreads, 1)
   const uint32_t full0 = sbase + P.bar_off;           // full[s]: decoders done
   const uint32_t empty0 = full0 + 8 * kStages;        // empty[s]: MMAs done
   const uint32_t acc_bar = empty0 + 8 * kStages;      // accumulator ready
+  const uint32_t wfull0 = acc_bar + 8;                // A window landed
+  const uint32_t wempty0 = wfull0 + 8 * kWinSlots;    // A window consumed
   volatile uint32_t &tmem_slot =
       *reinterpret_cast<uint32_t *>(smem + P.tmem_slot_off);
   volatile int &abort_flag =
@@ -203,6 +215,12 @@ __global__ void __launch_bounds__(TcCfg<FMT>::kThreads, 1)
       mbar_init(empty0 + 8 * s, 1);
     }
     mbar_init(acc_bar, 1);
+    if constexpr (FMT == TQ_FMT_A) {
+      for (int s = 0; s < kWinSlots; ++s) {
+        mbar_init(wfull0 + 8 * s, kDecoderWarps * 32);
+        mbar_init(wempty0 + 8 * s, kDecoderWarps * 32);
+      }
+    }
     mbar_init_fence();
   }
   if (warp == 0) tmem_alloc(sbase + P.tmem_slot_off, kTmemCols);
@@ -224,7 +242,8 @@ __global__ void __launch_bounds__(TcCfg<FMT>::kThreads, 1)
       }
     }
   } else {
-    // byte -> trit masks of its 5 digits: bits 0-4 t != 0, bits 5-9 t < 0
+    // byte -> its 5 trits (least significant digit first) as 2-bit fields:
+    // bit 2i: t_i != 0, bit 2i+1: t_i < 0
     uint16_t *tab = reinterpret_cast<uint16_t *>(smem + P.lut_off);
     for (int b = threadIdx.x; b < 256; b += blockDim.x) {
       uint32_t m = 0, rest = b < 243 ? b : 121;
@@ -232,10 +251,19 @@ __global__ void __launch_bounds__(TcCfg<FMT>::kThreads, 1)
       for (int i = 0; i < 5; ++i) {
         const uint32_t d = rest % 3;
         rest /= 3;
-        if (d != 1) m |= 1u << i;
-        if (d == 0) m |= 1u << (5 + i);
+        if (d != 1) m |= 1u << (2 * i);
+        if (d == 0) m |= 1u << (2 * i + 1);
       }
       tab[b] = (uint16_t)m;
+    }
+    // pair table (16 entries of keep, sign words) after the byte table,
+    // indexed by two 2-bit fields
+    uint32_t *ptab = reinterpret_cast<uint32_t *>(smem + P.lut_off + 512);
+    for (int i = threadIdx.x; i < 16; i += blockDim.x) {
+      const uint32_t z0 = i & 1, n0 = (i >> 1) & 1, z1 = (i >> 2) & 1,
+                     n1 = (i >> 3) & 1;
+      ptab[2 * i] = (z0 ? 0x0000FFFFu : 0u) | (z1 ? 0xFFFF0000u : 0u);
+      ptab[2 * i + 1] = (z0 && n0 ? 0x00008000u : 0u) | (z1 && n1 ? 0x80000000u : 0u);
     }
   }
   tc_fence_before_sync();
@@ -280,21 +308,40 @@ __global__ void __launch_bounds__(TcCfg<FMT>::kThreads, 1)
     const uint32_t lane8 = (uint32_t)lane * 8u;
     const uint32_t lut_base = sbase + P.lut_off;
     const int64_t gpr = K / 64;  // Format A groups per row (G = 64)
-    auto plane_of = [&](int it) { return (it_begin + it) / kblocks; };
-    // Codes stream into a per-thread ring of kCodeDepth blocks in shared
-    // memory with cp.async (each thread reads back only the bytes its own
-    // copies wrote), so kCodeDepth - 1 blocks of every row are in flight.
-    const int64_t plane_bytes = w.n * gpr * 13;  // Format A code bytes per plane
+    const int dt = wid * 32 + lane;  // decoder thread index
+    // Format B codes stream into a per-thread ring of kCodeDepth blocks in
+    // shared memory with cp.async (each thread reads back only the bytes its
+    // own copies wrote), so kCodeDepth - 1 blocks of every row are in flight.
     const uint32_t code_ring = sbase + P.code_off + r * 64 + kp * kKPT;
-    uint32_t sc[kCodeDepth];                      // Format A scales, in order
-#pragma unroll
-    for (int q = 0; q < kCodeDepth; ++q) sc[q] = 0;
-    auto issue = [&](int it) -> uint32_t {      // returns the block's scale
-      const uint32_t dst = code_ring + (uint32_t)(it % kCodeDepth) * P.code_slot;
-      if (it >= iters) return 0;
+    // Format A: the 16 trits k in [16 kp, 16 kp + 16) of a group lie in its
+    // code bytes m_lo .. m_lo + 3, from trit a_off of byte m_lo on
+    const int m_lo = (kKPT * kp) / 5;
+    const int a_off = kKPT * kp - 5 * m_lo;
+    // x chunks (16 B: one row, 8 k) ride in per-block cp.async groups: chunk
+    // id of block it lands at x_ring(it) + 16 id, copied and read by one thread.
+    auto x_ring = [&](int it) {
+      return sbase + P.xring_off + (uint32_t)(it % kCodeDepth) * (uint32_t)(N * 128);
+    };
+    auto issue = [&](int it) {
+      if (it >= iters) return;
       const int gi_it = it_begin + it;
       const int plane = gi_it / kblocks, kb = gi_it - plane * kblocks;
+      (void)plane;
+      {
+        const uint32_t xd = x_ring(it);
+#pragma unroll
+        for (int q = 0; q < kXPerThread; ++q) {
+          const int id = dt + q * kDecoderWarps * 32;
+          if (id < N * 8) {
+            const int n = id >> 3, c = id & 7;
+            const int64_t kk = (int64_t)kb * kBlockK + 8 * c;
+            const bool ok = n < batch && kk < K;
+            cp_async16(xd + 16 * id, ok ? x + (int64_t)n * ldx + kk : x, ok ? 16 : 0);
+          }
+        }
+      }
       if constexpr (FMT == TQ_FMT_B) {
+        const uint32_t dst = code_ring + (uint32_t)(it % kCodeDepth) * P.code_slot;
         const int64_t kk = (int64_t)kb * kBlockK + kKPT * kp;
         const uint8_t *p = w.codes + (row_ok ? grow : 0) * K + kk;
 #pragma unroll
@@ -302,121 +349,151 @@ __global__ void __launch_bounds__(TcCfg<FMT>::kThreads, 1)
           const bool ok = row_ok && kk + 16 * j < K;
           cp_async16(dst + 16 * j, ok ? p + 16 * j : w.codes, ok ? 16 : 0);
         }
-        return 0;
-      } else {
-        if (!row_ok) return 0;
-        const int64_t gi = grow * gpr + kb;
-        const uint8_t *plane_base = w.codes + plane * w.codes_plane_stride;
-        const uint8_t *grp = plane_base + gi * 13;
-        const uint8_t *end = plane_base + plane_bytes;
-        // 4-byte aligned window on the absolute address (a plane may start
-        // at any byte); copies stop at the end of this plane's data.
-        const uint8_t *win = reinterpret_cast<const uint8_t *>(
-            reinterpret_cast<uintptr_t>(grp) & ~(uintptr_t)3);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint8_t *src = win + 4 * q;
-          const int64_t left = end - src;
-          const int n = left >= 4 ? 4 : (left > 0 ? (int)left : 0);
-          cp_async4(dst + 4 * q, n > 0 ? src : w.codes, n);
-        }
-        return __ldg(w.scales + plane * w.scales_plane_stride + gi);
       }
     };
+    // Format A windows: the CTA's iterations [g0, g1) split at the plane
+    // boundary into at most two runs, each cut into windows of kWinBlocks.
+    const int g0 = it_begin, g1 = it_begin + iters;
+    const int run0_end =
+        kblocks > 0 ? min(g1, (g0 / kblocks + 1) * kblocks) : g0;
+    const int n_win0 = (run0_end - g0 + kWinBlocks - 1) / kWinBlocks;
+    const int n_win = n_win0 + (g1 - run0_end + kWinBlocks - 1) / kWinBlocks;
+    auto win_lo = [&](int j) {
+      return j < n_win0 ? g0 + kWinBlocks * j : run0_end + kWinBlocks * (j - n_win0);
+    };
+    auto win_hi = [&](int j) {
+      return min(win_lo(j) + kWinBlocks, j < n_win0 ? run0_end : g1);
+    };
+    const int64_t plane_bytes = w.n * gpr * 13;  // Format A code bytes per plane
+    // Every decoder thread copies its share of window j's chunks (chunk i:
+    // row i / 10, the row's code chunk i % 10 < 8 or scale chunk i % 10 - 8)
+    // into slot j % kWinSlots, once all decoders finished the window that
+    // used the slot before; the copies complete on wfull[slot]. Chunks stop
+    // at the end of the plane's codes or scales.
+    auto issue_win = [&](int j) -> bool {
+      if (j >= n_win) return true;
+      const int slot = j % kWinSlots;
+      if (j >= kWinSlots &&
+          !mbar_wait(wempty0 + 8 * slot, ((j / kWinSlots) - 1) & 1))
+        return false;
+      const int gs = win_lo(j);
+      const int plane = gs / kblocks, kb0 = gs - plane * kblocks;
+      const uint8_t *cbase = w.codes + plane * w.codes_plane_stride;
+      const uint8_t *cend = cbase + plane_bytes;
+      const uint16_t *sbase_p = w.scales + plane * w.scales_plane_stride;
+      const uint8_t *send = reinterpret_cast<const uint8_t *>(sbase_p + w.n * gpr);
+      const uint32_t wslot = sbase + P.code_off + (uint32_t)slot * P.code_slot;
+      for (int i = dt; i < kWinChunks; i += kDecoderWarps * 32) {
+        const int row = i / 10, ch = i - 10 * row;
+        const int64_t gr = row0 + row;
+        if (gr >= w.n) continue;
+        const int64_t gi0 = gr * gpr + kb0;
+        const bool is_scale = ch >= 8;
+        const uint8_t *first = is_scale
+            ? reinterpret_cast<const uint8_t *>(sbase_p + gi0)
+            : cbase + gi0 * 13;
+        const uint8_t *src = reinterpret_cast<const uint8_t *>(
+                                 reinterpret_cast<uintptr_t>(first) & ~(uintptr_t)15) +
+                             16 * (is_scale ? ch - 8 : ch);
+        const int64_t left = (is_scale ? send : cend) - src;
+        const int nb = left >= 16 ? 16 : (left > 0 ? (int)left : 0);
+        cp_async16(wslot + (uint32_t)(row * kWinRowBytes + 16 * ch),
+                   nb > 0 ? src : w.codes, nb);
+      }
+      cp_async_mbar_arrive(wfull0 + 8 * slot);
+      return true;
+    };
+    bool ok0 = true;
+    if constexpr (FMT == TQ_FMT_A) {
+      for (int j = 0; j + 1 < kWinSlots; ++j) ok0 = ok0 && issue_win(j);
+    }
 #pragma unroll
     for (int q = 0; q < kCodeDepth - 1; ++q) {
-      sc[q] = issue(q);
+      issue(q);
       cp_async_commit();
     }
-    // This thread's (at most two) 16-byte x chunks of block it; zero past
-    // the batch, past K and past the slice.
-    auto load_x = [&](int it, uint4 (&v)[kXPerThread]) {
-#pragma unroll
-      for (int q = 0; q < kXPerThread; ++q) {
-        v[q] = make_uint4(0, 0, 0, 0);
-        const int id = wid * 32 + lane + q * kDecoderWarps * 32;
-        const int n = id >> 3, c = id & 7;
-        if (it < iters && id < N * 8 && n < batch) {
-          const int64_t kk = (int64_t)((it_begin + it) % kblocks) * kBlockK + 8 * c;
-          if (kk < K) v[q] = *reinterpret_cast<const uint4 *>(x + (int64_t)n * ldx + kk);
-        }
-      }
-    };
-    uint4 xr0[kXPerThread], xr1[kXPerThread];
-    load_x(0, xr0);
-    load_x(1, xr1);
+    if (!__all_sync(0xFFFFFFFFu, ok0)) abort_flag = 1;
+    int wj = 0;                                  // current Format A window
+    int w_lo = n_win > 0 ? win_lo(0) : 0, w_hi = n_win > 0 ? win_hi(0) : 0;
+    uint32_t w_row = 0, c_off0 = 0, s_off0 = 0;  // its row base and offsets
     // Every decision before a warp-wide (.sync.aligned) instruction is made
     // uniform across the warp.
     for (int it = 0; it < iters && !__any_sync(0xFFFFFFFFu, abort_flag != 0);
          ++it) {
       const int s = it % kStages;
-      const int kb = (it_begin + it) % kblocks;
-      sc[kCodeDepth - 1] = issue(it + kCodeDepth - 1);
+      const int g = it_begin + it;
+      issue(it + kCodeDepth - 1);
       cp_async_commit();
-      cp_async_wait<kCodeDepth - 1>();  // this block's codes have landed
-      const uint32_t src = code_ring + (uint32_t)(it % kCodeDepth) * P.code_slot;
-      uint32_t cw[kKPT / 4 > 4 ? kKPT / 4 : 4];
-#pragma unroll
-      for (int j = 0; j < (kKPT / 16 > 1 ? kKPT / 16 : 1); ++j) {
-        uint4 a;
-        asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
-                     : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w)
-                     : "r"(src + 16 * j));
-        cw[4 * j] = a.x; cw[4 * j + 1] = a.y; cw[4 * j + 2] = a.z;
-        cw[4 * j + 3] = a.w;
-      }
-      if constexpr (FMT == TQ_FMT_B) {
-        if (!row_ok) {
-#pragma unroll
-          for (int q = 0; q < kKPT / 4; ++q) cw[q] = 0x79797979u;  // weight 0
-        }
-      }
-      const uint32_t cur_scale = sc[0];
-#pragma unroll
-      for (int q = 0; q + 1 < kCodeDepth; ++q) sc[q] = sc[q + 1];
-      uint64_t nz = 0, neg = 0;
+      cp_async_wait<kCodeDepth - 1>();  // this block's x (and B codes) landed
+      uint32_t bits = 0;  // Format A: the thread's 16 trits, 2 bits each
       uint32_t s_hi = 0, s_lo = 0;
+      uint32_t cw[4];
       if constexpr (FMT == TQ_FMT_A) {
+        if (g == w_lo) {  // first block of window wj
+          bool ok = issue_win(wj + kWinSlots - 1);
+          ok = ok && mbar_wait(wfull0 + 8 * (wj % kWinSlots), (wj / kWinSlots) & 1);
+          if (!__all_sync(0xFFFFFFFFu, ok)) {
+            abort_flag = 1;
+            break;
+          }
+          const int plane = g / kblocks, kb0 = g - plane * kblocks;
+          const int64_t gi0 = (row_ok ? grow : 0) * gpr + kb0;
+          c_off0 = (uint32_t)(reinterpret_cast<uintptr_t>(
+                                  w.codes + plane * w.codes_plane_stride + gi0 * 13) & 15);
+          s_off0 = (uint32_t)(reinterpret_cast<uintptr_t>(
+                                  w.scales + plane * w.scales_plane_stride + gi0) & 15);
+          w_row = sbase + P.code_off + (uint32_t)(wj % kWinSlots) * P.code_slot +
+                  (uint32_t)(r * kWinRowBytes);
+        }
         if (row_ok) {
-          uint32_t v[4];
-          const uint32_t sh =
-              8u * (uint32_t)(reinterpret_cast<uintptr_t>(
-                                  w.codes + plane_of(it) * w.codes_plane_stride +
-                                  (grow * gpr + kb) * 13) & 3);
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            v[q] = __funnelshift_r(cw[q], q < 3 ? cw[q + 1] : 0u, sh);
+          const uint32_t off = c_off0 + 13u * (uint32_t)(g - w_lo) + (uint32_t)m_lo;
+          uint32_t w0, w1;
+          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w0) : "r"(w_row + (off & ~3u)));
+          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w1) : "r"(w_row + (off & ~3u) + 4));
+          const uint32_t word = __funnelshift_r(w0, w1, 8u * (off & 3u));
           const uint16_t *tab =
               reinterpret_cast<const uint16_t *>(smem + P.lut_off);
-          // only the bytes that hold this thread's kKPT trits
-          constexpr int kBytes = (kKPT + 8) / 5;  // bytes any kKPT-window spans
-          const int m_lo = (kKPT * kp) / 5;
-#pragma unroll
-          for (int j = 0; j < kBytes; ++j) {
-            const int m = m_lo + j;
-            if (m < 13) {
-              const int wi = m >> 2;  // selected without indexing (no stack)
-              const uint32_t wv = wi == 0 ? v[0] : wi == 1 ? v[1] : wi == 2 ? v[2] : v[3];
-              const uint32_t e = tab[(wv >> (8 * (m & 3))) & 0xFFu];
-              nz |= (uint64_t)(e & 31u) << (5 * m);
-              neg |= (uint64_t)((e >> 5) & 31u) << (5 * m);
-            }
-          }
-          const float sf = __half2float(__ushort_as_half((uint16_t)cur_scale));
+          const uint32_t t0 = tab[word & 0xFFu], t1 = tab[(word >> 8) & 0xFFu],
+                         t2 = tab[(word >> 16) & 0xFFu], t3 = tab[word >> 24];
+          const uint32_t lo32 = t0 | t1 << 10 | t2 << 20 | t3 << 30;
+          bits = __funnelshift_r(lo32, t3 >> 2, 2u * (uint32_t)a_off);
+          uint16_t sbits;
+          asm volatile("ld.shared.u16 %0, [%1];"
+                       : "=h"(sbits)
+                       : "r"(w_row + kWinRowCodes + s_off0 + 2u * (uint32_t)(g - w_lo)));
+          const float sf = __half2float(__ushort_as_half(sbits));
           s_hi = bf16_bits_rn(sf);
           s_lo = bf16_bits_rn(sf - __uint_as_float(s_hi << 16));
+          s_hi |= s_hi << 16;  // both halves of a pair
+          s_lo |= s_lo << 16;
+        }
+        if (g + 1 == w_hi) {  // this thread is done reading window wj
+          mbar_arrive(wempty0 + 8 * (wj % kWinSlots));
+          ++wj;
+          if (wj < n_win) {
+            w_lo = win_lo(wj);
+            w_hi = win_hi(wj);
+          }
+        }
+      } else {
+        const uint32_t src = code_ring + (uint32_t)(it % kCodeDepth) * P.code_slot;
+        asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                     : "=r"(cw[0]), "=r"(cw[1]), "=r"(cw[2]), "=r"(cw[3])
+                     : "r"(src));
+        if (!row_ok) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) cw[q] = 0x79797979u;  // weight 0
         }
       }
       // decode this thread's kKPT k of its row: kKPT/2 hi and lo bf16 pairs
       uint32_t hi[kKPT / 2], lo[kKPT / 2];
 #pragma unroll
       for (int cc = 0; cc < kKPT / 8; ++cc) {
-        const int c = (kKPT / 8) * kp + cc;  // 8-k chunk of the block
         uint32_t h4[4], l4[4];
         if constexpr (FMT == TQ_FMT_B)
           decode8_b(cw[2 * cc], cw[2 * cc + 1], lut_base, lane8, h4, l4);
         else
-          decode8_a(nz, neg, c, s_hi, s_lo, h4, l4);
+          decode8_a(bits, cc, s_hi, s_lo, lut_base + 512, h4, l4);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           hi[4 * cc + q] = h4[q];
@@ -440,16 +517,22 @@ __global__ void __launch_bounds__(TcCfg<FMT>::kThreads, 1)
         tmem_st_wait();
       }
       uint8_t *st = smem + P.ring_off + s * P.stage_bytes;
-      // x tile: N rows x 64 k, 16 bytes per chunk (fetched two blocks ahead)
+      // x tile: N rows x 64 k, 16 bytes per chunk, from this thread's ring
+      {
+        const uint32_t xs = x_ring(it);
 #pragma unroll
-      for (int q = 0; q < kXPerThread; ++q) {
-        const int id = wid * 32 + lane + q * kDecoderWarps * 32;
-        if (id < N * 8)
-          *reinterpret_cast<uint4 *>(st + P.x_off +
-                                     tile_off(id >> 3, 8 * (id & 7), N)) = xr0[q];
-        xr0[q] = xr1[q];
+        for (int q = 0; q < kXPerThread; ++q) {
+          const int id = dt + q * kDecoderWarps * 32;
+          if (id < N * 8) {
+            uint4 v;
+            asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                         : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                         : "r"(xs + 16 * id));
+            *reinterpret_cast<uint4 *>(st + P.x_off +
+                                       tile_off(id >> 3, 8 * (id & 7), N)) = v;
+          }
+        }
       }
-      load_x(it + 2, xr1);
       fence_async_shared();   // x tile -> async proxy (MMA operand B)
       tc_fence_before_sync();  // A stores -> ordered before the arrive
       __syncwarp();
@@ -525,12 +608,13 @@ TcParams plan_tc(int fmt, int64_t batch) {
   P.stage_bytes = P.n_pad * kBlockK * 2;
   P.x_off = 0;
   P.ring_off = 0;
-  P.code_slot = kTileM * 64;
+  P.code_slot = kTileM * (fmt == TQ_FMT_A ? kWinRowBytes : 64);
   P.code_off = kStages * P.stage_bytes;
-  P.lut_off = P.code_off + kCodeDepth * P.code_slot;
-  const int table = fmt == TQ_FMT_B ? kLutBytes : 512;
+  P.xring_off = P.code_off + (fmt == TQ_FMT_A ? kWinSlots : kCodeDepth) * P.code_slot;
+  P.lut_off = P.xring_off + kCodeDepth * P.n_pad * 128;
+  const int table = fmt == TQ_FMT_B ? kLutBytes : 512 + 128;
   P.bar_off = P.lut_off + table;
-  P.tmem_slot_off = P.bar_off + (2 * kStages + 1) * 8 + 8;
+  P.tmem_slot_off = P.bar_off + (2 * kStages + 1 + 2 * kWinSlots) * 8 + 8;
   P.smem = (size_t)P.tmem_slot_off + 16;
   // one CTA per SM: each allocates the whole tensor memory
   if (P.smem < 120 * 1024) P.smem = 120 * 1024;

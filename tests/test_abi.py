@@ -104,6 +104,8 @@ def test_validation_before_launch(tq):
     assert _linear(tq, _wa(tq, group=32)) == E.TQ_ERR_UNSUPPORTED
     assert _linear(tq, _wa(tq, k_cols=100)) == E.TQ_ERR_SHAPE
     assert _linear(tq, _wa(tq, codes=0x10008)) == E.TQ_ERR_ALIGNMENT
+    assert _linear(tq, _wa(tq, scales=0x20002)) == E.TQ_ERR_ALIGNMENT
+    assert _linear(tq, _wa(tq, scales=0x20008)) == E.TQ_ERR_ALIGNMENT  # A: 16 B
     assert _linear(tq, _wa(tq, format=7)) == E.TQ_ERR_INVALID_ARG
     assert _linear(tq, _wa(tq), x=None) == E.TQ_ERR_INVALID_ARG
     assert _linear(tq, _wa(tq), batch=0) == E.TQ_ERR_INVALID_ARG
