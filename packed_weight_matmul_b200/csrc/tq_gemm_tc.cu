@@ -318,38 +318,52 @@ __global__ void __launch_bounds__(TcCfg<FMT>::kThreads, 1)
     const int m_lo = (kKPT * kp) / 5;
     const int a_off = kKPT * kp - 5 * m_lo;
     // x chunks (16 B: one row, 8 k) ride in per-block cp.async groups: chunk
-    // id of block it lands at x_ring(it) + 16 id, copied and read by one thread.
-    auto x_ring = [&](int it) {
-      return sbase + P.xring_off + (uint32_t)(it % kCodeDepth) * (uint32_t)(N * 128);
+    // id of a block lands at x_ring(slot) + 16 id, copied and read by one
+    // thread; slot = the block's iteration mod kCodeDepth.
+    auto x_ring = [&](int slot) {
+      return sbase + P.xring_off + (uint32_t)slot * (uint32_t)(N * 128);
     };
-    auto issue = [&](int it) {
-      if (it >= iters) return;
-      const int gi_it = it_begin + it;
-      const int plane = gi_it / kblocks, kb = gi_it - plane * kblocks;
-      (void)plane;
-      {
-        const uint32_t xd = x_ring(it);
+    // this thread's x chunks: row n, k offset 8c inside a block
+    const __nv_bfloat16 *x_src[kXPerThread];
+    bool x_live[kXPerThread];
+#pragma unroll
+    for (int q = 0; q < kXPerThread; ++q) {
+      const int id = dt + q * kDecoderWarps * 32;
+      const int n = id >> 3, c = id & 7;
+      x_live[q] = id < N * 8;
+      x_src[q] = n < batch ? x + (int64_t)n * ldx + 8 * c : nullptr;
+    }
+    // The next block to issue: its iteration, k-block and ring slot, kept
+    // as counters (blocks are issued in order).
+    int nx_it = 0, nx_slot = 0;
+    int nx_kb = kblocks > 0 ? it_begin % kblocks : 0;
+    auto issue_next = [&]() {
+      if (nx_it < iters) {
+        const uint32_t xd = x_ring(nx_slot);
 #pragma unroll
         for (int q = 0; q < kXPerThread; ++q) {
-          const int id = dt + q * kDecoderWarps * 32;
-          if (id < N * 8) {
-            const int n = id >> 3, c = id & 7;
-            const int64_t kk = (int64_t)kb * kBlockK + 8 * c;
-            const bool ok = n < batch && kk < K;
-            cp_async16(xd + 16 * id, ok ? x + (int64_t)n * ldx + kk : x, ok ? 16 : 0);
+          if (x_live[q]) {
+            const int id = dt + q * kDecoderWarps * 32;
+            const int64_t kk = (int64_t)nx_kb * kBlockK + 8 * (id & 7);
+            const bool ok = x_src[q] != nullptr && kk < K;
+            cp_async16(xd + 16 * id, ok ? x_src[q] + (int64_t)nx_kb * kBlockK : x,
+                       ok ? 16 : 0);
+          }
+        }
+        if constexpr (FMT == TQ_FMT_B) {
+          const uint32_t dst = code_ring + (uint32_t)nx_slot * P.code_slot;
+          const int64_t kk = (int64_t)nx_kb * kBlockK + kKPT * kp;
+          const uint8_t *p = w.codes + (row_ok ? grow : 0) * K + kk;
+#pragma unroll
+          for (int j = 0; j < kKPT / 16; ++j) {
+            const bool ok = row_ok && kk + 16 * j < K;
+            cp_async16(dst + 16 * j, ok ? p + 16 * j : w.codes, ok ? 16 : 0);
           }
         }
       }
-      if constexpr (FMT == TQ_FMT_B) {
-        const uint32_t dst = code_ring + (uint32_t)(it % kCodeDepth) * P.code_slot;
-        const int64_t kk = (int64_t)kb * kBlockK + kKPT * kp;
-        const uint8_t *p = w.codes + (row_ok ? grow : 0) * K + kk;
-#pragma unroll
-        for (int j = 0; j < kKPT / 16; ++j) {
-          const bool ok = row_ok && kk + 16 * j < K;
-          cp_async16(dst + 16 * j, ok ? p + 16 * j : w.codes, ok ? 16 : 0);
-        }
-      }
+      ++nx_it;
+      nx_slot = nx_slot + 1 == kCodeDepth ? 0 : nx_slot + 1;
+      nx_kb = nx_kb + 1 == kblocks ? 0 : nx_kb + 1;
     };
     // Format A windows: the CTA's iterations [g0, g1) split at the plane
     // boundary into at most two runs, each cut into windows of kWinBlocks.
@@ -409,20 +423,21 @@ __global__ void __launch_bounds__(TcCfg<FMT>::kThreads, 1)
     }
 #pragma unroll
     for (int q = 0; q < kCodeDepth - 1; ++q) {
-      issue(q);
+      issue_next();
       cp_async_commit();
     }
     if (!__all_sync(0xFFFFFFFFu, ok0)) abort_flag = 1;
     int wj = 0;                                  // current Format A window
     int w_lo = n_win > 0 ? win_lo(0) : 0, w_hi = n_win > 0 ? win_hi(0) : 0;
     uint32_t w_row = 0, c_off0 = 0, s_off0 = 0;  // its row base and offsets
+    int s = 0, cur = 0;    // stage of block it, its x / code ring slot
+    uint32_t e_par = 1;    // parity of the stage's previous use (from round 1)
     // Every decision before a warp-wide (.sync.aligned) instruction is made
     // uniform across the warp.
     for (int it = 0; it < iters && !__any_sync(0xFFFFFFFFu, abort_flag != 0);
          ++it) {
-      const int s = it % kStages;
       const int g = it_begin + it;
-      issue(it + kCodeDepth - 1);
+      issue_next();  // block it + kCodeDepth - 1
       cp_async_commit();
       cp_async_wait<kCodeDepth - 1>();  // this block's x (and B codes) landed
       uint32_t bits = 0;  // Format A: the thread's 16 trits, 2 bits each
@@ -476,7 +491,7 @@ __global__ void __launch_bounds__(TcCfg<FMT>::kThreads, 1)
           }
         }
       } else {
-        const uint32_t src = code_ring + (uint32_t)(it % kCodeDepth) * P.code_slot;
+        const uint32_t src = code_ring + (uint32_t)cur * P.code_slot;
         asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
                      : "=r"(cw[0]), "=r"(cw[1]), "=r"(cw[2]), "=r"(cw[3])
                      : "r"(src));
@@ -501,7 +516,7 @@ __global__ void __launch_bounds__(TcCfg<FMT>::kThreads, 1)
         }
       }
       if (it >= kStages) {
-        const bool ok = mbar_wait(empty0 + 8 * s, ((it / kStages) - 1) & 1);
+        const bool ok = mbar_wait(empty0 + 8 * s, e_par);
         if (!__all_sync(0xFFFFFFFFu, ok)) {
           abort_flag = 1;
           break;
@@ -519,7 +534,7 @@ __global__ void __launch_bounds__(TcCfg<FMT>::kThreads, 1)
       uint8_t *st = smem + P.ring_off + s * P.stage_bytes;
       // x tile: N rows x 64 k, 16 bytes per chunk, from this thread's ring
       {
-        const uint32_t xs = x_ring(it);
+        const uint32_t xs = x_ring(cur);
 #pragma unroll
         for (int q = 0; q < kXPerThread; ++q) {
           const int id = dt + q * kDecoderWarps * 32;
@@ -537,6 +552,11 @@ __global__ void __launch_bounds__(TcCfg<FMT>::kThreads, 1)
       tc_fence_before_sync();  // A stores -> ordered before the arrive
       __syncwarp();
       if (lane == 0) mbar_arrive(full0 + 8 * s);
+      if (++s == kStages) {
+        s = 0;
+        e_par ^= 1u;
+      }
+      cur = cur + 1 == kCodeDepth ? 0 : cur + 1;
     }
     cp_async_wait<0>();
     // ---- epilogue: warps of the first half read their TMEM lane quarter ----
