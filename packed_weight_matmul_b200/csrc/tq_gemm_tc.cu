@@ -1,5 +1,6 @@
 // Fused packed GEMM on the fifth-generation tensor cores (tcgen05), for the
-// batches where x * W_hat^T is a real contraction (batch >= 8 here):
+// batches the GEMV kernels do not take (Format B batch >= 5, Format A
+// batch >= 2), where x * W_hat^T becomes a real contraction:
 //   Format A: y[b][n] = sum_p sum_g s_p[n][g] sum_{j in g} t_p[n][j] x[b][j]
 //             (precisit.com page, "Three values and a shared scale"; second
 //             plane per the FUCINA README, "The method")
@@ -9,8 +10,8 @@
 // One CTA computes a 128-row tile of y^T over the whole of K (or a cluster
 // slice of it) for N = batch rounded up to 16 (<= 64), accumulating in tensor
 // memory (128 lanes x N fp32 columns). Per 64-wide K block (and per plane):
-//   - 8 decoder warps (two per TMEM lane quarter; a thread owns one row and
-//     half of the block's k) turn the codes of their rows into bf16 operands
+//   - 16 decoder warps (four per TMEM lane quarter; a thread owns one row
+//     and 16 k of the block) turn the codes of their rows into bf16 operands
 //     and write them straight into tensor memory with tcgen05.st: the A
 //     operand never passes through shared memory, whose bandwidth then only
 //     carries the code-book lookups. Each weight w is split into
@@ -18,7 +19,10 @@
 //     products exact to ~2^-16 relative, well inside the 2e-3 tolerance, with
 //     bf16 x used as is. For Format A, s*t splits exactly (an fp16 scale has
 //     11 significant bits: 8 in s_hi, 3 in s_lo). The x tile is staged in
-//     shared memory (operand B, K-major canonical layout).
+//     shared memory (operand B, K-major canonical layout). x and Format B
+//     codes arrive through per-thread cp.async rings; Format A codes and
+//     scales arrive in coalesced windows of 8 blocks that all decoders fetch
+//     together (completion and reuse on mbarriers).
 //   - One thread issues the 2 x 4 MMAs (M=128, N, K=16; A from tensor
 //     memory, B from shared memory) of the block and commits them to the
 //     stage's mbarrier, which frees the stage for the decoders. Tensor memory
