@@ -436,6 +436,17 @@ __global__ void __launch_bounds__(TcCfg<FMT>::kThreads, 1)
     uint32_t w_row = 0, c_off0 = 0, s_off0 = 0;  // its row base and offsets
     int s = 0, cur = 0;    // stage of block it, its x / code ring slot
     uint32_t e_par = 1;    // parity of the stage's previous use (from round 1)
+    // A block's TMEM stores complete while the next block decodes: its
+    // tcgen05.wait::st and full-barrier arrive come one iteration later.
+    int s_prev = 0;
+    bool pending = false;  // the previous block still awaits its arrive
+    auto arrive_prev = [&]() {
+      tmem_st_wait();
+      tc_fence_before_sync();  // A stores -> ordered before the arrive
+      __syncwarp();
+      if (lane == 0) mbar_arrive(full0 + 8 * s_prev);
+      pending = false;
+    };
     // Every decision before a warp-wide (.sync.aligned) instruction is made
     // uniform across the warp.
     for (int it = 0; it < iters && !__any_sync(0xFFFFFFFFu, abort_flag != 0);
@@ -519,6 +530,7 @@ __global__ void __launch_bounds__(TcCfg<FMT>::kThreads, 1)
           lo[4 * cc + q] = l4[q];
         }
       }
+      if (pending) arrive_prev();
       if (it >= kStages) {
         const bool ok = mbar_wait(empty0 + 8 * s, e_par);
         if (!__all_sync(0xFFFFFFFFu, ok)) {
@@ -533,7 +545,6 @@ __global__ void __launch_bounds__(TcCfg<FMT>::kThreads, 1)
                             (uint32_t)(kKPT / 2) * (uint32_t)kp;
         tmem_st_cols(ta, hi);
         tmem_st_cols(ta + 32, lo);
-        tmem_st_wait();
       }
       uint8_t *st = smem + P.ring_off + s * P.stage_bytes;
       // x tile: N rows x 64 k, 16 bytes per chunk, from this thread's ring
@@ -553,15 +564,15 @@ __global__ void __launch_bounds__(TcCfg<FMT>::kThreads, 1)
         }
       }
       fence_async_shared();   // x tile -> async proxy (MMA operand B)
-      tc_fence_before_sync();  // A stores -> ordered before the arrive
-      __syncwarp();
-      if (lane == 0) mbar_arrive(full0 + 8 * s);
+      s_prev = s;
+      pending = true;
       if (++s == kStages) {
         s = 0;
         e_par ^= 1u;
       }
       cur = cur + 1 == kCodeDepth ? 0 : cur + 1;
     }
+    if (pending) arrive_prev();
     cp_async_wait<0>();
     // ---- epilogue: warps of the first half read their TMEM lane quarter ----
     if (kp == 0) {
