@@ -119,7 +119,8 @@ tq_status tq_build_lut(float alpha, const float ladder[5], float lut_out[256]);
  *   planes      1 or 2. Plane 2 quantizes R = fp32(W - s1 t1) with the same G.
  *   codes_out   device, planes * n * (k/G) * ceil(G/5) bytes, dense planar
  *               layout, 16-byte aligned.
- *   scales_out  device, planes * n * (k/G) fp16, 4-byte aligned.
+ *   scales_out  device, planes * n * (k/G) fp16, 4-byte aligned (tq_linear
+ *               takes Format A scales 16-byte aligned: allocate for that).
  *   dev_status  device int32 or NULL: TQ_ERR_NONFINITE / TQ_ERR_RANGE.
  * Each group: S = sum |W_j| in fp64 over ascending j, s = fp16_RNE(S / G),
  * t_j = 0 if s == 0 else sign(W_j) [|W_j| > s/2]. Deterministic. */
