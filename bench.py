@@ -1,18 +1,20 @@
 """Benchmark of the packed ternary matmul library on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl tq|reference]
-                    [--workload NAME]
+                    [--workload NAME] [--batch B ...]
 
 Metric: effective weight GB/s (packed bytes the fused matmul must read: codes,
-scales, code book) and % of measured HBM peak. One step is one pass of the hot
-path over one batch of synthetic input for the chosen workload (default
-`fmt_b_4096`: Format B 4096 x 4096 layers, ladder 3^-(k-1), alpha 0.02, no
-rho, x at batch 1 and at batch 4). Distinct layer copies rotate so that no
-timed launch re-reads codes from L2. Every step runs as CUDA-graph replays of
+scales, code book) and % of measured HBM peak, batch 1-64. One step is one
+pass of the hot path over one batch of synthetic input for the chosen
+workload. The default, `decode_step`, is the 60-block decode step of
+Gemma-4-31B-shaped Format B linear layers (q, k, v 8192 x 5376; o 5376 x
+8192; gate, up 21504 x 5376; down 5376 x 21504; 31.4 GB of codes resident) at
+batch 1, 4, 16 and 64: one CUDA graph of the 420 ordered tq_linear calls per
+batch, all four graphs in every step. Every step runs as CUDA-graph replays of
 the library's C-ABI calls, timed with CUDA events on the launching stream.
 
-`--impl reference` times the CPU oracle (single thread) on a bounded sample of
-the same workload and prints the same JSON line with "impl": "reference".
+`--impl reference` times the CPU oracle (all host cores) on a bounded sample
+of the same workload and prints the same JSON line with "impl": "reference".
 Multi-GPU (torchrun): independent replicas, one per GPU, no data-path
 collective; timing is the max over ranks.
 """
@@ -271,11 +273,12 @@ class FmtB4096(Workload):
         self.xb_h = {b: I.bits(I.x_normal(b, self.K, 20 + b))
                      for b in self.BATCHES}
 
-    def oracle_pass(self, rows):
-        """One oracle pass over `rows` rows at every batch; returns bytes."""
-        for b in self.BATCHES:
-            self.oref.linear_B(self.codes_h[:rows], self.lut_h, self.xb_h[b])
-        return len(self.BATCHES) * rows * self.K
+    def oracle_jobs(self, rows, r0=0):
+        """Independent oracle calls of one pass over rows [r0, r0 + rows) at
+        every batch: (callable, algorithmic bytes)."""
+        c = self.codes_h[r0:r0 + rows]
+        return [(lambda b=b: self.oref.linear_B(c, self.lut_h, self.xb_h[b]),
+                 len(c) * self.K) for b in self.BATCHES]
 
     def sample_desc(self, rows):
         return (f"{rows} of {self.N} rows of one {self.N}x{self.K} layer at "
@@ -345,11 +348,12 @@ class FmtBGemma(Workload):
         self.xb_h = {b: I.bits(I.x_normal(b, self.K, 30 + b))
                      for b in self.BATCHES}
 
-    def oracle_pass(self, rows):
-        for b in self.BATCHES:
-            self.oref.linear_B(self.codes_h[:rows], self.lut_h, self.xb_h[b],
-                               self.rho_h, 1)
-        return len(self.BATCHES) * rows * self.K
+    def oracle_jobs(self, rows, r0=0):
+        c = self.codes_h[r0:r0 + rows]
+        rho = self.rho_h[r0:r0 + rows]
+        return [(lambda b=b: self.oref.linear_B(
+            c, self.lut_h, self.xb_h[b], rho, 1), len(c) * self.K)
+            for b in self.BATCHES]
 
     def sample_desc(self, rows):
         return (f"{rows} of 21504 rows of the up layer (21504x5376, rho per "
@@ -417,16 +421,21 @@ class FmtALarge(Workload):
         self.xb_h = {b: I.bits(I.x_normal(b, self.K, 40 + b))
                      for b in self.BATCHES}
 
-    def oracle_pass(self, rows):
-        rows = min(rows, 64)
-        codes, scales = self.oref.quantize_pack_A(self.Wh[:rows], self.G, 2)
-        nbytes = 2 * rows * self.K + 2 * rows * (self.K // self.G) * 15
+    def oracle_jobs(self, rows, r0=0):
+        rows = max(0, min(rows, 64 - r0))
+        codes, scales = self.pkg
+        codes = codes[:, r0:r0 + rows]
+        scales = scales[:, r0:r0 + rows]
+        Wr = self.Wh[r0:r0 + rows]
+        plane = rows * (self.K // self.G) * 15
+        jobs = [(lambda: self.oref.quantize_pack_A(Wr, self.G, 2),
+                 2 * rows * self.K + 2 * plane)]
         for p in (1, 2):
             for b in self.BATCHES:
-                self.oref.linear_A(codes[:p], scales[:p], rows, self.K,
-                                   self.xb_h[b], self.G, p)
-                nbytes += p * rows * (self.K // self.G) * 15
-        return nbytes
+                jobs.append((lambda p=p, b=b: self.oref.linear_A(
+                    codes[:p], scales[:p], rows, self.K, self.xb_h[b], self.G,
+                    p), p * plane))
+        return jobs
 
     def sample_desc(self, rows):
         return (f"{min(rows, 64)} rows x 8192 of the Format A workload: "
@@ -437,26 +446,32 @@ class FmtALarge(Workload):
 class DecodeStep(Workload):
     """60 blocks x {q, k, v 8192x5376; o 5376x8192; gate, up 21504x5376; down
     5376x21504} Format B layers (31.4 GB of codes), alpha 0.02, no rho, one
-    x per distinct k, at one batch (--batch, default 1). One step = the 420
-    ordered tq_linear calls; tokens/s = batch / step time."""
+    x per distinct k and batch. One step = the 420 ordered tq_linear calls at
+    every batch of `batches` (one CUDA graph per batch); tokens/s of a batch
+    = batch / its graph time. The step's result read back in the end-to-end
+    leg is the last layer's output at every batch."""
     name = "decode_step"
     SOURCES = Workload.SOURCES
     MAX_ROWS = 256
 
-    def __init__(self, batch=1, blocks=I.GEMMA_BLOCKS):
-        self.batch = batch
+    def __init__(self, batches=I.DECODE_BATCHES, blocks=I.GEMMA_BLOCKS):
+        self.BATCHES = tuple(batches)
         self.blocks = blocks
-        self.BATCHES = (batch,)
 
     def describe(self):
+        bs = ", ".join(map(str, self.BATCHES))
         return {"workload": f"{self.name}: {self.blocks} blocks x 7 Format B "
                 "layers (q,k,v 8192x5376; o 5376x8192; gate,up 21504x5376; "
-                "down 5376x21504), codes uniform 0..242, alpha=0.02, no rho; "
-                f"x bf16 N(0,1) at batch {self.batch}",
+                "down 5376x21504), codes uniform 0..242, ladder "
+                "a_k=3^-(k-1), alpha=0.02, no rho; x bf16 N(0,1); one graph "
+                f"of the {7 * self.blocks} ordered layers per batch, batch "
+                f"{bs}",
+                "layers": 7 * self.blocks,
                 "bytes_resident": sum(l.n * l.k for _, l in
                                       I.decode_step_layers(self.blocks)),
-                "l2": "31.4 GB resident: every launch reads from HBM",
-                "batches": [self.batch], "parallelism": "replicas"}
+                "l2": "31.4 GB of codes resident (250x L2): every launch "
+                      "streams its layer from HBM",
+                "batches": list(self.BATCHES), "parallelism": "replicas"}
 
     def setup(self, tq, dev):
         lut = tq.tq_build_lut(I.ALPHA, I.ladder_pow3().numpy())
@@ -466,21 +481,38 @@ class DecodeStep(Workload):
                       for s, l in self.layers]
         self.w = [tq.weights_b(c, self.lut_d) for c in self.codes]
         ks = sorted({l.k for _, l in self.layers})
-        self.x = {k: I.x_normal(self.batch, k, 50 + k % 97).to(dev)
-                  for k in ks}
-        self.y = [torch.zeros(self.batch, l.n, device=dev)
-                  for _, l in self.layers]
-        self.pin_io(list(self.x.values()), self.y)
+        self.x = {(b, k): I.x_normal(b, k, 50 + b).to(dev)
+                  for b in self.BATCHES for k in ks}
+        # one output buffer per (batch, position in the block): layers are
+        # not chained, the last layer's output is the step's result
+        self.y = {(b, j): torch.zeros(b, l.n, device=dev)
+                  for b in self.BATCHES
+                  for j, l in enumerate(I.BLOCK_LAYERS)}
+        last = len(I.BLOCK_LAYERS) - 1
+        self.pin_io(list(self.x.values()),
+                    [self.y[(b, last)] for b in self.BATCHES])
+
+    def step_bytes(self):
+        return sum(l.n * l.k + 972 for _, l in self.layers)
 
     def capture(self, tq):
-        calls = [lambda i=i, l=l: tq.tq_linear(self.w[i], self.x[l.k],
-                                                self.y[i])
-                 for i, (_, l) in enumerate(self.layers)]
-        nbytes = sum(l.n * l.k + 972 for _, l in self.layers)
-        return [Step(f"batch{self.batch}", capture_graph(calls), nbytes,
-                     len(calls), f"linear_b_decode_batch{self.batch}",
-                     2.0 * self.batch * sum(l.n * l.k for _, l in
-                                            self.layers))]
+        steps = []
+        nl = len(I.BLOCK_LAYERS)
+        for b in self.BATCHES:
+            calls = [lambda i=i, l=l, b=b: tq.tq_linear(
+                self.w[i], self.x[(b, l.k)], self.y[(b, i % nl)])
+                for i, (_, l) in enumerate(self.layers)]
+            steps.append(Step(f"batch{b}", capture_graph(calls),
+                              self.step_bytes(), len(calls),
+                              f"linear_b_decode_batch{b}",
+                              2.0 * b * sum(l.n * l.k for _, l in
+                                            self.layers)))
+        return steps
+
+    def extra(self, steps, per_ms):
+        """tokens/s per batch: batch / the time of its 420-layer graph."""
+        return {"tokens_per_s": {f"batch{b}": b / (p / 1e3)
+                                 for b, p in zip(self.BATCHES, per_ms)}}
 
     def oracle_setup(self):
         from oracle import oref
@@ -488,20 +520,128 @@ class DecodeStep(Workload):
         self.sample = [(l, I.codes_uniform(256, l.k, s).numpy())
                        for s, l in I.decode_step_layers(1)]
         self.lut_h = oref.build_lut(I.ALPHA, I.ladder_pow3().numpy())
-        self.xb = {l.k: I.bits(I.x_normal(self.batch, l.k, 1))
-                   for l, _ in self.sample}
+        self.xb = {(b, l.k): I.bits(I.x_normal(b, l.k, 50 + b))
+                   for b in self.BATCHES for l, _ in self.sample}
 
-    def oracle_pass(self, rows):
-        rows = min(rows, 256)
-        nbytes = 0
-        for l, codes in self.sample:
-            self.oref.linear_B(codes[:rows], self.lut_h, self.xb[l.k])
-            nbytes += rows * l.k
-        return nbytes
+    def oracle_jobs(self, rows, r0=0):
+        """Independent oracle calls of one pass over rows [r0, r0 + rows) of
+        each of the 7 layer shapes of one block, at every batch: (callable,
+        bytes)."""
+        rows = max(0, min(rows, 256 - r0))
+        jobs = []
+        for b in self.BATCHES:
+            for l, codes in self.sample:
+                jobs.append((lambda c=codes[r0:r0 + rows],
+                             x=self.xb[(b, l.k)]:
+                             self.oref.linear_B(c, self.lut_h, x),
+                             rows * l.k))
+        return jobs
 
     def sample_desc(self, rows):
         return (f"{min(rows, 256)} rows of each of the 7 layer shapes of one "
-                f"block at batch {self.batch}")
+                f"block at batch {', '.join(map(str, self.BATCHES))}")
+
+
+class Layer(Workload):
+    """One layer shape on its own (`--fmt`, `--n`, `--k`, `--planes`,
+    `--batch`): Format B codes uniform on 0..242 with the 3^-(k-1) ladder
+    (alpha 0.02, no rho), or a Format A package (G = 64) quantized on the GPU
+    from bf16 0.02*StudentT(5) weights; x bf16 N(0,1). Enough distinct copies
+    of the package rotate that they exceed 3x L2. Used for per-kernel
+    profiles and sweeps."""
+    name = "layer"
+    MAX_ROWS = 256
+
+    def __init__(self, fmt="B", n=8192, k=5376, batches=(1,), planes=1):
+        self.fmt, self.n, self.k = fmt.upper(), n, k
+        self.BATCHES = tuple(batches)
+        self.planes = planes
+        if self.fmt == "A":
+            self.pkg = planes * n * (k // 64) * 15
+        else:
+            self.pkg = n * k + 972
+        self.copies = max(1, -(-3 * L2_BYTES // self.pkg))
+
+    def describe(self):
+        what = (f"Format A {self.n}x{self.k}, G=64, {self.planes} plane(s), "
+                "quantized from bf16 0.02*StudentT(5)" if self.fmt == "A" else
+                f"Format B {self.n}x{self.k}, codes uniform 0..242, ladder "
+                "a_k=3^-(k-1), alpha=0.02, no rho")
+        return {"workload": f"{self.name}: {what}; x bf16 N(0,1) at batch "
+                f"{', '.join(map(str, self.BATCHES))}",
+                "layers_rotated": self.copies,
+                "bytes_resident": self.copies * self.pkg,
+                "l2": "rotating distinct copies, resident bytes > 3x L2",
+                "batches": list(self.BATCHES), "parallelism": "replicas"}
+
+    def setup(self, tq, dev):
+        n, k = self.n, self.k
+        if self.fmt == "A":
+            W = I.student_t_bf16(n, k, seed=3).to(dev)
+            nb = self.planes * n * (k // 64)
+            c0 = torch.empty(nb * 13, dtype=torch.uint8, device=dev)
+            s0 = torch.empty(nb + 8, dtype=torch.int16, device=dev)
+            st = torch.zeros(1, dtype=torch.int32, device=dev)
+            tq.tq_quantize_pack(W, 64, self.planes, c0, s0, st)
+            del W
+            self.keep = [(c0.clone(), s0.clone()) for _ in range(self.copies)]
+            self.w = [tq.weights_a(c, s, n, k, 64, self.planes)
+                      for c, s in self.keep]
+        else:
+            lut = tq.tq_build_lut(I.ALPHA, I.ladder_pow3().numpy())
+            self.lut_d = torch.from_numpy(lut).to(dev)
+            self.keep = [I.codes_uniform(n, k, 5 + i, device=dev)
+                         for i in range(self.copies)]
+            self.w = [tq.weights_b(c, self.lut_d) for c in self.keep]
+        self.x = {b: I.x_normal(b, k, 60 + b).to(dev) for b in self.BATCHES}
+        self.y = {b: torch.zeros(b, n, device=dev) for b in self.BATCHES}
+        self.pin_io(list(self.x.values()), list(self.y.values()))
+
+    def capture(self, tq):
+        steps = []
+        for b in self.BATCHES:
+            calls = [lambda i=i, b=b: tq.tq_linear(self.w[i], self.x[b],
+                                                   self.y[b])
+                     for i in range(self.copies)]
+            steps.append(Step(f"batch{b}", capture_graph(calls),
+                              self.copies * self.pkg, self.copies,
+                              f"linear_{self.fmt.lower()}_layer_batch{b}",
+                              2.0 * b * self.planes * self.n * self.k *
+                              self.copies))
+        return steps
+
+    def oracle_setup(self):
+        from oracle import oref
+        self.oref = oref
+        rows = 256
+        if self.fmt == "A":
+            Wh = I.bits(I.student_t_bf16(rows, self.k, seed=3))
+            self.pkg_h = oref.quantize_pack_A(Wh, 64, self.planes)
+        else:
+            self.codes_h = I.codes_uniform(rows, self.k, 5).numpy()
+            self.lut_h = oref.build_lut(I.ALPHA, I.ladder_pow3().numpy())
+        self.xb = {b: I.bits(I.x_normal(b, self.k, 60 + b))
+                   for b in self.BATCHES}
+
+    def oracle_jobs(self, rows, r0=0):
+        rows = max(0, min(rows, 256 - r0))
+        jobs = []
+        for b in self.BATCHES:
+            if self.fmt == "A":
+                c, s = self.pkg_h
+                c, s = c[:, r0:r0 + rows], s[:, r0:r0 + rows]
+                jobs.append((lambda b=b, c=c, s=s: self.oref.linear_A(
+                    c, s, rows, self.k, self.xb[b], 64, self.planes),
+                    self.planes * rows * (self.k // 64) * 15))
+            else:
+                c = self.codes_h[r0:r0 + rows]
+                jobs.append((lambda b=b, c=c: self.oref.linear_B(
+                    c, self.lut_h, self.xb[b]), rows * self.k))
+        return jobs
+
+    def sample_desc(self, rows):
+        return (f"{min(rows, 256)} rows of the {self.n}x{self.k} layer at "
+                f"batch {', '.join(map(str, self.BATCHES))}")
 
 
 class FmtASmall(Workload):
@@ -545,45 +685,122 @@ class FmtASmall(Workload):
         cfg = I.fmt_a_small()
         self.Wh = I.bits(cfg["W"])
         self.xb = I.bits(cfg["x"])
+        self.pkg = oref.quantize_pack_A(self.Wh, 64, 1)
 
-    def oracle_pass(self, rows):
-        rows = min(rows, 512)
-        codes, scales = self.oref.quantize_pack_A(self.Wh[:rows], 64, 1)
-        self.oref.linear_A(codes, scales, rows, 1024, self.xb)
-        return rows * 1024 * 2 + 2 * rows * 16 * 15
+    def oracle_jobs(self, rows, r0=0):
+        rows = max(0, min(rows, 512 - r0))
+        codes, scales = self.pkg
+        codes, scales = codes[:, r0:r0 + rows], scales[:, r0:r0 + rows]
+        Wr = self.Wh[r0:r0 + rows]
+        return [(lambda: self.oref.quantize_pack_A(Wr, 64, 1),
+                 rows * 1024 * 2 + rows * 16 * 15),
+                (lambda: self.oref.linear_A(codes, scales, rows, 1024,
+                                            self.xb), rows * 16 * 15)]
 
     def sample_desc(self, rows):
         return f"{min(rows, 512)} rows of the 512x1024 workload"
 
 
 def make_workload(args):
+    batches = tuple(args.batch) if args.batch else None
     if args.workload == "decode_step":
-        return DecodeStep(batch=args.batch)
+        return DecodeStep(batches=batches or I.DECODE_BATCHES)
+    if args.workload == "layer":
+        return Layer(args.fmt, args.n, args.k, batches or (1,), args.planes)
     return WORKLOADS[args.workload]()
 
 
 WORKLOADS = {"fmt_b_4096": FmtB4096, "fmt_b_gemma": FmtBGemma,
              "fmt_a_large": FmtALarge, "decode_step": DecodeStep,
-             "fmt_a_small": FmtASmall}
+             "fmt_a_small": FmtASmall, "layer": Layer}
 
 
-# ---- the two arms ------------------------------------------------------------------------
+# ---- the oracle on the host cores ---------------------------------------------------
 
-def time_oracle(wl, seconds):
-    """Time the single-threaded oracle for about `seconds` on whole passes."""
-    wl.oracle_setup()
-    rows = 64
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def host_threads():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+class OracleRunner:
+    """Runs one pass of a workload's oracle sample: on one thread, or with
+    the sample's rows split across `threads` host threads (the oracle's C
+    calls release the GIL; rows are independent, so the results are the
+    same)."""
+
+    def __init__(self, wl, threads):
+        import concurrent.futures as cf
+        self.wl, self.threads = wl, threads
+        self.pool = cf.ThreadPoolExecutor(threads) if threads > 1 else None
+
+    def run(self, rows):
+        """One pass over `rows` rows of the sample; returns its bytes."""
+        if self.pool is None:
+            jobs = self.wl.oracle_jobs(rows, 0)
+            for f, _ in jobs:
+                f()
+            return sum(nb for _, nb in jobs)
+        per = max(1, rows // self.threads)
+        jobs = []
+        for r0 in range(0, rows, per):
+            jobs += self.wl.oracle_jobs(min(per, rows - r0), r0)
+        for fut in [self.pool.submit(f) for f, _ in jobs]:
+            fut.result()
+        return sum(nb for _, nb in jobs)
+
+    def close(self):
+        if self.pool is not None:
+            self.pool.shutdown()
+
+
+def time_oracle(wl, seconds, threads):
+    """Time the oracle on whole passes for about `seconds`: returns (bytes,
+    seconds, rows per pass, passes)."""
+    runner = OracleRunner(wl, threads)
+    rows = min(wl.MAX_ROWS, 8 * threads)
     t0 = time.perf_counter()
-    wl.oracle_pass(rows)
+    runner.run(rows)
     dt = time.perf_counter() - t0
     rows = int(max(1, min(wl.MAX_ROWS, rows * seconds / max(dt, 1e-6) / 4)))
     total_bytes, t_total, passes = 0, 0.0, 0
     while t_total < seconds:
         t0 = time.perf_counter()
-        total_bytes += wl.oracle_pass(rows)
+        total_bytes += runner.run(rows)
         t_total += time.perf_counter() - t0
         passes += 1
+    runner.close()
     return total_bytes, t_total, rows, passes
+
+
+def cpu_baseline(wl, seconds):
+    """The oracle as it stands, timed on the host: one thread, then all the
+    threads this process may run on. The all-threads leg is the value."""
+    wl.oracle_setup()
+    legs = {}
+    for name, threads in (("single_thread", 1), ("all_cores", host_threads())):
+        nbytes, secs, rows, passes = time_oracle(wl, seconds, threads)
+        legs[name] = {"value": nbytes / secs / 1e9, "cores": threads,
+                      "sample": f"{passes} passes over " + wl.sample_desc(rows)
+                                + f" ({secs:.1f} s, {threads} thread(s))"}
+    top = legs["all_cores"]
+    return {"value": top["value"], "unit": "GB/s", "cores": top["cores"],
+            "kind": "oracle", "sample": top["sample"],
+            "single_thread": legs["single_thread"],
+            "cpu_model": cpu_model(),
+            "hardware_concurrency": os.cpu_count()}
 
 
 def run_reference(args, world, rank):
@@ -591,28 +808,33 @@ def run_reference(args, world, rank):
         return
     wl = make_workload(args)
     wl.oracle_setup()
-    # size each step so the whole run ends within about two minutes
+    threads = host_threads()
+    runner = OracleRunner(wl, threads)
+    # size each step so that the whole run ends within args.ref_seconds
+    probe = min(wl.MAX_ROWS, 4 * threads)
     t0 = time.perf_counter()
-    wl.oracle_pass(16)
-    per_row = (time.perf_counter() - t0) / 16
+    runner.run(probe)
+    per_row = (time.perf_counter() - t0) / probe
     budget = args.ref_seconds / max(1, args.steps + args.warmup)
     rows = int(max(1, min(wl.MAX_ROWS, budget / max(per_row, 1e-9))))
     for _ in range(args.warmup):
-        wl.oracle_pass(rows)
+        runner.run(rows)
     t0 = time.perf_counter()
     nbytes = 0
     for _ in range(args.steps):
-        nbytes += wl.oracle_pass(rows)
+        nbytes += runner.run(rows)
     dt = time.perf_counter() - t0
+    runner.close()
     value = nbytes / dt / 1e9
-    sample = wl.sample_desc(rows) + " per step"
+    sample = wl.sample_desc(rows) + f" per step, {threads} host thread(s)"
     line = {"impl": "reference", "metric": METRIC, "value": value,
             "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64", "data": "synthetic", "config": wl.describe(),
-            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1,
-                             "kind": "oracle", "sample": sample},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads,
+                             "kind": "oracle", "sample": sample,
+                             "cpu_model": cpu_model()},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -685,10 +907,6 @@ def run_tq(args, world, rank, local):
     # dominant kernel: the graph with the largest share of the step
     dom = int(np.argmax(per))
     s = steps[dom]
-    per_launch_s = per[dom] / 1e3 / s.launches
-    bytes_per_launch = s.bytes / s.launches
-    achieved = bytes_per_launch / per_launch_s / 1e9
-    traffic = ncu_traffic(s.kernel, wl.SOURCES, 1)
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
@@ -696,44 +914,74 @@ def run_tq(args, world, rank, local):
         "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic", "config": wl.describe(),
         "pct_hbm_peak": 100.0 * value / world / pk["hbm_gbs"],
-        "roofline": {"bound": "hbm", "achieved": achieved,
-                     "peak": pk["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved / pk["hbm_gbs"],
-                     "traffic": traffic, "kernel": s.kernel,
-                     "peak_src": pk["src"],
-                     "algorithmic_bytes_per_launch": bytes_per_launch},
+        "roofline": roofline(s, per[dom], pk, wl),
         "per_graph_ms": {st.name: float(p) for st, p in zip(steps, per)},
         "per_graph_gbs": {st.name: st.bytes / (p / 1e3) / 1e9
                           for st, p in zip(steps, per)},
+        "per_graph_roof_frac": {st.name: roofline(st, p, pk, wl)["frac"]
+                                for st, p in zip(steps, per)},
         "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "clocks": clk,
         "gpu_launches": int(sum(st.launches for st in steps) * args.steps),
     }
-    if isinstance(wl, DecodeStep):
-        line["tokens_per_s"] = world * wl.batch * args.steps / (elapsed_ms / 1e3)
-        line["e2e_tokens_per_s"] = world * wl.batch * args.steps / (e2e_ms / 1e3)
+    if hasattr(wl, "extra"):
+        line.update(wl.extra(steps, per))
     if world == 1 and not args.no_cpu_baseline:
-        nbytes, secs, rows, passes = time_oracle(wl, args.cpu_seconds)
-        line["cpu_baseline"] = {
-            "value": nbytes / secs / 1e9, "unit": "GB/s", "cores": 1,
-            "kind": "oracle",
-            "sample": f"{passes} passes over " + wl.sample_desc(rows) +
-                      f" "
-                      f"({secs:.1f} s, single thread)"}
+        line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
     print(json.dumps(line), flush=True)
+
+
+def roofline(step, ms, pk, wl):
+    """Roofline of one graph's kernel: achieved = its algorithmic bytes (or
+    flops) per launch / its average CUDA-event launch time, against the lower
+    of the HBM roof (measured copy bandwidth) and the tensor roof (sustained
+    dense bf16 throughput, expressed in packed bytes through the graph's
+    flops per byte)."""
+    per_launch_s = ms / 1e3 / step.launches
+    bytes_per_launch = step.bytes / step.launches
+    flops_per_launch = step.flops / step.launches
+    hbm = pk["hbm_gbs"]
+    tensor_tflops = pk["bf16_tflops_sustained"]
+    tensor_gbs = (tensor_tflops * 1e12 * bytes_per_launch / flops_per_launch
+                  / 1e9 if flops_per_launch > 0 else float("inf"))
+    traffic = ncu_traffic(step.kernel, wl.SOURCES, bytes_per_launch)
+    out = {"traffic": traffic, "kernel": step.kernel, "peak_src": pk["src"],
+           "algorithmic_bytes_per_launch": bytes_per_launch,
+           "algorithmic_flops_per_launch": flops_per_launch,
+           "launch_us": per_launch_s * 1e6}
+    if tensor_gbs < hbm:
+        achieved = flops_per_launch / per_launch_s / 1e12
+        out.update({"bound": "tensor", "achieved": achieved,
+                    "peak": tensor_tflops, "unit": "TFLOP/s",
+                    "frac": achieved / tensor_tflops,
+                    "peak_kind": "dense bf16, sustained"})
+    else:
+        achieved = bytes_per_launch / per_launch_s / 1e9
+        out.update({"bound": "hbm", "achieved": achieved, "peak": hbm,
+                    "unit": "GB/s", "frac": achieved / hbm,
+                    "peak_kind": "HBM copy"})
+    return out
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["tq", "reference"], default="tq")
     ap.add_argument("--workload", choices=sorted(WORKLOADS),
-                    default="fmt_b_4096")
-    ap.add_argument("--batch", type=int, default=1,
-                    help="batch of the decode_step workload")
+                    default="decode_step")
+    ap.add_argument("--batch", type=int, nargs="+", default=None,
+                    help="batches of the decode_step and layer workloads "
+                         "(default 1 4 16 64 and 1)")
+    ap.add_argument("--fmt", choices=["A", "B", "a", "b"], default="B",
+                    help="layer workload: weight format")
+    ap.add_argument("--n", type=int, default=8192, help="layer workload: rows")
+    ap.add_argument("--k", type=int, default=5376,
+                    help="layer workload: columns")
+    ap.add_argument("--planes", type=int, default=1,
+                    help="layer workload: Format A planes")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-seconds", type=float, default=90.0,

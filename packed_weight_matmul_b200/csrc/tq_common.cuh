@@ -1,6 +1,8 @@
 // Shared declarations of the tq CUDA library (sm_100a).
 #pragma once
 
+#include <atomic>
+
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -32,6 +34,26 @@ struct WeightsView {
   int64_t codes_plane_stride;   // bytes
   int64_t scales_plane_stride;  // elements
 };
+
+// Raise a kernel's dynamic shared-memory limit to `bytes` once per device.
+// The attribute is one value per function and context; every caller asks for
+// the same (largest) value, so concurrent callers cannot lower it under one
+// another's launch. Occupancy follows each launch's own request.
+template <auto Kern>
+cudaError_t ensure_smem_limit(int bytes) {
+  static std::atomic<uint64_t> done{0};  // bit d: set on device d (< 64)
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = dev < 64 ? 1ull << dev : 0ull;
+  if (bit != 0 && (done.load(std::memory_order_acquire) & bit) != 0)
+    return cudaSuccess;
+  e = cudaFuncSetAttribute(Kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           bytes);
+  if (e == cudaSuccess && bit != 0)
+    done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
 
 // ---- launchers (each enqueues on `stream`, returns the launch error) ----
 cudaError_t launch_quantize_pack(const uint16_t *W, int64_t n, int64_t k,

@@ -686,8 +686,8 @@ cudaError_t launch_tc(const WeightsView &w, const __nv_bfloat16 *x,
   const int iters = (FMT == TQ_FMT_A ? w.planes : 1) * kblocks;
   P.ks_count = pick_ks(tiles, iters, sms);
   auto kern = gemm_tc_kernel<FMT>;
-  cudaError_t e = cudaFuncSetAttribute(
-      kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P.smem);
+  if (P.smem > 227 * 1024) return cudaErrorInvalidValue;
+  cudaError_t e = ensure_smem_limit<gemm_tc_kernel<FMT>>(227 * 1024);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(tiles * P.ks_count), 1, 1);

@@ -310,12 +310,16 @@ int max_clusters(int dev, int ks, size_t smem) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  // An error already pending belongs to the caller: leave it for them and
+  // skip the query (the launcher then uses its SM-count fallback).
+  if (cudaPeekAtLastError() != cudaSuccess) return 0;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, gemv_a_kernel, &cfg) != cudaSuccess ||
-      n < 1) {
-    cudaGetLastError();
+  const cudaError_t q = cudaOccupancyMaxActiveClusters(&n, gemv_a_kernel, &cfg);
+  if (q != cudaSuccess) {
+    cudaGetLastError();  // clears only the query's own error
     return 0;
   }
+  if (n < 1) return 0;
   if (dev >= 0 && dev < 16) cache[dev][slot].store(n, std::memory_order_relaxed);
   return n;
 }
@@ -330,8 +334,7 @@ cudaError_t gemv_a(const WeightsView &w, const __nv_bfloat16 *x, float *y,
   GemvAParams P;
   P.ng = w.k / kG;
   const size_t big = 160 * 1024;  // any request of one CTA per SM
-  cudaError_t e = cudaFuncSetAttribute(
-      gemv_a_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMax);
+  cudaError_t e = ensure_smem_limit<gemv_a_kernel>(kSmemMax);
   if (e != cudaSuccess) return e;
   // K slices: at most 8 (portable cluster), at least one full window each.
   // Each CTA owns an SM; its time is about windows x (its rows' lookups +

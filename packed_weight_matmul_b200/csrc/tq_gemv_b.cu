@@ -428,9 +428,9 @@ cudaError_t launch_cfg(const WeightsView &w, const __nv_bfloat16 *x,
   const uint32_t red_bytes = (uint32_t)(nchunks * rows_max * B * 4);
   const uint32_t hi_ring = (kRedAddr + red_bytes + 127u) & ~127u;
   const size_t smem = hi_ring + (size_t)hi_warps * kRing;
+  if (smem > (size_t)kSmemMax) return cudaErrorInvalidValue;
   auto kern = gemv_b_kernel<B, R, D, NT, CM>;
-  cudaError_t e = cudaFuncSetAttribute(
-      kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = ensure_smem_limit<gemv_b_kernel<B, R, D, NT, CM>>(kSmemMax);
   if (e != cudaSuccess) return e;
   kern<<<(unsigned)ctas, NT, smem, stream>>>(w.codes, w.n, w.k, w.lut,
                                               w.scales, w.rps, x, ldx, y, ldy,
@@ -453,6 +453,18 @@ bool gemv_b_supported(const WeightsView &w, int64_t batch) {
 
 cudaError_t gemv_b(const WeightsView &w, const __nv_bfloat16 *x, int64_t batch,
                    int64_t ldx, float *y, int64_t ldy, cudaStream_t stream) {
+  // The kernel places its code book and rings at fixed shared-window
+  // addresses, which assumes the dynamic window starts at or below
+  // kRingLoAddr (the per-CTA reserved shared memory comes first). Refuse a
+  // device where it would not, instead of launching a kernel that could only
+  // write NaN.
+  int dev = 0, reserved = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock,
+                             dev);
+  if (e != cudaSuccess) return e;
+  if ((uint32_t)reserved > kRingLoAddr) return cudaErrorNotSupported;
   const int sms = device_sms();
   switch (batch) {
     case 1: return launch_cfg<1, 8, 2, 512, true>(w, x, ldx, y, ldy, sms, stream);

@@ -153,3 +153,63 @@ def test_unpack_b_rejects_bad_codes():
     lut = oref.build_lut(0.02, I.ladder_pow3().numpy())
     _, st = _unpack(U.weights_b_dev(codes, lut), 64, 64)
     assert st == oref.ERR_BAD_CODE
+
+
+# ---- tq_unpack at the workloads' full sizes ---------------------------------
+# The decoded bf16 weights must be bit-exact on every workload: a lossless
+# round trip ("Does your weight format deserve a kernel?", "Five trits in a
+# byte"). Inputs come from the oracle and the seeded generators only.
+
+def test_unpack_a_large_all_rows_two_planes_bit_exact(large):
+    W = large["W"]
+    n, k = W.shape
+    codes, scales = oref.quantize_pack_A(I.bits(W), 64, 2)
+    got, st = _unpack(U.weights_a_dev(codes, scales, n, k, 64, 2), n, k)
+    assert st == 0
+    assert np.array_equal(got, oref.unpack_A(codes, scales, n, k, 64, 2))
+    # plane 1 alone (the plane stride leaves plane 2 unread)
+    got1, st1 = _unpack(U.weights_a_dev(codes[:1], scales[:1], n, k, 64, 1),
+                        n, k)
+    assert st1 == 0
+    assert np.array_equal(got1, oref.unpack_A(codes[:1], scales[:1], n, k, 64,
+                                              1))
+
+
+def test_unpack_b_4096_bit_exact():
+    cfg = I.fmt_b_4096()
+    codes = cfg["codes"]
+    lut = oref.build_lut(cfg["alpha"], cfg["ladder"].numpy())
+    got, st = _unpack(U.weights_b_dev(codes, lut), 4096, 4096)
+    assert st == 0
+    assert np.array_equal(got, oref.unpack_B(codes.numpy(), lut))
+
+
+@pytest.mark.parametrize("layer", I.FMT_B_GEMMA_LAYERS,
+                         ids=lambda l: l.name)
+def test_unpack_b_gemma_layers_with_rho_bit_exact(layer):
+    cfg = I.fmt_b_gemma_layer(layer)
+    codes, rho, rps = cfg["codes"], cfg["rho"], cfg["rps"]
+    lut = oref.build_lut(cfg["alpha"], cfg["ladder"].numpy())
+    got, st = _unpack(U.weights_b_dev(codes, lut, rho, rps), layer.n, layer.k)
+    assert st == 0
+    ref = oref.unpack_B(codes.numpy(), lut, I.bits(rho), rps)
+    assert np.array_equal(got, ref)
+
+
+def _decode_step_shapes():
+    seen, out = set(), []
+    for seed, layer in I.decode_step_layers(1):
+        if (layer.n, layer.k) not in seen:
+            seen.add((layer.n, layer.k))
+            out.append((seed, layer))
+    return out
+
+
+@pytest.mark.parametrize("seed,layer", _decode_step_shapes(),
+                         ids=lambda v: getattr(v, "name", str(v)))
+def test_unpack_b_decode_step_layer_bit_exact(seed, layer):
+    codes = I.codes_uniform(layer.n, layer.k, seed)
+    lut = oref.build_lut(I.ALPHA, I.ladder_pow3().numpy())
+    got, st = _unpack(U.weights_b_dev(codes, lut), layer.n, layer.k)
+    assert st == 0
+    assert np.array_equal(got, oref.unpack_B(codes.numpy(), lut))
