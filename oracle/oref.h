@@ -116,6 +116,15 @@ int oref_linear_B(const uint8_t *codes, int64_t n, int64_t k, const float *lut,
                   int64_t nrows, const uint16_t *x, int64_t batch, int64_t ldx,
                   double *y);
 
+/* Encoder (section 3.1; per-row / per-head scale, section 3.3): the greedy
+ * 5-step ternary path of every weight over the ladder with zero-bias zeta,
+ * r_0 = W / a with a = alpha = max |W| (rps = 0) or a = max |W| over the
+ * rows n / rps (rps > 0, then rho[g] = fp16(a_g / alpha)). Decisions in fp32.
+ * codes [n][k]; rho [ceil(n / rps)] (rps > 0); *alpha_out = alpha. */
+int oref_encode_B(const uint16_t *W, int64_t n, int64_t k,
+                  const float ladder[5], float zeta, int32_t rps,
+                  uint8_t *codes, uint16_t *rho, float *alpha_out);
+
 #ifdef __cplusplus
 }
 #endif

@@ -87,6 +87,8 @@ def _declare(L):
     L.oref_unpack_B.argtypes = [P, i64, i64, P, P, i32, P]
     L.oref_weights_B.restype = C.c_int
     L.oref_weights_B.argtypes = [P, i64, i64, P, P, i32, P, i64, P]
+    L.oref_encode_B.restype = C.c_int
+    L.oref_encode_B.argtypes = [P, i64, i64, P, C.c_float, i32, P, P, P]
     L.oref_linear_B.restype = C.c_int
     L.oref_linear_B.argtypes = [P, i64, i64, P, P, i32, P, i64, P, i64, i64,
                                 P]
@@ -261,3 +263,17 @@ def linear_B(codes, lut, x_bits, rho=None, rps=0, rows=None, check=True,
                                     _p(rows), nr, _p(x), batch, ldx, _p(y))
     return _ret(y, st, check)
 
+
+
+def encode_B(W_bits, ladder, zeta=0.5, rps=0, check=True, L=None):
+    """W_bits: uint16 [n][k] bf16 patterns -> (codes uint8 [n][k],
+    rho uint16 [ceil(n / rps)] fp16 patterns or None, alpha float)."""
+    W = _c(W_bits, np.uint16)
+    n, k = W.shape
+    ladder = _c(ladder, np.float32)
+    codes = np.zeros((n, k), np.uint8)
+    rho = np.zeros(((n + rps - 1) // rps,), np.uint16) if rps > 0 else None
+    alpha = np.zeros(1, np.float32)
+    st = (L or lib()).oref_encode_B(_p(W), n, k, _p(ladder), C.c_float(zeta),
+                                    rps, _p(codes), _p(rho), _p(alpha))
+    return _ret((codes, rho, float(alpha[0])), st, check)

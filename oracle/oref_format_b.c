@@ -123,3 +123,96 @@ int oref_linear_B(const uint8_t *codes, int64_t n, int64_t k, const float *lut,
   free(w);
   return status;
 }
+
+/* ---- encoder (section 3.1 "Encoding", section 3.3 "Per-row scale") -------
+ *
+ * The page's greedy 5-step ternary path: with the residual r_0 = x / a, step
+ * i picks c_i in {-1, 0, +1} minimising |r_{i-1} - c s_i|, except that a
+ * zero-bias zeta prefers c_i = 0 when |r_{i-1}| < zeta s_i, and leaves the
+ * residual r_i = r_{i-1} - c_i s_i. The scale a is the global alpha =
+ * max |W| (section 3.1), or, with a per-row (or per-head) scale, the maximum
+ * |W| over the row (or the head's rows), alpha_n, with rho_n = alpha_n / alpha
+ * stored in fp16 (section 3.3).
+ *
+ * Readings where the page leaves a step open:
+ *   E1 precision: the page fixes none; every step that decides a digit runs
+ *      in IEEE fp32 in the order written here: r_0 = fp32(x / a); the zero
+ *      bias threshold is fp32(zeta * s_i); the non-zero candidate is the one
+ *      with the sign of r (the nearer of -1 and +1), taken only when
+ *      |fp32(r - c s_i)| < |r| strictly (a tie, and r = 0, give 0); then
+ *      r = fp32(r - c_i s_i);
+ *   E2 the scale group of row n is n / rows_per_scale (1: per row; the head
+ *      size: per head), one alpha_g and one rho per group, as the rho layout
+ *      of the matmul (B3); rows_per_scale = 0 uses the global alpha, no rho;
+ *   E3 rho_g = fp16(alpha_g / alpha): the fp64 quotient rounded once to fp16;
+ *   E4 a zero scale (an all-zero group, or an all-zero matrix) gives the
+ *      all-zero word (code 121) and rho = 0;
+ *   E5 alpha = max |W| is a bf16 magnitude, exact in fp32; NaN or Inf in W is
+ *      OREF_ERR_NONFINITE (the outputs are then unspecified).
+ */
+static uint8_t encode_word(float r, const float s[5], const float zs[5]) {
+  int code = 0, p3 = 1;
+  for (int i = 0; i < 5; ++i) { /* step i + 1 of the path */
+    int c = 0;
+    const float ar = fabsf(r);
+    if (!(ar < zs[i])) {
+      const int cand = r > 0.0f ? 1 : (r < 0.0f ? -1 : 0);
+      if (cand != 0) {
+        const float rn = r - (float)cand * s[i];
+        if (fabsf(rn) < ar) {
+          c = cand;
+          r = rn;
+        }
+      }
+    }
+    code += (c + 1) * p3; /* c_1 is the least significant digit (B1) */
+    p3 *= 3;
+  }
+  return (uint8_t)code;
+}
+
+int oref_encode_B(const uint16_t *W, int64_t n, int64_t k,
+                  const float ladder[5], float zeta, int32_t rps,
+                  uint8_t *codes, uint16_t *rho, float *alpha_out) {
+  if (!W || !ladder || !codes || !alpha_out || n < 0 || k < 0 || rps < 0)
+    return OREF_ERR_INVALID_ARG;
+  if (rps > 0 && !rho) return OREF_ERR_INVALID_ARG;
+  int status = OREF_OK;
+  /* alpha = max |W| over the whole matrix */
+  double amax = 0.0;
+  for (int64_t i = 0; i < n * k; ++i) {
+    const double v = fabs(oref_bf16_to_f64(W[i]));
+    if (!isfinite(v)) {
+      status = OREF_ERR_NONFINITE;
+      continue;
+    }
+    if (v > amax) amax = v;
+  }
+  const float alpha = (float)amax; /* exact (E5) */
+  *alpha_out = alpha;
+  float s[5], zs[5];
+  for (int i = 0; i < 5; ++i) {
+    s[i] = ladder[i];
+    zs[i] = zeta * ladder[i]; /* fp32 product (E1) */
+  }
+  const int64_t group_rows = rps > 0 ? rps : (n > 0 ? n : 1);
+  for (int64_t g0 = 0; g0 < n; g0 += group_rows) {
+    const int64_t g1 = g0 + group_rows < n ? g0 + group_rows : n;
+    float a = alpha;
+    if (rps > 0) {
+      double gmax = 0.0;
+      for (int64_t i = g0 * k; i < g1 * k; ++i) {
+        const double v = fabs(oref_bf16_to_f64(W[i]));
+        if (isfinite(v) && v > gmax) gmax = v;
+      }
+      a = (float)gmax;
+      rho[g0 / rps] = a == 0.0f ? 0 : oref_f64_to_f16((double)a / (double)alpha);
+    }
+    for (int64_t i = g0 * k; i < g1 * k; ++i) {
+      const float x = (float)oref_bf16_to_f64(W[i]);
+      const float r0 = a == 0.0f ? 0.0f : x / a; /* E1, E4 */
+      codes[i] = encode_word(r0, s, zs);
+    }
+  }
+  return status;
+}

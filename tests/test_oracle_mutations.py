@@ -51,6 +51,21 @@ MUTATIONS = {
     "dropped_rho_in_matmul": ("oref_format_b.c",
                               "w_out[i * k + j] = scale * (double)lut[c];",
                               "w_out[i * k + j] = (double)lut[c];"),
+    "encode_tie_to_nonzero": ("oref_format_b.c",
+                              "if (fabsf(rn) < ar) {", "if (fabsf(rn) <= ar) {"),
+    "encode_zero_bias_ignored": ("oref_format_b.c",
+                                 "if (!(ar < zs[i])) {", "if (1) {"),
+    "encode_residual_not_updated": ("oref_format_b.c",
+                                    "          r = rn;\n", "\n"),
+    "encode_digit_order_reversed": ("oref_format_b.c",
+                                    "code += (c + 1) * p3;",
+                                    "code += (c + 1) * (81 / p3);"),
+    "encode_rho_inverted": ("oref_format_b.c",
+                            "oref_f64_to_f16((double)a / (double)alpha)",
+                            "oref_f64_to_f16((double)alpha / (double)a)"),
+    "encode_global_scale_for_rows": ("oref_format_b.c",
+                                     "      a = (float)gmax;",
+                                     "      a = alpha;"),
     "round_ties_up": ("oref_fp.c",
                       "return (fmod(f, 2.0) == 0.0) ? f : f + 1.0;",
                       "return f + 1.0;"),

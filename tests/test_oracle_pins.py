@@ -399,3 +399,123 @@ def test_linear_B_brute_force(oref):
     assert np.array_equal(
         oref.linear_B(codes, lut, xb, rho.view(np.uint16), rps, rows=rows),
         y[:, rows])
+
+
+# ---- Format B encoder ("A Discrete Weight Language...", sections 3.1, 3.3) --
+
+def balanced_ternary_word(m):
+    """Digits d_1..d_5 in {-1, 0, 1} with m = sum d_i 3^(5-i) (integer
+    arithmetic, most significant first), |m| <= 121."""
+    d = []
+    for i in range(5):
+        p = 3 ** (4 - i)
+        q = int(round(m / p))
+        q = max(-1, min(1, q))
+        d.append(q)
+        m -= q * p
+    assert m == 0
+    return d
+
+
+def code_of_word(d):
+    return sum((di + 1) * 3 ** i for i, di in enumerate(d))
+
+
+def bf16_bits_of(values):
+    t = torch.tensor(values, dtype=torch.float32).to(torch.bfloat16)
+    return I.bits(t)
+
+
+def test_encode_balanced_ternary_closed_form(oref):
+    # integers m in [-121, 121] are exact in bf16; alpha = max |W| = 121, so
+    # r_0 = m / 121 and the ladder s_i = 3^(5-i) / 121 makes the greedy path
+    # spell the balanced-ternary digits of m (every decision has a margin of
+    # at least s_5 / 2, far above fp32 rounding)
+    ms = np.arange(-121, 122)
+    W = bf16_bits_of(ms.astype(np.float32)[None, :])
+    ladder = np.array([3.0 ** (4 - i) / 121.0 for i in range(5)], np.float32)
+    for zeta in (0.0, 0.25, 0.5):
+        codes, rho, alpha = oref.encode_B(W, ladder, zeta, 0)
+        assert alpha == 121.0 and rho is None
+        want = [code_of_word(balanced_ternary_word(int(m))) for m in ms]
+        assert codes[0].tolist() == want
+    assert codes[0][121] == 121  # m = 0: the all-zero word
+
+
+def test_encode_tie_goes_to_zero_and_zero_bias(oref):
+    ladder = np.array([1.0, 0.5, 0.25, 0.125, 0.0625], np.float32)
+    # alpha = 1; r_0 = 0.5 = s_1 / 2 exactly: a tie, c_1 = 0 (then c_2 = +1)
+    W = bf16_bits_of(np.array([[1.0, 0.5, 0.50390625, -0.5, 0.7, 0.0]],
+                              np.float32))
+    codes, _, _ = oref.encode_B(W, ladder, 0.5, 0)
+    c0 = codes[0].astype(np.int64)
+    first = c0 % 3 - 1  # c_1 (least significant digit)
+    second = (c0 // 3) % 3 - 1
+    assert first.tolist() == [1, 0, 1, 0, 1, 0]
+    assert second[1] == 1 and second[3] == -1
+    # zeta = 0.8 prefers 0 while |r| < 0.8 s_1: 0.7 and 0.50390625 give 0
+    codes, _, _ = oref.encode_B(W, ladder, 0.8, 0)
+    assert (codes[0].astype(np.int64) % 3 - 1).tolist() == [1, 0, 0, 0, 0, 0]
+
+
+def _decode_words(codes, ladder):
+    d = digits_of(codes) - 1  # [..., 5] with c_1 first
+    return (d * np.asarray(ladder, np.float64)).sum(axis=-1)
+
+
+@pytest.mark.parametrize("ladder,bound", [
+    ([1.0, 1 / 3, 1 / 9, 1 / 27, 1 / 81], 1 / 162),
+    ([1.0, 0.5, 0.25, 0.125, 0.0625], 1 / 32)])
+def test_encode_greedy_residual_bound(oref, ladder, bound):
+    # s_{i+1} <= s_i / 2 and |r_0| <= 1: each greedy step leaves
+    # |r_i| <= s_i / 2, so |x / a - sum c_i s_i| <= s_5 / 2
+    lad = np.array(ladder, np.float32)
+    W = I.student_t_bf16(64, 256, seed=31)
+    Wb = I.bits(W)
+    codes, rho, alpha = oref.encode_B(Wb, lad, 0.5, 0)
+    x = W.double().numpy()
+    assert alpha == float(np.abs(x).max())
+    err = np.abs(x / alpha - _decode_words(codes, lad))
+    assert err.max() <= bound * (1 + 1e-5)
+    # per-row scale: the same bound against each row's own maximum
+    codes, rho, alpha = oref.encode_B(Wb, lad, 0.5, 1)
+    rowmax = np.abs(x).max(axis=1, keepdims=True)
+    err = np.abs(x / rowmax - _decode_words(codes, lad))
+    assert err.max() <= bound * (1 + 1e-5)
+
+
+def test_encode_row_and_head_scales(oref):
+    lad = I.ladder_pow3().numpy()
+    W = I.student_t_bf16(8, 128, seed=32).float()
+    W[3] = 0.0                       # an all-zero row
+    W[5] *= 8.0                      # exact power-of-two rescales
+    W[6] *= 0.25
+    Wb = I.bits(W.to(torch.bfloat16))
+    x = W.to(torch.bfloat16).double().numpy()
+    codes, rho, alpha = oref.encode_B(Wb, lad, 0.5, 1)
+    rowmax = np.abs(x).max(axis=1)
+    assert alpha == rowmax.max()
+    # rho = fp16(alpha_n / alpha), through numpy's IEEE float16 rounding
+    want = np.where(rowmax > 0, rowmax / alpha, 0.0).astype(np.float16)
+    assert np.array_equal(rho, want.view(np.uint16))
+    assert np.all(codes[3] == 121) and rho[3] == 0
+    # scaling a row by a power of two leaves its words unchanged
+    base = I.student_t_bf16(8, 128, seed=32)
+    cb, _, _ = oref.encode_B(I.bits(base), lad, 0.5, 1)
+    assert np.array_equal(codes[5], cb[5]) and np.array_equal(codes[6], cb[6])
+    # per-head: one scale per 4 rows
+    codes4, rho4, _ = oref.encode_B(Wb, lad, 0.5, 4)
+    hmax = np.abs(x).reshape(2, 4, 128).max(axis=(1, 2))
+    assert np.array_equal(rho4, (hmax / alpha).astype(np.float16).view(np.uint16))
+    err = np.abs(x / np.repeat(hmax, 4)[:, None] - _decode_words(codes4, lad))
+    assert err.max() <= 1 / 162 * (1 + 1e-5)
+
+
+def test_encode_zero_matrix_and_nonfinite(oref):
+    lad = I.ladder_pow3().numpy()
+    codes, rho, alpha = oref.encode_B(np.zeros((2, 16), np.uint16), lad, 0.5, 1)
+    assert alpha == 0.0 and np.all(codes == 121) and np.all(rho == 0)
+    W = I.bits(I.student_t_bf16(2, 16, seed=1))
+    W[1, 3] = 0x7FC0  # bf16 NaN
+    _, st = oref.encode_B(W, lad, 0.5, 0, check=False)
+    assert st == oref.ERR_NONFINITE
