@@ -97,6 +97,18 @@ int oref_linear_A(const uint8_t *codes, const uint16_t *scales, int64_t n,
                   int64_t nrows, const uint16_t *x, int64_t batch, int64_t ldx,
                   double *y);
 
+/* Expert-indexed matmul (FUCINA README, "The method"): one Format A matrix
+ * per expert, the second plane only on the hot-expert prefix 0..n_hot-1;
+ * token t uses expert ids[t]: y[t][n] = sum_k w_{ids[t]}[n][k] x[t][k] (fp64,
+ * exact decoded weights). Plane p of expert e at codes_p + e * n * (k/G) *
+ * ceil(G/5) and scales_p + e * n * (k/G). y: [n_tokens][n]. */
+int oref_linear_experts_A(const uint8_t *codes1, const uint16_t *scales1,
+                          const uint8_t *codes2, const uint16_t *scales2,
+                          int32_t n_experts, int32_t n_hot, int64_t n,
+                          int64_t k, int32_t G, const int32_t *ids,
+                          int64_t n_tokens, const uint16_t *x, int64_t ldx,
+                          double *y);
+
 /* ---- Format B: 243-entry ladder code book, one code per byte ------------ */
 /* LUT[b] = fp32(alpha * sum_{i=1..5} c_i(b) a_i), sum in fp64 over i
  * ascending, c_i(b) = (i-1)-th base-3 digit of b minus 1 (first digit least

@@ -81,6 +81,9 @@ def _declare(L):
     L.oref_linear_A.restype = C.c_int
     L.oref_linear_A.argtypes = [P, P, i64, i64, i32, i32, P, i64, P, i64,
                                 i64, P]
+    L.oref_linear_experts_A.restype = C.c_int
+    L.oref_linear_experts_A.argtypes = [P, P, P, P, i32, i32, i64, i64, i32,
+                                        P, i64, P, i64, P]
     L.oref_build_lut.restype = C.c_int
     L.oref_build_lut.argtypes = [C.c_float, P, P]
     L.oref_unpack_B.restype = C.c_int
@@ -277,3 +280,21 @@ def encode_B(W_bits, ladder, zeta=0.5, rps=0, check=True, L=None):
     st = (L or lib()).oref_encode_B(_p(W), n, k, _p(ladder), C.c_float(zeta),
                                     rps, _p(codes), _p(rho), _p(alpha))
     return _ret((codes, rho, float(alpha[0])), st, check)
+
+
+def linear_experts_A(codes1, scales1, codes2, scales2, n_experts, n_hot, n, k,
+                     ids, x_bits, G=64, check=True, L=None):
+    """Expert-indexed Format A matmul: plane 1 of every expert in codes1 /
+    scales1 ([E][n][k/G][nb], [E][n][k/G]), plane 2 of the n_hot hot experts
+    in codes2 / scales2; token t uses expert ids[t]. Returns y [tokens][n]."""
+    codes1, scales1 = _c(codes1, np.uint8), _c(scales1, np.uint16)
+    codes2 = _c(codes2, np.uint8) if n_hot else None
+    scales2 = _c(scales2, np.uint16) if n_hot else None
+    ids = _c(ids, np.int32)
+    x = _c(x_bits, np.uint16)
+    tokens, ldx = x.shape
+    y = np.zeros((tokens, n), np.float64)
+    st = (L or lib()).oref_linear_experts_A(
+        _p(codes1), _p(scales1), _p(codes2), _p(scales2), n_experts, n_hot,
+        n, k, G, _p(ids), tokens, _p(x), ldx, _p(y))
+    return _ret(y, st, check)

@@ -275,3 +275,66 @@ int oref_linear_A(const uint8_t *codes, const uint16_t *scales, int64_t n,
   free(t);
   return status;
 }
+
+/* ---- expert-indexed matmul (FUCINA README, "The method") -----------------
+ *
+ * A mixture-of-experts layer stores one Format A matrix per expert. Hot
+ * experts carry both ternary planes, W ~ d1 T1 + d2 T2; cold experts carry
+ * one. Experts are written hot-first, so the second plane covers the expert
+ * prefix 0 .. n_hot - 1. Every token t is routed to one expert ids[t] (a
+ * token routed to several experts appears once per expert) and
+ *   y[t][n] = sum_k w_{ids[t]}[n][k] x[t][k],
+ *   w_e = s1 t1 + s2 t2 (e < n_hot) or s1 t1 (e >= n_hot),
+ * fp64, k ascending (the exact decoded weights, as oref_linear_A).
+ * Layouts: plane 1 of expert e: codes1 + e * n * (k/G) * ceil(G/5) bytes,
+ * scales1 + e * n * (k/G); plane 2 of expert e < n_hot: the same offsets in
+ * codes2 / scales2. ids outside 0 .. n_experts - 1 are OREF_ERR_INVALID_ARG.
+ * y: [n_tokens][n]. */
+int oref_linear_experts_A(const uint8_t *codes1, const uint16_t *scales1,
+                          const uint8_t *codes2, const uint16_t *scales2,
+                          int32_t n_experts, int32_t n_hot, int64_t n,
+                          int64_t k, int32_t G, const int32_t *ids,
+                          int64_t n_tokens, const uint16_t *x, int64_t ldx,
+                          double *y) {
+  if (!codes1 || !scales1 || !ids || !x || !y) return OREF_ERR_INVALID_ARG;
+  if (n_experts < 1 || n_hot < 0 || n_hot > n_experts || n_tokens < 0)
+    return OREF_ERR_INVALID_ARG;
+  if (n_hot > 0 && (!codes2 || !scales2)) return OREF_ERR_INVALID_ARG;
+  if (ldx < k) return OREF_ERR_INVALID_ARG;
+  const int st = check_A(codes1, scales1, n, k, G, 1);
+  if (st != OREF_OK) return st;
+  const int64_t gpr = k / G;
+  const int64_t cstride = n * gpr * oref_bytes_per_group(G); /* bytes */
+  const int64_t sstride = n * gpr;                           /* scales */
+  double *w1 = (double *)malloc(sizeof(double) * (size_t)(k > 0 ? k : 1));
+  double *w2 = (double *)malloc(sizeof(double) * (size_t)(k > 0 ? k : 1));
+  int status = OREF_OK;
+  for (int64_t t = 0; t < n_tokens; ++t) {
+    const int32_t e = ids[t];
+    if (e < 0 || e >= n_experts) {
+      status = OREF_ERR_INVALID_ARG;
+      break;
+    }
+    for (int64_t r = 0; r < n; ++r) {
+      int s = oref_weights_A(codes1 + e * cstride, scales1 + e * sstride, n, k,
+                             G, 1, &r, 1, w1);
+      if (s != OREF_OK) set_status(&status, s);
+      if (e < n_hot) {
+        s = oref_weights_A(codes2 + e * cstride, scales2 + e * sstride, n, k,
+                           G, 1, &r, 1, w2);
+        if (s != OREF_OK) set_status(&status, s);
+      }
+      double acc = 0.0;
+      for (int64_t j = 0; j < k; ++j) {
+        /* s1 t1 + s2 t2: both terms are fp16 values times a trit; their
+         * fp64 sum is exact */
+        const double wj = e < n_hot ? w1[j] + w2[j] : w1[j];
+        acc += wj * oref_bf16_to_f64(x[t * ldx + j]);
+      }
+      y[t * n + r] = acc;
+    }
+  }
+  free(w1);
+  free(w2);
+  return status;
+}

@@ -66,6 +66,14 @@ MUTATIONS = {
     "encode_global_scale_for_rows": ("oref_format_b.c",
                                      "      a = (float)gmax;",
                                      "      a = alpha;"),
+    "experts_hot_prefix_off_by_one": ("oref_format_a.c",
+                                      "const double wj = e < n_hot ?",
+                                      "const double wj = e <= n_hot ?"),
+    "experts_ignore_expert_id": ("oref_format_a.c",
+                                 "int s = oref_weights_A(codes1 + e * cstride,",
+                                 "int s = oref_weights_A(codes1,"),
+    "experts_drop_second_plane": ("oref_format_a.c",
+                                  "? w1[j] + w2[j] : w1[j];", "? w1[j] : w1[j];"),
     "round_ties_up": ("oref_fp.c",
                       "return (fmod(f, 2.0) == 0.0) ? f : f + 1.0;",
                       "return f + 1.0;"),

@@ -519,3 +519,34 @@ def test_encode_zero_matrix_and_nonfinite(oref):
     W[1, 3] = 0x7FC0  # bf16 NaN
     _, st = oref.encode_B(W, lad, 0.5, 0, check=False)
     assert st == oref.ERR_NONFINITE
+
+
+# ---- expert-indexed matmul (FUCINA README, "The method") -------------------
+
+def test_linear_experts_A_brute_force(oref):
+    # 5 experts, the first 2 hot (both planes); tokens routed to every expert,
+    # some twice; exact dyadic inputs, so every product and sum is exact
+    E, hot, n, k, G, tokens = 5, 2, 4, 128, 64, 7
+    rng = np.random.default_rng(41)
+    t1 = rng.integers(-1, 2, (E, n, k // G, G))
+    t2 = rng.integers(-1, 2, (hot, n, k // G, G))
+    s_vals = np.array([0.0, 0.125, 0.75, 1.5, 3.0, 2.0 ** -10], np.float16)
+    s1 = rng.choice(s_vals, (E, n, k // G)).view(np.uint16)
+    s2 = rng.choice(s_vals, (hot, n, k // G)).view(np.uint16)
+    c1, c2 = pack_independent(t1), pack_independent(t2)
+    ids = np.array([0, 4, 1, 3, 1, 2, 0], np.int32)
+    xb, x = dyadic_x(tokens, k, k + 4, 17)
+    w1 = (f16_bits_to_f64(s1)[..., None] * t1).reshape(E, n, k)
+    w2 = (f16_bits_to_f64(s2)[..., None] * t2).reshape(hot, n, k)
+    y = oref.linear_experts_A(c1, s1, c2, s2, E, hot, n, k, ids, xb, G)
+    for t, e in enumerate(ids):
+        w = w1[e] + (w2[e] if e < hot else 0.0)  # plane 2 only for hot ones
+        assert np.array_equal(y[t], w @ x[t]), (t, e)
+    # no hot experts: plane 1 everywhere
+    y0 = oref.linear_experts_A(c1, s1, None, None, E, 0, n, k, ids, xb, G)
+    for t, e in enumerate(ids):
+        assert np.array_equal(y0[t], w1[e] @ x[t])
+    _, st = oref.linear_experts_A(c1, s1, c2, s2, E, hot, n, k,
+                                  np.array([5], np.int32), xb[:1], G,
+                                  check=False)
+    assert st == oref.ERR_INVALID_ARG
