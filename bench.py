@@ -701,6 +701,69 @@ class FmtASmall(Workload):
         return f"{min(rows, 512)} rows of the 512x1024 workload"
 
 
+class EncodeB(Workload):
+    """Format B encoder (tq_encode_b) on the Gemma-shaped layers: up
+    21504x5376 with one scale per row and q 8192x5376 with one scale per
+    128-row head, W = bf16(0.02 StudentT(5)), the page's fitted ladder
+    (1, 0.33, 0.115, 0.037, 0.012), zero bias 0.5. Algorithmic bytes: W read
+    once (2 B/weight), codes written (1 B/weight) and rho."""
+    name = "encode_b"
+    MAX_ROWS = 256
+    BATCHES = ()
+    LADDER = (1.0, 0.33, 0.115, 0.037, 0.012)
+    SHAPES = ((21504, 5376, 1), (8192, 5376, 128))
+    SOURCES = ("tq_encode.cu",)
+
+    def describe(self):
+        return {"workload": f"{self.name}: Format B encoder, up 21504x5376 "
+                "(rho per row) and q 8192x5376 (rho per 128-row head), W "
+                "bf16 0.02*StudentT(5), ladder (1, 0.33, 0.115, 0.037, "
+                "0.012), zeta 0.5",
+                "l2": "231 MB and 88 MB of W per launch (> L2)",
+                "batches": [], "parallelism": "replicas"}
+
+    def setup(self, tq, dev):
+        self.W, self.codes, self.rho = [], [], []
+        for i, (n, k, rps) in enumerate(self.SHAPES):
+            self.W.append(I.student_t_bf16(n, k, seed=80 + i).to(dev))
+            self.codes.append(torch.empty(n, k, dtype=torch.uint8, device=dev))
+            self.rho.append(torch.empty((n + rps - 1) // rps,
+                                        dtype=torch.int16, device=dev))
+        self.alpha = torch.zeros(len(self.SHAPES), device=dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.pin_io([self.W[1]], [self.alpha])
+
+    def capture(self, tq):
+        steps = []
+        for i, (n, k, rps) in enumerate(self.SHAPES):
+            g = capture_graph([lambda i=i, rps=rps: tq.tq_encode_b(
+                self.W[i], self.LADDER, 0.5, rps, self.codes[i], self.rho[i],
+                self.alpha[i:i + 1], self.status)])
+            nbytes = 3 * n * k + 2 * ((n + rps - 1) // rps)
+            steps.append(Step(f"encode_{n}x{k}_rps{rps}", g, nbytes, 3,
+                              "encode_b"))
+        return steps
+
+    def oracle_setup(self):
+        from oracle import oref
+        self.oref = oref
+        self.sample = [I.bits(I.student_t_bf16(256, k, seed=80 + i))
+                       for i, (n, k, rps) in enumerate(self.SHAPES)]
+
+    def oracle_jobs(self, rows, r0=0):
+        rows = max(0, min(rows, 256 - r0))
+        lad = np.array(self.LADDER, np.float32)
+        jobs = []
+        for (n, k, rps), Wh in zip(self.SHAPES, self.sample):
+            Wr = Wh[r0:r0 + rows]
+            jobs.append((lambda Wr=Wr, rps=rps: self.oref.encode_B(
+                Wr, lad, 0.5, rps if rps == 1 else 0), 3 * rows * k))
+        return jobs
+
+    def sample_desc(self, rows):
+        return f"{min(rows, 256)} rows of each encoder layer shape"
+
+
 def make_workload(args):
     batches = tuple(args.batch) if args.batch else None
     if args.workload == "decode_step":
@@ -712,7 +775,7 @@ def make_workload(args):
 
 WORKLOADS = {"fmt_b_4096": FmtB4096, "fmt_b_gemma": FmtBGemma,
              "fmt_a_large": FmtALarge, "decode_step": DecodeStep,
-             "fmt_a_small": FmtASmall, "layer": Layer}
+             "fmt_a_small": FmtASmall, "layer": Layer, "encode_b": EncodeB}
 
 
 # ---- the oracle on the host cores ---------------------------------------------------
@@ -846,6 +909,8 @@ def run_tq(args, world, rank, local):
     torch.cuda.set_device(dev)
     wl = make_workload(args)
     wl.setup(tq, dev)
+    if args.force_path:
+        tq.tq_testing_force_linear_path(args.force_path)
     steps = wl.capture(tq)
     stream = torch.cuda.current_stream()
 
@@ -925,6 +990,9 @@ def run_tq(args, world, rank, local):
         "clocks": clk,
         "gpu_launches": int(sum(st.launches for st in steps) * args.steps),
     }
+    if args.force_path:
+        line["config"]["forced_path"] = {1: "cuda cores",
+                                         2: "tensor cores"}[args.force_path]
     if hasattr(wl, "extra"):
         line.update(wl.extra(steps, per))
     if world == 1 and not args.no_cpu_baseline:
@@ -982,6 +1050,9 @@ def main():
                     help="layer workload: columns")
     ap.add_argument("--planes", type=int, default=1,
                     help="layer workload: Format A planes")
+    ap.add_argument("--force-path", type=int, default=0, choices=[0, 1, 2],
+                    help="kernel family for comparisons: 0 automatic, "
+                         "1 CUDA cores, 2 tensor cores")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-seconds", type=float, default=90.0,

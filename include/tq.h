@@ -49,8 +49,15 @@
  *     `dev_status`: the first error code wins (atomic compare-and-swap from
  *     TQ_OK). The caller sets *dev_status = TQ_OK before the call and reads it
  *     after synchronising. With dev_status == NULL data errors go unreported.
- *   - The library keeps no device allocations and no mutable global state;
- *     all entry points are reentrant.
+ *   - The library keeps no device allocations. Its host state is a few
+ *     per-process caches, each written once under std::call_once or an
+ *     atomic (the driver's tensor-map encoder, a kernel's shared-memory limit
+ *     per device, resident-cluster counts per device), and the test hooks of
+ *     tq_testing.h. All entry points are reentrant and thread-safe.
+ *   - Every wait inside a kernel is bounded (2 s). A wait that gives up ends
+ *     the kernel's work early; tq_linear then leaves NaN in every output it
+ *     could not finish, which is how a time-out is reported. TQ_ERR_TIMEOUT is
+ *     reserved: no entry point returns it.
  */
 #ifndef TQ_H
 #define TQ_H
@@ -129,6 +136,38 @@ tq_status tq_quantize_pack(const void *W_bf16, int64_t n, int64_t k,
                            uint16_t *scales_out, int32_t *dev_status,
                            void *cuda_stream);
 
+/* Format B encoder ("A Discrete Weight Language for Large Language Models",
+ * alphaneural.io, section 3.1 "Encoding" and section 3.3 "Per-row scale").
+ * Every weight x of W becomes the word c_1..c_5 of the greedy 5-step ternary
+ * path over the ladder s_1..s_5 = ladder[0..4] of r_0 = x / a: step i keeps
+ * c_i = 0 while |r_{i-1}| < zeta s_i (the zero bias), else takes the sign of
+ * r_{i-1} when that moves r strictly closer to 0 (ties give 0); r_i =
+ * r_{i-1} - c_i s_i; code = sum (c_i + 1) 3^(i-1). Decisions are made in
+ * IEEE fp32: r_0 = fp32(x / a), threshold fp32(zeta s_i), r = fp32(r - c s).
+ *   W_bf16          device, bf16 [n][k] contiguous, 16-byte aligned;
+ *                   k % 16 == 0.
+ *   ladder          host, 5 finite amplitudes > 0.
+ *   zeta            zero bias in [0, 1]; 0.5 (or less) is the plain nearest
+ *                   choice.
+ *   rows_per_scale  0: a = alpha = max |W| over the matrix, no rho.
+ *                   r > 0: a = max |W| over rows [g r, g r + r) of group
+ *                   g = n / r (1: per row; the head size: per head) and
+ *                   rho_out[g] = fp16(a / alpha) (0 for an all-zero group).
+ *   codes_out       device, uint8 [n][k], 16-byte aligned.
+ *   rho_out         device, fp16 [ceil(n / r)], 2-byte aligned (r > 0).
+ *   alpha_out       device fp32: alpha = max |W| (build the code book with
+ *                   tq_build_lut(alpha, ladder)).
+ *   dev_status      device int32 or NULL: TQ_ERR_NONFINITE for NaN / Inf in
+ *                   W (those weights are skipped by the maxima; their codes
+ *                   are unspecified).
+ * An all-zero group (or matrix) gives code 121 (the all-zero word).
+ * Deterministic. */
+tq_status tq_encode_b(const void *W_bf16, int64_t n, int64_t k,
+                      const float ladder[5], float zeta,
+                      int32_t rows_per_scale, uint8_t *codes_out,
+                      uint16_t *rho_out, float *alpha_out, int32_t *dev_status,
+                      void *cuda_stream);
+
 /* Decode a package to bf16 (precisit.com page, "Three values and a shared
  * scale": W_hat = bf16(s t); alphaneural.io page, section 3.3).
  *   A: W_hat = bf16_RNE(fp32_RN(s1 t1 [+ s2 t2])).
@@ -152,7 +191,13 @@ tq_status tq_unpack(const tq_weights *w, void *W_bf16_out, int32_t *dev_status,
  * Codes are not validated here (tq_unpack does that): a Format B code >= 243
  * reads a NaN table entry; an invalid Format A byte gives an unspecified
  * finite value. Accuracy: |y - y_exact| <= 2e-3 * ||x_b||_2 * max_k |w[n][k]|
- * where y_exact uses the exact decoded weights. */
+ * where y_exact uses the exact decoded weights.
+ * Format A reads: a row's codes and scales are fetched in whole 16-byte
+ * blocks, from the block holding the first byte to the block holding the
+ * last. A 16-byte block never crosses a page, so these reads stay in mapped
+ * memory without padding; the bytes beyond the package are ignored.
+ * A bounded wait that gives up leaves NaN in the outputs it could not finish
+ * (the return value is still TQ_OK; see the conventions above). */
 tq_status tq_linear(const tq_weights *w, const void *x_bf16, int64_t batch,
                     int64_t ldx, float *y, int64_t ldy, void *cuda_stream);
 

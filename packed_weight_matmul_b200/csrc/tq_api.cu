@@ -5,6 +5,8 @@
 #include <string.h>
 
 #include "tq_common.cuh"
+#include "tq_linear.cuh"
+#include "tq_testing.h"
 
 namespace {
 
@@ -134,6 +136,30 @@ tq_status tq_unpack(const tq_weights *w, void *W_bf16_out, int32_t *dev_status,
                                      static_cast<cudaStream_t>(cuda_stream)));
 }
 
+tq_status tq_encode_b(const void *W_bf16, int64_t n, int64_t k,
+                      const float ladder[5], float zeta,
+                      int32_t rows_per_scale, uint8_t *codes_out,
+                      uint16_t *rho_out, float *alpha_out, int32_t *dev_status,
+                      void *cuda_stream) {
+  if (W_bf16 == nullptr || ladder == nullptr || codes_out == nullptr ||
+      alpha_out == nullptr)
+    return TQ_ERR_INVALID_ARG;
+  if (n < 0 || k < 0 || rows_per_scale < 0) return TQ_ERR_INVALID_ARG;
+  if (rows_per_scale > 0 && rho_out == nullptr) return TQ_ERR_INVALID_ARG;
+  if (!(zeta >= 0.0f && zeta <= 1.0f)) return TQ_ERR_INVALID_ARG;
+  for (int i = 0; i < 5; ++i)
+    if (!(ladder[i] > 0.0f) || isinf(ladder[i])) return TQ_ERR_INVALID_ARG;
+  if (k % 16 != 0) return TQ_ERR_SHAPE;
+  if (!aligned(W_bf16, 16) || !aligned(codes_out, 16) ||
+      !aligned(alpha_out, 4) || (rho_out != nullptr && !aligned(rho_out, 2)))
+    return TQ_ERR_ALIGNMENT;
+  if (dev_status != nullptr && !aligned(dev_status, 4)) return TQ_ERR_ALIGNMENT;
+  return from_cuda(tq::launch_encode_b(
+      static_cast<const uint16_t *>(W_bf16), n, k, ladder, zeta,
+      rows_per_scale, codes_out, rows_per_scale > 0 ? rho_out : nullptr,
+      alpha_out, dev_status, static_cast<cudaStream_t>(cuda_stream)));
+}
+
 tq_status tq_linear(const tq_weights *w, const void *x_bf16, int64_t batch,
                     int64_t ldx, float *y, int64_t ldy, void *cuda_stream) {
   tq::WeightsView v;
@@ -153,6 +179,32 @@ tq_status tq_linear(const tq_weights *w, const void *x_bf16, int64_t batch,
   return from_cuda(tq::launch_linear(
       v, static_cast<const __nv_bfloat16 *>(x_bf16), batch, ldx, y, ldy,
       stream));
+}
+
+tq_status tq_testing_linear_wait_fault(int32_t withhold_first_arrive,
+                                       uint64_t wait_limit_ns) {
+  tq::g_test_skip_first_arrive.store(withhold_first_arrive != 0 ? 1 : 0);
+  tq::g_test_wait_ns.store(wait_limit_ns);
+  return TQ_OK;
+}
+
+tq_status tq_testing_force_linear_path(int32_t path) {
+  if (path < 0 || path > 2) return TQ_ERR_INVALID_ARG;
+  tq::g_test_force_path.store(path);
+  return TQ_OK;
+}
+
+tq_status tq_testing_tc_self_check(int32_t enable, uint64_t record_out[4],
+                                   int32_t reset) {
+  tq::g_test_self_check.store(enable != 0 ? 1 : 0);
+  if (record_out == nullptr) return TQ_OK;
+  return from_cuda(tq::tc_check_record(record_out, reset != 0));
+}
+
+tq_status tq_testing_tc_trace(uint64_t *mapped_host_buffer) {
+  tq::g_test_trace.store(
+      reinterpret_cast<unsigned long long>(mapped_host_buffer));
+  return TQ_OK;
 }
 
 const char *tq_status_string(tq_status status) {

@@ -62,6 +62,10 @@ cudaError_t launch_quantize_pack(const uint16_t *W, int64_t n, int64_t k,
                                  cudaStream_t stream);
 cudaError_t launch_unpack(const WeightsView &w, uint16_t *out,
                           int32_t *status, cudaStream_t stream);
+cudaError_t launch_encode_b(const uint16_t *W, int64_t n, int64_t k,
+                            const float ladder[5], float zeta, int rps,
+                            uint8_t *codes, uint16_t *rho, float *alpha,
+                            int32_t *status, cudaStream_t stream);
 cudaError_t launch_linear(const WeightsView &w, const __nv_bfloat16 *x,
                           int64_t batch, int64_t ldx, float *y, int64_t ldy,
                           cudaStream_t stream);

@@ -1,38 +1,61 @@
 // Fused packed GEMM on the fifth-generation tensor cores (tcgen05), for the
-// batches the GEMV kernels do not take (Format B batch >= 5, Format A
-// batch >= 2), where x * W_hat^T becomes a real contraction:
+// batches where x * W_hat^T is a real contraction:
 //   Format A: y[b][n] = sum_p sum_g s_p[n][g] sum_{j in g} t_p[n][j] x[b][j]
 //             (precisit.com page, "Three values and a shared scale"; second
 //             plane per the FUCINA README, "The method")
 //   Format B: y[b][n] = rho[n / rps] * sum_k LUT[code[n][k]] x[b][k]
 //             (alphaneural.io page, sections 3.2, 3.3 and 4.2)
 //
-// One CTA computes a 128-row tile of y^T over the whole of K (or a cluster
-// slice of it) for N = batch rounded up to 16 (<= 64), accumulating in tensor
-// memory (128 lanes x N fp32 columns). Per 64-wide K block (and per plane):
-//   - 16 decoder warps (four per TMEM lane quarter; a thread owns one row
-//     and 16 k of the block) turn the codes of their rows into bf16 operands
-//     and write them straight into tensor memory with tcgen05.st: the A
-//     operand never passes through shared memory, whose bandwidth then only
-//     carries the code-book lookups. Each weight w is split into
-//     w_hi = bf16(w) and w_lo = bf16(w - w_hi): two MMAs (hi, then lo) give
-//     products exact to ~2^-16 relative, well inside the 2e-3 tolerance, with
-//     bf16 x used as is. For Format A, s*t splits exactly (an fp16 scale has
-//     11 significant bits: 8 in s_hi, 3 in s_lo). The x tile is staged in
-//     shared memory (operand B, K-major canonical layout). x and Format B
-//     codes arrive through per-thread cp.async rings; Format A codes and
-//     scales arrive in coalesced windows of 8 blocks that all decoders fetch
-//     together (completion and reuse on mbarriers).
-//   - One thread issues the 2 x 4 MMAs (M=128, N, K=16; A from tensor
-//     memory, B from shared memory) of the block and commits them to the
-//     stage's mbarrier, which frees the stage for the decoders. Tensor memory
-//     holds the accumulator and 6 A stages of 64 columns (32 hi + 32 lo).
-//   - After the last block the accumulator is read back with tcgen05.ld,
-//     rho applied (Format B) and y stored.
-// Waits are bounded; on a time-out the CTA writes NaN to its outputs, gives
-// in-flight MMAs a bounded chance to finish, frees its tensor memory and
-// exits. Decisions in front of warp-wide tcgen05 instructions are uniform.
+// Warp-specialised, one CTA per SM (it holds the whole tensor memory).
+// Without a split of K the CTAs are persistent and walk the 128-row tiles of
+// y^T: tile t, t + CTAs, ... With a split, a cluster of `ks` CTAs takes one
+// tile, each CTA a slice of K. For each 128-wide k block ("iteration"):
+//   - the code producer warp copies the tile's codes into a shared-memory
+//     ring with 1-D bulk copies, one per row (Format B: the block's 128
+//     codes; Format A: windows of 4 blocks = 8 groups of 13 bytes plus their
+//     fp16 scales, as aligned 16-byte supersets of each row's run);
+//   - the x producer copies the x tile (batch rounded up to 16 rows = N of
+//     the MMA, 128 k) with 2-D tensor copies in the canonical K-major layout
+//     (core matrices of 8 rows x 16 bytes); rows past the batch and k past K
+//     read as zero;
+//   - 8 decoder warps (two per tensor-memory lane quarter; a thread owns one
+//     row and 64 k) turn the codes into bf16 operands and store them straight
+//     into tensor memory (tcgen05.st): A never passes through shared memory.
+//     Each weight w is split into w_hi = bf16(w) and w_lo = bf16(w - w_hi),
+//     so the two MMAs (hi, lo) carry 16 significant bits of w: exact for
+//     Format A (an fp16 scale has 11), relative error <= 2^-17 for Format B;
+//   - one thread issues the 16 MMAs (M = 128, N, K = 16, A from tensor
+//     memory, B from shared memory) and commits them to the barriers that
+//     free the x stage and the A stage, and after the tile's last block to
+//     the accumulator barrier;
+//   - 4 epilogue warps read the accumulator (double-buffered in tensor
+//     memory, so the next tile's MMAs proceed meanwhile) and store y, or,
+//     with a split, keep the partial tile in shared memory; after a cluster
+//     barrier each CTA adds the `ks` partials of the rows it owns in rank
+//     order (distributed shared memory; deterministic), applies rho and
+//     stores y; a second barrier keeps every CTA alive while peers read.
+// Decoding uses a 64 KB table in shared memory at a 64 KB-aligned address,
+// replicated once per lane, so that one byte permute of a code word with the
+// lane's base word is the complete lookup address and a warp's lookups hit
+// distinct banks:
+//   Format B: entry c of lane l at tab + 256 c + 4 l holds bf16 hi | lo << 16
+//             of LUT[c];
+//   Format A: entry b of lane l at tab + 256 b + 8 l holds, for the 5 trits
+//             of code byte b, "selector bytes" 0x10 + 0x22 d (d = t + 1):
+//             trits 0..3 in the first word, trits 2..4 in the second. Four
+//             selector bytes, merged across code bytes with byte permutes,
+//             select through one more byte permute the bf16 pair {-s, 0, +s}
+//             of two weights (for the hi and for the lo part of the scale).
+// All waits are bounded (normally 2 s); on a time-out the CTA stops, writes
+// NaN to the outputs it owns, lets issued MMAs finish, frees its tensor
+// memory and exits. Decisions in front of warp-wide tcgen05 instructions are
+// uniform across the warp.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <cooperative_groups.h>
+
+#include <mutex>
 
 #include "tq_common.cuh"
 #include "tq_linear.cuh"
@@ -40,674 +63,1021 @@
 #include "tq_sm100_mma.cuh"
 
 namespace tq {
+
+// Test hooks (tq_testing_linear_wait_fault): a shorter wait limit and, when
+// set, decoders that withhold their first "A stage ready" arrive.
+std::atomic<uint64_t> g_test_wait_ns{0};
+std::atomic<int> g_test_skip_first_arrive{0};
+std::atomic<int> g_test_self_check{0};
+// Mapped host buffer of the self-checking kernel's progress trace (or 0):
+// entry [block * 8 + role] holds the last step the role reached.
+std::atomic<unsigned long long> g_test_trace{0};
+
+// Record of the self-checking instantiation (test hook): [0] first
+// violation (site << 48 | warp << 40 | block), [1] its value, [2] number of
+// violations, [3] waits that gave up.
+__device__ unsigned long long g_tc_check[4];
+
 namespace {
 
 constexpr int kTileM = 128;
 constexpr int kMaxN = 64;
-constexpr int kBlockK = 64;                       // k per stage
-// Decoder warps per CTA (a multiple of 4: the TMEM lane quarters): 16, four
-// per scheduler, 16 k per thread. The decode is bound by instruction issue
-// and latency, so every warp the register budget allows is a decoder.
-template <int FMT>
-struct TcCfg {
-  static constexpr int kDecoderWarps = 16;
-  static constexpr int kKParts = kDecoderWarps / 4;  // k parts of a block
-  static constexpr int kKPT = kBlockK / kKParts;     // k per decoder thread
+constexpr int kKB = 128;                 // k per iteration
+constexpr int kAStages = 3;              // A stages in tensor memory
+constexpr uint32_t kTmemCols = 512;      // the whole tensor memory
+constexpr uint32_t kAccCols = 64;        // one accumulator (N <= 64)
+constexpr uint32_t kAStage0 = 2 * kAccCols;
+constexpr uint32_t kAStageCols = 128;    // 64 hi + 64 lo columns
+constexpr int kDecWarps = 8;
+constexpr int kWarpCodes = 0, kWarpX = 1, kWarpMma = 2, kWarpEpi = 3,
+              kWarpDec = 7;
+constexpr int kThreads = 32 * (kWarpDec + kDecWarps);  // 480
+constexpr int kMaxCodeStages = 8;
+constexpr int kMaxXStages = 4;
+constexpr uint32_t kBRow = 144;          // Format B row slot: 128 codes + pad
+constexpr int kAWin = 4;                 // Format A window: 4 blocks, 8 groups
+constexpr uint32_t kARowCodes = 128;     // 104 code bytes + <= 15 skew
+constexpr uint32_t kARow = 160;          // + 16 scale bytes + <= 15 skew
+constexpr int kSmemMax = 227 * 1024;
 
-  static constexpr int kXPerThread =
-      (kMaxN * 8 + kDecoderWarps * 32 - 1) / (kDecoderWarps * 32);
-  static constexpr int kThreads = 32 * (1 + kDecoderWarps);
-};
-constexpr int kStages = 6;                        // A in TMEM, x in smem
-constexpr int kCodeDepth = 6;                     // x (and B code) ring depth
-// Format A codes arrive in windows of kWinBlocks k-blocks: per row the
-// window's 8 groups (104 code bytes) and 8 scales (16 bytes), fetched as
-// 16-byte aligned chunks (so up to 128 + 32 bytes with the alignment slack)
-// by all decoder threads together, lanes on consecutive chunks of a row.
-constexpr int kWinBlocks = 8;
-constexpr int kWinSlots = 3;                      // windows in the ring
-constexpr int kWinRowCodes = 128;
-constexpr int kWinRowBytes = kWinRowCodes + 32;
-constexpr int kWinChunks = kTileM * kWinRowBytes / 16;  // 16-byte copies
-constexpr uint32_t kTmemCols = 512;               // the whole tensor memory
-constexpr uint32_t kAccCols = 64;                 // accumulator: N <= 64
-constexpr uint32_t kStageCols = 64;               // A stage: 32 hi + 32 lo
-constexpr int kLutStride = 128;                   // 32 lane copies x 4 B
-constexpr int kLutBytes = 256 * kLutStride;       // 32 KB
+// Barrier block (byte offsets).
+constexpr uint32_t kBarCodeFull = 0, kBarCodeEmpty = 64, kBarXFull = 128,
+                   kBarXEmpty = 160, kBarAFull = 192, kBarAEmpty = 216,
+                   kBarAccFull = 240, kBarAccEmpty = 256, kBarDrain = 296,
+                   kTmemSlot = 304, kAbort = 308, kBarBytes = 320;
 
-// Offset of element (row r, k in [0,64)) inside an A (or x) K-block tile:
-// four k16 sub-tiles of rows*32 bytes, each in the canonical K-major layout
-// (LBO = 128: the second 8-k column; SBO = 256: the next 8 rows).
-__device__ __forceinline__ uint32_t tile_off(int r, int k, int rows) {
-  return (uint32_t)((k >> 4) * rows * 32 + (r >> 3) * 256 +
-                    ((k >> 3) & 1) * 128 + (r & 7) * 16 + (k & 7) * 2);
-}
-
-struct TcParams {
-  int ks_count;     // CTAs per cluster, each taking a slice of K
-  int n_pad;        // N of the MMA (batch rounded up to 16)
-  int stage_bytes;  // x tile
-  int x_off;        // x tile offset inside a stage
-  int ring_off, lut_off, bar_off, tmem_slot_off;
-  int code_off, code_slot;  // B: kCodeDepth slots of 128 rows x 64 B;
-                            // A: kWinSlots windows of 128 rows x 160 B
-  int xring_off;            // x ring: kCodeDepth slots of n_pad rows x 128 B
+struct TcPlan {
+  int n_pad, ks, tiles, kblocks, iters;
+  uint32_t base;  // window address where the dynamic shared memory starts
+  uint32_t tab;   // 64 KB table, 64 KB aligned
+  uint32_t code_lo, code_hi;   // code ring: stages [0, code_lo_n) at code_lo,
+  int code_lo_n, code_stages;  // the others at code_hi
+  uint32_t code_stage_bytes;
+  uint32_t x_ring, x_stage_bytes;
+  int x_stages;
+  uint32_t red;  // partial tile [128][n_pad] fp32 (split of K only)
+  uint32_t bars;
+  uint64_t wait_ns;
+  int skip_first_arrive;
   size_t smem;
 };
 
-// Asynchronous global -> shared copies; `n` < size bytes are read, the rest
-// of the destination is zero-filled.
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, int n) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst),
-               "l"(src), "r"(n)
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t s) {
+  return __byte_perm(a, b, s);
+}
+
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(a)
                : "memory");
+  return v;
 }
 
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
+// Table lookups: not volatile, so the compiler may schedule them freely; the
+// table is complete before the barrier that precedes every role's loop.
+__device__ __forceinline__ uint32_t lut32(uint32_t a) {
+  uint32_t v;
+  asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
 }
 
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+__device__ __forceinline__ uint2 lut64(uint32_t a) {
+  uint2 v;
+  asm("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+  return v;
 }
 
-// Arrives on `bar` once every cp.async this thread issued so far has landed
-// (the barrier's count includes this arrival).
-__device__ __forceinline__ void cp_async_mbar_arrive(uint32_t bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar)
+__device__ __forceinline__ void sts128(uint32_t a, uint32_t x, uint32_t y,
+                                       uint32_t z, uint32_t w) {
+  asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(a), "r"(x),
+               "r"(y), "r"(z), "r"(w)
                : "memory");
-}
-
-// Warp-wide store of N (8 or 16) consecutive TMEM columns.
-template <int N>
-__device__ __forceinline__ void tmem_st_cols(uint32_t ta,
-                                             const uint32_t (&v)[N]) {
-  if constexpr (N == 16) {
-    tmem_st16(ta, v);
-  } else {
-    static_assert(N == 8, "8 or 16 columns");
-    tmem_st8(ta, v);
-  }
 }
 
 __device__ __forceinline__ uint32_t bf16_bits_rn(float v) {
   return __bfloat16_as_ushort(__float2bfloat16_rn(v));
 }
 
-// Format B: 8 codes (two words) of one row -> 4 hi and 4 lo bf16 pairs. The
-// table word of code c for this lane holds bf16(w) | bf16(w - bf16(w)) << 16.
-__device__ __forceinline__ void decode8_b(uint32_t w0, uint32_t w1,
-                                          uint32_t lut_base, uint32_t lane8,
-                                          uint32_t (&hi)[4],
-                                          uint32_t (&lo)[4]) {
-  uint32_t v[8];
+// End of the window that starts at iteration ws: at most `win` iterations,
+// inside the slice and inside one plane.
+__device__ __forceinline__ int window_end(int ws, int it1, int kblocks,
+                                          int win) {
+  const int plane_end = (ws / kblocks + 1) * kblocks;
+  int we = ws + win;
+  if (we > it1) we = it1;
+  if (we > plane_end) we = plane_end;
+  return we;
+}
+
+// Selector bytes 0x10 + 0x22 d of the five trits of code byte b (digits d,
+// least significant first): trits 0..3 in .x, trits 2..4 in .y. A byte
+// permute with selector byte 0x10 / 0x32 / 0x54 takes bytes 0-1 / 2-3 / 4-5
+// of its two sources: -s / zero / +s.
+__device__ __forceinline__ uint2 selector_entry(uint32_t b) {
+  uint32_t rest = b < 243u ? b : 121u;  // invalid bytes: all trits 0
+  uint32_t s[5];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    const uint32_t w = e < 4 ? w0 : w1;
-    const uint32_t a2 = __byte_perm(w, lane8, 0x5504u | ((uint32_t)(e & 3) << 4));
-    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v[e]) : "r"(lut_base + (a2 >> 1)));
+  for (int i = 0; i < 5; ++i) {
+    s[i] = 0x10u + 0x22u * (rest % 3u);
+    rest /= 3u;
   }
+  return make_uint2(s[0] | s[1] << 8 | s[2] << 16 | s[3] << 24,
+                    s[2] | s[3] << 8 | s[4] << 16);
+}
+
+// Format B: 64 codes of one row (16 words) -> 32 hi and 32 lo bf16 pairs.
+__device__ __forceinline__ void decode_b(const uint32_t (&cw)[16],
+                                         uint32_t lane_tab, uint32_t (&hi)[32],
+                                         uint32_t (&lo)[32]) {
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    hi[q] = __byte_perm(v[2 * q], v[2 * q + 1], 0x5410u);
-    lo[q] = __byte_perm(v[2 * q], v[2 * q + 1], 0x7632u);
+  for (int j = 0; j < 16; ++j) {
+    const uint32_t v0 = lut32(prmt(cw[j], lane_tab, 0x7604u));
+    const uint32_t v1 = lut32(prmt(cw[j], lane_tab, 0x7614u));
+    const uint32_t v2 = lut32(prmt(cw[j], lane_tab, 0x7624u));
+    const uint32_t v3 = lut32(prmt(cw[j], lane_tab, 0x7634u));
+    hi[2 * j] = prmt(v0, v1, 0x5410u);
+    lo[2 * j] = prmt(v0, v1, 0x7632u);
+    hi[2 * j + 1] = prmt(v2, v3, 0x5410u);
+    lo[2 * j + 1] = prmt(v2, v3, 0x7632u);
   }
 }
 
-// Format A: trits 8c..8c+7 of the thread's 16, given as 2-bit fields
-// (bit 2j: t_j != 0, bit 2j+1: t_j < 0) -> 4 hi and 4 lo pairs of s*t.
-// s2 = s | s << 16 (hi or lo part of the scale in both halves); pair_tab[f]
-// holds, for the 4 bits f of a pair, the keep mask (0xFFFF per nonzero half)
-// and the sign mask (0x8000 per negative half), so a pair is one
-// (s2 & keep) ^ sign. XOR (not OR) keeps a negative lo part exact.
-__device__ __forceinline__ void decode8_a(uint32_t bits, int c,
-                                          uint32_t s_hi2, uint32_t s_lo2,
-                                          uint32_t pair_tab,
-                                          uint32_t (&hi)[4],
-                                          uint32_t (&lo)[4]) {
+// Format A: one group (13 code bytes, realigned into b[0..3]) -> 32 hi and
+// 32 lo bf16 pairs of s*t. (nh, ph) = (-s_hi with a zero upper half, +s_hi)
+// are the byte sources of the selecting permute; (nl, pl) the same for s_lo.
+__device__ __forceinline__ void decode_a(const uint32_t (&b)[4],
+                                         uint32_t lane_tab, uint32_t nh,
+                                         uint32_t ph, uint32_t nl, uint32_t pl,
+                                         uint32_t (&hi)[32],
+                                         uint32_t (&lo)[32]) {
+  uint2 T[13];
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const uint32_t f = (bits >> (16 * c + 4 * q)) & 15u;
-    uint32_t keep, sign;
-    asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];"
-                 : "=r"(keep), "=r"(sign)
-                 : "r"(pair_tab + f * 8u));
-    hi[q] = (s_hi2 & keep) ^ sign;
-    lo[q] = (s_lo2 & keep) ^ sign;
+  for (int m = 0; m < 13; ++m)
+    T[m] = lut64(prmt(b[m >> 2], lane_tab, 0x7604u | ((uint32_t)(m & 3) << 4)));
+  // E[j]: selector bytes of trits 4j .. 4j+3 (code byte m holds trits
+  // 5m .. 5m+4); the pattern repeats every 4 code bytes (20 trits).
+  uint32_t E[16];
+#pragma unroll
+  for (int p = 0; p < 3; ++p) {
+    const uint2 t0 = T[4 * p], t1 = T[4 * p + 1], t2 = T[4 * p + 2],
+                t3 = T[4 * p + 3];
+    E[5 * p + 0] = t0.x;
+    E[5 * p + 1] = prmt(t0.y, t1.x, 0x6542u);
+    E[5 * p + 2] = prmt(t1.y, t2.x, 0x5421u);
+    E[5 * p + 3] = prmt(t2.y, t3.x, 0x4210u);
+    E[5 * p + 4] = prmt(t3.x, t3.y, 0x6321u);
+  }
+  E[15] = T[12].x;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const uint32_t e2 = E[j] >> 16;
+    hi[2 * j] = prmt(nh, ph, E[j]);
+    lo[2 * j] = prmt(nl, pl, E[j]);
+    hi[2 * j + 1] = prmt(nh, ph, e2);
+    lo[2 * j + 1] = prmt(nl, pl, e2);
   }
 }
 
-template <int FMT>
-__global__ void __launch_bounds__(TcCfg<FMT>::kThreads, 1)
-    gemm_tc_kernel(WeightsView w, const __nv_bfloat16 *__restrict__ x,
-                   int64_t batch, int64_t ldx, float *__restrict__ y,
-                   int64_t ldy, TcParams P) {
-  constexpr int kDecoderWarps = TcCfg<FMT>::kDecoderWarps;
-  constexpr int kKPT = TcCfg<FMT>::kKPT;
-  constexpr int kXPerThread = TcCfg<FMT>::kXPerThread;
+// Self-checking instantiation (CK): every address a role computes is checked
+// against the region it must lie in; a violation is recorded (first one in
+// full, all of them counted) and the access goes to a safe address instead.
+__device__ __noinline__ void ck_record(uint32_t site, uint64_t value) {
+  const unsigned long long tag =
+      ((unsigned long long)site << 48) |
+      ((unsigned long long)(threadIdx.x >> 5) << 40) | blockIdx.x;
+  if (atomicCAS(&g_tc_check[0], 0ull, tag) == 0ull) g_tc_check[1] = value;
+  atomicAdd(&g_tc_check[2], 1ull);
+}
+
+// This CTA's dynamic shared window [lo, lo + size) and a safe address in it.
+struct SmemWin {
+  uint32_t lo, size, safe;
+};
+
+template <bool CK>
+__device__ __forceinline__ uint32_t ck_smem(const SmemWin &W, uint32_t a,
+                                            uint32_t bytes, uint32_t site) {
+  if constexpr (CK) {
+    if (a < W.lo || a + bytes > W.lo + W.size ||
+        (a & (bytes >= 16 ? 15u : bytes - 1u)) != 0u) {
+      ck_record(site, a);
+      return W.safe;  // in the window, aligned
+    }
+  }
+  return a;
+}
+
+template <bool CK>
+__device__ __forceinline__ uint32_t ck_tmem(uint32_t ta, uint32_t cols,
+                                            uint32_t lane_base, uint32_t site) {
+  if constexpr (CK) {
+    if ((ta & 0xFFFFu) + cols > kTmemCols || (ta >> 16) != lane_base) {
+      ck_record(site, ta);
+      return (lane_base << 16) | kAStage0;
+    }
+  }
+  return ta;
+}
+
+// Progress trace of the self-checking kernel: a store to mapped host memory
+// (it outlives a fault of the context), made visible system-wide at once.
+template <bool CK>
+__device__ __forceinline__ void ck_trace(unsigned long long *trace, int role,
+                                         int tile, int it, int step) {
+  if constexpr (CK) {
+    if (trace != nullptr) {
+      const unsigned long long v = ((unsigned long long)(tile + 1) << 32) |
+                                   ((unsigned long long)(it & 0xFFFF) << 16) |
+                                   (unsigned long long)(step & 0xFFFF);
+      asm volatile("st.volatile.global.u64 [%0], %1;" ::"l"(
+                       trace + blockIdx.x * 8 + role),
+                   "l"(v)
+                   : "memory");
+      __threadfence_system();
+    }
+  }
+}
+
+template <int FMT, bool CK>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_tc_kernel(const WeightsView w, int64_t batch, float *__restrict__ y,
+                   int64_t ldy, const TcPlan P,
+                   const __grid_constant__ CUtensorMap tmap_x,
+                   unsigned long long *trace) {
+  constexpr int kWin = FMT == TQ_FMT_A ? kAWin : 1;
   extern __shared__ __align__(1024) uint8_t smem[];
-  const uint32_t sbase = smem_u32(smem);
-  const uint32_t ring = sbase + P.ring_off;
-  const uint32_t full0 = sbase + P.bar_off;           // full[s]: decoders done
-  const uint32_t empty0 = full0 + 8 * kStages;        // empty[s]: MMAs done
-  const uint32_t acc_bar = empty0 + 8 * kStages;      // accumulator ready
-  const uint32_t wfull0 = acc_bar + 8;                // A window landed
-  const uint32_t wempty0 = wfull0 + 8 * kWinSlots;    // A window consumed
-  volatile uint32_t &tmem_slot =
-      *reinterpret_cast<uint32_t *>(smem + P.tmem_slot_off);
-  volatile int &abort_flag =
-      *reinterpret_cast<int *>(smem + P.tmem_slot_off + 4);
-
+  const uint32_t base = smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int ks = blockIdx.x % P.ks_count;  // rank in the cluster
-  const int64_t row0 = (int64_t)(blockIdx.x / P.ks_count) * kTileM;
-  const int N = P.n_pad;
-  const int64_t K = w.k;
-  const int kblocks = (int)((K + kBlockK - 1) / kBlockK);
-  const int planes = FMT == TQ_FMT_A ? w.planes : 1;
-  const int iters_all = planes * kblocks;
-  // this CTA's slice of the (plane, k-block) iterations
-  const int it_begin = (int)((int64_t)iters_all * ks / P.ks_count);
-  const int iters = (int)((int64_t)iters_all * (ks + 1) / P.ks_count) - it_begin;
-  const uint32_t idesc = idesc_bf16_f32(kTileM, N);
+  const int ks = P.ks;
+  const int nclusters = (int)gridDim.x / ks;
+  const int cid = (int)blockIdx.x / ks;
+  const int64_t N = w.n, K = w.k;
+  const int n_pad = P.n_pad;
+  const int nb = (int)(batch < n_pad ? batch : n_pad);
+  const int64_t gpr = K / 64;  // Format A groups per row
+  const int rank = ks > 1 ? (int)cluster_rank() : 0;
+  // this CTA's iterations of every tile
+  const int it0 = (int)((int64_t)P.iters * rank / ks);
+  const int it1 = (int)((int64_t)P.iters * (rank + 1) / ks);
+  // rows of every tile this CTA owns in the cluster reduction
+  const int r_lo = kTileM * rank / ks, r_hi = kTileM * (rank + 1) / ks;
+  // partial tile of a K split (same offset in every CTA of the cluster)
+  float *const part = reinterpret_cast<float *>(smem + (P.red - P.base));
 
-  if (threadIdx.x == 0) {
-    abort_flag = 0;
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(full0 + 8 * s, kDecoderWarps);
-      mbar_init(empty0 + 8 * s, 1);
-    }
-    mbar_init(acc_bar, 1);
-    if constexpr (FMT == TQ_FMT_A) {
-      for (int s = 0; s < kWinSlots; ++s) {
-        mbar_init(wfull0 + 8 * s, kDecoderWarps * 32);
-        mbar_init(wempty0 + 8 * s, kDecoderWarps * 32);
+  // The plan places everything for a window at P.base. A CTA's own shared
+  // addresses need not start there: in a cluster they also name the CTA's
+  // rank (a shared::cta address is a shared::cluster one), so every planned
+  // address moves by this CTA's offset. It keeps the table's 64 KB alignment
+  // unless it is not a multiple of 64 KB: then no work is safe, the outputs
+  // are NaN, and a CTA of a cluster still takes the cluster's two barriers
+  // (its partial tile is NaN, so the rows the others finish are NaN too).
+  const uint32_t delta = base - P.base;
+  if ((delta & 0xFFFFu) != 0u) {
+    const float qnan = __int_as_float(0x7FC00000);
+    if (ks == 1) {
+      for (int t = cid; t < P.tiles; t += nclusters)
+        for (int i = threadIdx.x; i < kTileM * nb; i += blockDim.x) {
+          const int64_t row = (int64_t)t * kTileM + i % kTileM;
+          if (row < N) y[(int64_t)(i / kTileM) * ldy + row] = qnan;
+        }
+    } else {
+      namespace cg = cooperative_groups;
+      cg::cluster_group cluster = cg::this_cluster();
+      for (int i = threadIdx.x; i < kTileM * n_pad; i += blockDim.x)
+        part[i] = qnan;
+      cluster.sync();
+      for (int i = threadIdx.x; i < (r_hi - r_lo) * nb; i += blockDim.x) {
+        const int64_t row = (int64_t)cid * kTileM + r_lo + i % (r_hi - r_lo);
+        if (cid < P.tiles && row < N)
+          y[(int64_t)(i / (r_hi - r_lo)) * ldy + row] = qnan;
       }
+      cluster.sync();
     }
+    return;
+  }
+  const uint32_t tab = P.tab + delta;
+  const uint32_t B0 = P.bars + delta;
+  const uint32_t x_ring = P.x_ring + delta;
+  const uint32_t code_lo = P.code_lo + delta, code_hi = P.code_hi + delta;
+  const uint32_t abort_addr = B0 + kAbort;
+  const uint64_t lim = P.wait_ns;
+  const SmemWin W{base, (uint32_t)P.smem, B0};
+
+  auto code_stage = [&](int s) -> uint32_t {
+    return s < P.code_lo_n
+               ? code_lo + (uint32_t)s * P.code_stage_bytes
+               : code_hi + (uint32_t)(s - P.code_lo_n) * P.code_stage_bytes;
+  };
+
+  // ---- set-up -------------------------------------------------------------
+  if (threadIdx.x == 0) {
+    if constexpr (CK) {
+      ck_smem<CK>(W, tab, 0x10000u, 1);
+      ck_smem<CK>(W, B0, kBarBytes, 1);
+      ck_smem<CK>(W, x_ring, (uint32_t)P.x_stages * P.x_stage_bytes, 1);
+      if (P.ks > 1) ck_smem<CK>(W, P.red + delta, (uint32_t)(kTileM * P.n_pad * 4), 1);
+      for (int s = 0; s < P.code_stages; ++s)
+        ck_smem<CK>(W, code_stage(s), P.code_stage_bytes, 1);
+    }
+    st_volatile_s32(abort_addr, 0);
+    for (int s = 0; s < P.code_stages; ++s) {
+      mbar_init(B0 + kBarCodeFull + 8 * s, 1);
+      mbar_init(B0 + kBarCodeEmpty + 8 * s, kDecWarps);
+    }
+    for (int s = 0; s < P.x_stages; ++s) {
+      mbar_init(B0 + kBarXFull + 8 * s, 1);
+      mbar_init(B0 + kBarXEmpty + 8 * s, 1);
+    }
+    for (int s = 0; s < kAStages; ++s) {
+      mbar_init(B0 + kBarAFull + 8 * s, kDecWarps);
+      mbar_init(B0 + kBarAEmpty + 8 * s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(B0 + kBarAccFull + 8 * b, 1);
+      mbar_init(B0 + kBarAccEmpty + 8 * b, 4);
+    }
+    mbar_init(B0 + kBarDrain, 1);
     mbar_init_fence();
   }
-  if (warp == 0) tmem_alloc(sbase + P.tmem_slot_off, kTmemCols);
-  // Lookup tables.
+  if (warp == kWarpMma) {
+    __syncwarp();
+    tmem_alloc(B0 + kTmemSlot, kTmemCols);
+  }
+  if (warp == kWarpX && lane == 0)
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&tmap_x) : "memory");
+  // the lane-replicated table
   if constexpr (FMT == TQ_FMT_B) {
-    // entry e, lane copy l at e*128 + 4*l: bf16(w) | bf16(w - bf16(w)) << 16
-    for (int e = threadIdx.x; e < 256; e += blockDim.x) {
+    for (int i = threadIdx.x; i < 256 * 8; i += blockDim.x) {
+      const int e = i >> 3, j = i & 7;
       const float v = __ldg(w.lut + e);
       const uint32_t h = bf16_bits_rn(v);
-      const float hv = __uint_as_float(h << 16);
-      const uint32_t l = bf16_bits_rn(v - hv);
-      const uint32_t word = h | (l << 16);
-      const uint4 w4 = make_uint4(word, word, word, word);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int jj = (j + e) & 7;
-        *reinterpret_cast<uint4 *>(smem + P.lut_off + e * kLutStride + jj * 16) =
-            w4;
-      }
+      const uint32_t l = bf16_bits_rn(v - __uint_as_float(h << 16));
+      const uint32_t word = h | l << 16;
+      sts128(tab + (uint32_t)e * 256u + (uint32_t)j * 16u, word, word, word,
+             word);
     }
   } else {
-    // byte -> its 5 trits (least significant digit first) as 2-bit fields:
-    // bit 2i: t_i != 0, bit 2i+1: t_i < 0
-    uint16_t *tab = reinterpret_cast<uint16_t *>(smem + P.lut_off);
-    for (int b = threadIdx.x; b < 256; b += blockDim.x) {
-      uint32_t m = 0, rest = b < 243 ? b : 121;
-#pragma unroll
-      for (int i = 0; i < 5; ++i) {
-        const uint32_t d = rest % 3;
-        rest /= 3;
-        if (d != 1) m |= 1u << (2 * i);
-        if (d == 0) m |= 1u << (2 * i + 1);
-      }
-      tab[b] = (uint16_t)m;
-    }
-    // pair table (16 entries of keep, sign words) after the byte table,
-    // indexed by two 2-bit fields
-    uint32_t *ptab = reinterpret_cast<uint32_t *>(smem + P.lut_off + 512);
-    for (int i = threadIdx.x; i < 16; i += blockDim.x) {
-      const uint32_t z0 = i & 1, n0 = (i >> 1) & 1, z1 = (i >> 2) & 1,
-                     n1 = (i >> 3) & 1;
-      ptab[2 * i] = (z0 ? 0x0000FFFFu : 0u) | (z1 ? 0xFFFF0000u : 0u);
-      ptab[2 * i + 1] = (z0 && n0 ? 0x00008000u : 0u) | (z1 && n1 ? 0x80000000u : 0u);
+    for (int i = threadIdx.x; i < 256 * 16; i += blockDim.x) {
+      const int e = i >> 4, j = i & 15;
+      const uint2 v = selector_entry((uint32_t)e);
+      sts128(tab + (uint32_t)e * 256u + (uint32_t)j * 16u, v.x, v.y, v.x,
+             v.y);
     }
   }
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
-  const uint32_t tmem = tmem_slot;
+  uint32_t tmem;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(tmem) : "r"(B0 + kTmemSlot)
+               : "memory");
 
-  if (warp == 0) {
-    // ---- MMA issuer ----
+  if (warp == kWarpCodes) {
+    // ---- code producer: bulk copies of each window's rows -------------------
+    int s = 0, u = 0;  // ring slot, windows issued so far
+    bool ok = true;
+    for (int t = cid; ok && t < P.tiles; t += nclusters) {
+      const int64_t row0 = (int64_t)t * kTileM;
+      const int rows = (int)(N - row0 < kTileM ? N - row0 : kTileM);
+      for (int ws = it0; ws < it1;) {
+        const int we = window_end(ws, it1, P.kblocks, kWin);
+        if (u >= P.code_stages)
+          ok = mbar_wait(B0 + kBarCodeEmpty + 8 * s,
+                         (uint32_t)((u / P.code_stages) + 1) & 1u, abort_addr,
+                         lim);
+        ok = __all_sync(0xFFFFFFFFu, ok);
+        if constexpr (CK) if (!ok && lane == 0) ck_record(21, (uint64_t)u);
+        if (!ok) break;
+        const uint32_t full = B0 + kBarCodeFull + 8 * s;
+        const uint32_t dst0 = code_stage(s);
+        if (lane == 0) ck_trace<CK>(trace, 0, t, ws, 1);
+        if constexpr (FMT == TQ_FMT_B) {
+          const int64_t k0 = (int64_t)ws * kKB;
+          const uint32_t sz = (uint32_t)(K - k0 < kKB ? K - k0 : kKB);
+          if (lane == 0) mbar_arrive_expect_tx(full, sz * (uint32_t)rows);
+          __syncwarp();
+          for (int r = lane; r < rows; r += 32) {
+            uint32_t d = dst0 + (uint32_t)r * kBRow;
+            const uint8_t *src = w.codes + (row0 + r) * K + k0;
+            if constexpr (CK) {
+              d = ck_smem<CK>(W, d, sz, 2);
+              if (row0 + r >= N || k0 + sz > K) {
+                ck_record(3, (uint64_t)((row0 + r) * K + k0));
+                src = w.codes;
+              }
+            }
+            bulk_g2s(d, src, sz, full);
+          }
+        } else {
+          const int plane = ws / P.kblocks;
+          const int64_t g0 = 2 * (int64_t)(ws - plane * P.kblocks);
+          const int64_t want = 2 * (int64_t)(we - ws);
+          const uintptr_t ng = (uintptr_t)(want < gpr - g0 ? want : gpr - g0);
+          const uintptr_t cbase = reinterpret_cast<uintptr_t>(w.codes) +
+                                  (uintptr_t)(plane * w.codes_plane_stride);
+          const uintptr_t sbase =
+              reinterpret_cast<uintptr_t>(w.scales) +
+              (uintptr_t)(2 * plane * w.scales_plane_stride);
+          const uintptr_t m16 = ~(uintptr_t)15;
+          uint32_t bytes = 0;
+          for (int r = lane; r < rows; r += 32) {
+            const int64_t gi = (row0 + r) * gpr + g0;
+            const uintptr_t c = cbase + (uintptr_t)(gi * 13);
+            const uintptr_t sc = sbase + (uintptr_t)(gi * 2);
+            bytes += (uint32_t)(((c + 13 * ng + 15) & m16) - (c & m16));
+            bytes += (uint32_t)(((sc + 2 * ng + 15) & m16) - (sc & m16));
+          }
+          bytes = __reduce_add_sync(0xFFFFFFFFu, bytes);
+          if (lane == 0) mbar_arrive_expect_tx(full, bytes);
+          __syncwarp();
+          for (int r = lane; r < rows; r += 32) {
+            const int64_t gi = (row0 + r) * gpr + g0;
+            const uintptr_t c = cbase + (uintptr_t)(gi * 13);
+            const uintptr_t sc = sbase + (uintptr_t)(gi * 2);
+            uint32_t dst = dst0 + (uint32_t)r * kARow;
+            const uint32_t csz = (uint32_t)(((c + 13 * ng + 15) & m16) - (c & m16));
+            const uint32_t ssz = (uint32_t)(((sc + 2 * ng + 15) & m16) - (sc & m16));
+            if constexpr (CK) {
+              dst = ck_smem<CK>(W, dst, kARow, 4);
+              if (csz > kARowCodes || ssz > kARow - kARowCodes) ck_record(5, csz << 16 | ssz);
+            }
+            bulk_g2s(dst, reinterpret_cast<const void *>(c & m16), csz, full);
+            bulk_g2s(dst + kARowCodes, reinterpret_cast<const void *>(sc & m16),
+                     ssz, full);
+          }
+        }
+        if (lane == 0) ck_trace<CK>(trace, 0, t, ws, 2);
+        ws = we;
+        ++u;
+        s = s + 1 == P.code_stages ? 0 : s + 1;
+      }
+    }
+    if (lane == 0) ck_trace<CK>(trace, 0, 0xFFFF, 0, 3);
+    // no copy may still be landing in shared memory when the CTA exits
+    // (after a time-out some fills are never consumed)
     if (lane == 0) {
-      int it = 0;
-      for (; it < iters; ++it) {
-        const int s = it % kStages;
-        if (!mbar_wait(full0 + 8 * s, (it / kStages) & 1)) {
-          abort_flag = 1;
+      for (int j = u > P.code_stages ? u - P.code_stages : 0; j < u; ++j)
+        mbar_wait(B0 + kBarCodeFull + 8 * (j % P.code_stages),
+                  (uint32_t)(j / P.code_stages) & 1u);
+    }
+  } else if (warp == kWarpX) {
+    // ---- x producer: 16 tensor copies of 8 k x n_pad rows per iteration -----
+    if (lane == 0) {
+      int s = 0, u = 0;
+      bool ok = true;
+      const uint32_t box = (uint32_t)n_pad * 16u;
+      for (int t = cid; ok && t < P.tiles; t += nclusters) {
+        for (int it = it0; it < it1; ++it) {
+          if (u >= P.x_stages &&
+              !mbar_wait(B0 + kBarXEmpty + 8 * s,
+                         (uint32_t)((u / P.x_stages) + 1) & 1u, abort_addr,
+                         lim)) {
+            if constexpr (CK) ck_record(22, (uint64_t)u);
+            ok = false;
+            break;
+          }
+          const uint32_t full = B0 + kBarXFull + 8 * s;
+          const uint32_t dst = x_ring + (uint32_t)s * P.x_stage_bytes;
+          const int k0 = (it % P.kblocks) * kKB;
+          ck_trace<CK>(trace, 1, t, it, 1);
+          mbar_arrive_expect_tx(full, 16u * box);
+#pragma unroll 1
+          for (int c = 0; c < 16; ++c) {
+            uint32_t d = dst + (uint32_t)c * box;
+            if constexpr (CK) {
+              d = ck_smem<CK>(W, d, box, 6);
+              if ((d & 127u) != 0u) ck_record(7, d);
+            }
+            tma_load_2d(d, &tmap_x, k0 + 8 * c, 0, full);
+          }
+          ++u;
+          s = s + 1 == P.x_stages ? 0 : s + 1;
+        }
+      }
+      for (int j = u > P.x_stages ? u - P.x_stages : 0; j < u; ++j)
+        mbar_wait(B0 + kBarXFull + 8 * (j % P.x_stages),
+                  (uint32_t)(j / P.x_stages) & 1u);
+    }
+  } else if (warp == kWarpMma) {
+    // ---- MMA issuer ---------------------------------------------------------
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(kTileM, n_pad);
+      const uint32_t lbo = (uint32_t)n_pad * 16u;  // next 8 k of the x tile
+      int xs = 0, ux = 0, as = 0, ua = 0;
+      int ca = 0;  // accumulator commits
+      bool ok = true;
+      int i = 0;
+      for (int t = cid; ok && t < P.tiles; t += nclusters, ++i) {
+        const int buf = i & 1;
+        if (i >= 2 && !mbar_wait(B0 + kBarAccEmpty + 8 * buf,
+                                 (uint32_t)((i >> 1) + 1) & 1u, abort_addr,
+                                 lim)) {
+          if constexpr (CK) ck_record(23, (uint64_t)i);
+          ok = false;
           break;
         }
         tc_fence_after_sync();
-        const uint32_t st = ring + s * P.stage_bytes;
-        const uint32_t a_st = tmem + kAccCols + (uint32_t)s * kStageCols;
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-          const uint64_t bx =
-              smem_desc_kmajor(st + P.x_off + ks * N * 32, 128, 256);
-          // k16 step ks: 8 columns of the hi half, then of the lo half
-          mma_bf16_ts(tmem, a_st + 8 * ks, bx, idesc,
-                      (it > 0 || ks > 0) ? 1u : 0u);
-          mma_bf16_ts(tmem, a_st + 32 + 8 * ks, bx, idesc, 1u);
-        }
-        mma_commit(empty0 + 8 * s);  // frees the stage when these finish
-      }
-      mma_commit(acc_bar);  // after every MMA issued above
-    }
-  } else {
-    // ---- decoders ----
-    const int wid = warp - 1;
-    const int quarter = warp & 3;  // TMEM lanes this warp may access
-    const int kp = wid >> 2;       // which part of the 64 k of a block
-    const int r = quarter * 32 + lane;
-    const int64_t grow = row0 + r;
-    const bool row_ok = grow < w.n;
-    const uint32_t lane8 = (uint32_t)lane * 8u;
-    const uint32_t lut_base = sbase + P.lut_off;
-    const int64_t gpr = K / 64;  // Format A groups per row (G = 64)
-    const int dt = wid * 32 + lane;  // decoder thread index
-    // Format B codes stream into a per-thread ring of kCodeDepth blocks in
-    // shared memory with cp.async (each thread reads back only the bytes its
-    // own copies wrote), so kCodeDepth - 1 blocks of every row are in flight.
-    const uint32_t code_ring = sbase + P.code_off + r * 64 + kp * kKPT;
-    // Format A: the 16 trits k in [16 kp, 16 kp + 16) of a group lie in its
-    // code bytes m_lo .. m_lo + 3, from trit a_off of byte m_lo on
-    const int m_lo = (kKPT * kp) / 5;
-    const int a_off = kKPT * kp - 5 * m_lo;
-    // x chunks (16 B: one row, 8 k) ride in per-block cp.async groups: chunk
-    // id of a block lands at x_ring(slot) + 16 id, copied and read by one
-    // thread; slot = the block's iteration mod kCodeDepth.
-    auto x_ring = [&](int slot) {
-      return sbase + P.xring_off + (uint32_t)slot * (uint32_t)(N * 128);
-    };
-    // this thread's x chunks: row n, k offset 8c inside a block
-    const __nv_bfloat16 *x_src[kXPerThread];
-    bool x_live[kXPerThread];
-#pragma unroll
-    for (int q = 0; q < kXPerThread; ++q) {
-      const int id = dt + q * kDecoderWarps * 32;
-      const int n = id >> 3, c = id & 7;
-      x_live[q] = id < N * 8;
-      x_src[q] = n < batch ? x + (int64_t)n * ldx + 8 * c : nullptr;
-    }
-    // The next block to issue: its iteration, k-block and ring slot, kept
-    // as counters (blocks are issued in order).
-    int nx_it = 0, nx_slot = 0;
-    int nx_kb = kblocks > 0 ? it_begin % kblocks : 0;
-    auto issue_next = [&]() {
-      if (nx_it < iters) {
-        const uint32_t xd = x_ring(nx_slot);
-#pragma unroll
-        for (int q = 0; q < kXPerThread; ++q) {
-          if (x_live[q]) {
-            const int id = dt + q * kDecoderWarps * 32;
-            const int64_t kk = (int64_t)nx_kb * kBlockK + 8 * (id & 7);
-            const bool ok = x_src[q] != nullptr && kk < K;
-            cp_async16(xd + 16 * id, ok ? x_src[q] + (int64_t)nx_kb * kBlockK : x,
-                       ok ? 16 : 0);
-          }
-        }
-        if constexpr (FMT == TQ_FMT_B) {
-          const uint32_t dst = code_ring + (uint32_t)nx_slot * P.code_slot;
-          const int64_t kk = (int64_t)nx_kb * kBlockK + kKPT * kp;
-          const uint8_t *p = w.codes + (row_ok ? grow : 0) * K + kk;
-#pragma unroll
-          for (int j = 0; j < kKPT / 16; ++j) {
-            const bool ok = row_ok && kk + 16 * j < K;
-            cp_async16(dst + 16 * j, ok ? p + 16 * j : w.codes, ok ? 16 : 0);
-          }
-        }
-      }
-      ++nx_it;
-      nx_slot = nx_slot + 1 == kCodeDepth ? 0 : nx_slot + 1;
-      nx_kb = nx_kb + 1 == kblocks ? 0 : nx_kb + 1;
-    };
-    // Format A windows: the CTA's iterations [g0, g1) split at the plane
-    // boundary into at most two runs, each cut into windows of kWinBlocks.
-    const int g0 = it_begin, g1 = it_begin + iters;
-    const int run0_end =
-        kblocks > 0 ? min(g1, (g0 / kblocks + 1) * kblocks) : g0;
-    const int n_win0 = (run0_end - g0 + kWinBlocks - 1) / kWinBlocks;
-    const int n_win = n_win0 + (g1 - run0_end + kWinBlocks - 1) / kWinBlocks;
-    auto win_lo = [&](int j) {
-      return j < n_win0 ? g0 + kWinBlocks * j : run0_end + kWinBlocks * (j - n_win0);
-    };
-    auto win_hi = [&](int j) {
-      return min(win_lo(j) + kWinBlocks, j < n_win0 ? run0_end : g1);
-    };
-    const int64_t plane_bytes = w.n * gpr * 13;  // Format A code bytes per plane
-    // Every decoder thread copies its share of window j's chunks (chunk i:
-    // row i / 10, the row's code chunk i % 10 < 8 or scale chunk i % 10 - 8)
-    // into slot j % kWinSlots, once all decoders finished the window that
-    // used the slot before; the copies complete on wfull[slot]. Chunks stop
-    // at the end of the plane's codes or scales.
-    auto issue_win = [&](int j) -> bool {
-      if (j >= n_win) return true;
-      const int slot = j % kWinSlots;
-      if (j >= kWinSlots &&
-          !mbar_wait(wempty0 + 8 * slot, ((j / kWinSlots) - 1) & 1))
-        return false;
-      const int gs = win_lo(j);
-      const int plane = gs / kblocks, kb0 = gs - plane * kblocks;
-      const uint8_t *cbase = w.codes + plane * w.codes_plane_stride;
-      const uint8_t *cend = cbase + plane_bytes;
-      const uint16_t *sbase_p = w.scales + plane * w.scales_plane_stride;
-      const uint8_t *send = reinterpret_cast<const uint8_t *>(sbase_p + w.n * gpr);
-      const uint32_t wslot = sbase + P.code_off + (uint32_t)slot * P.code_slot;
-      for (int i = dt; i < kWinChunks; i += kDecoderWarps * 32) {
-        const int row = i / 10, ch = i - 10 * row;
-        const int64_t gr = row0 + row;
-        if (gr >= w.n) continue;
-        const int64_t gi0 = gr * gpr + kb0;
-        const bool is_scale = ch >= 8;
-        const uint8_t *first = is_scale
-            ? reinterpret_cast<const uint8_t *>(sbase_p + gi0)
-            : cbase + gi0 * 13;
-        const uint8_t *src = reinterpret_cast<const uint8_t *>(
-                                 reinterpret_cast<uintptr_t>(first) & ~(uintptr_t)15) +
-                             16 * (is_scale ? ch - 8 : ch);
-        const int64_t left = (is_scale ? send : cend) - src;
-        const int nb = left >= 16 ? 16 : (left > 0 ? (int)left : 0);
-        cp_async16(wslot + (uint32_t)(row * kWinRowBytes + 16 * ch),
-                   nb > 0 ? src : w.codes, nb);
-      }
-      cp_async_mbar_arrive(wfull0 + 8 * slot);
-      return true;
-    };
-    bool ok0 = true;
-    if constexpr (FMT == TQ_FMT_A) {
-      for (int j = 0; j + 1 < kWinSlots; ++j) ok0 = ok0 && issue_win(j);
-    }
-#pragma unroll
-    for (int q = 0; q < kCodeDepth - 1; ++q) {
-      issue_next();
-      cp_async_commit();
-    }
-    if (!__all_sync(0xFFFFFFFFu, ok0)) abort_flag = 1;
-    int wj = 0;                                  // current Format A window
-    int w_lo = n_win > 0 ? win_lo(0) : 0, w_hi = n_win > 0 ? win_hi(0) : 0;
-    uint32_t w_row = 0, c_off0 = 0, s_off0 = 0;  // its row base and offsets
-    int s = 0, cur = 0;    // stage of block it, its x / code ring slot
-    uint32_t e_par = 1;    // parity of the stage's previous use (from round 1)
-    // A block's TMEM stores complete while the next block decodes: its
-    // tcgen05.wait::st and full-barrier arrive come one iteration later.
-    int s_prev = 0;
-    bool pending = false;  // the previous block still awaits its arrive
-    auto arrive_prev = [&]() {
-      tmem_st_wait();
-      tc_fence_before_sync();  // A stores -> ordered before the arrive
-      __syncwarp();
-      if (lane == 0) mbar_arrive(full0 + 8 * s_prev);
-      pending = false;
-    };
-    // Every decision before a warp-wide (.sync.aligned) instruction is made
-    // uniform across the warp.
-    for (int it = 0; it < iters && !__any_sync(0xFFFFFFFFu, abort_flag != 0);
-         ++it) {
-      const int g = it_begin + it;
-      issue_next();  // block it + kCodeDepth - 1
-      cp_async_commit();
-      cp_async_wait<kCodeDepth - 1>();  // this block's x (and B codes) landed
-      uint32_t bits = 0;  // Format A: the thread's 16 trits, 2 bits each
-      uint32_t s_hi = 0, s_lo = 0;
-      uint32_t cw[4];
-      if constexpr (FMT == TQ_FMT_A) {
-        if (g == w_lo) {  // first block of window wj
-          bool ok = issue_win(wj + kWinSlots - 1);
-          ok = ok && mbar_wait(wfull0 + 8 * (wj % kWinSlots), (wj / kWinSlots) & 1);
-          if (!__all_sync(0xFFFFFFFFu, ok)) {
-            abort_flag = 1;
+        const uint32_t d = tmem + (uint32_t)buf * kAccCols;
+        for (int it = it0; it < it1; ++it) {
+          if (!mbar_wait(B0 + kBarXFull + 8 * xs,
+                         (uint32_t)(ux / P.x_stages) & 1u, abort_addr, lim) ||
+              !mbar_wait(B0 + kBarAFull + 8 * as,
+                         (uint32_t)(ua / kAStages) & 1u, abort_addr, lim)) {
+            if constexpr (CK) ck_record(24, (uint64_t)ux << 32 | (uint32_t)ua);
+            ok = false;
             break;
           }
-          const int plane = g / kblocks, kb0 = g - plane * kblocks;
-          const int64_t gi0 = (row_ok ? grow : 0) * gpr + kb0;
-          c_off0 = (uint32_t)(reinterpret_cast<uintptr_t>(
-                                  w.codes + plane * w.codes_plane_stride + gi0 * 13) & 15);
-          s_off0 = (uint32_t)(reinterpret_cast<uintptr_t>(
-                                  w.scales + plane * w.scales_plane_stride + gi0) & 15);
-          w_row = sbase + P.code_off + (uint32_t)(wj % kWinSlots) * P.code_slot +
-                  (uint32_t)(r * kWinRowBytes);
-        }
-        if (row_ok) {
-          const uint32_t off = c_off0 + 13u * (uint32_t)(g - w_lo) + (uint32_t)m_lo;
-          uint32_t w0, w1;
-          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w0) : "r"(w_row + (off & ~3u)));
-          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w1) : "r"(w_row + (off & ~3u) + 4));
-          const uint32_t word = __funnelshift_r(w0, w1, 8u * (off & 3u));
-          const uint16_t *tab =
-              reinterpret_cast<const uint16_t *>(smem + P.lut_off);
-          const uint32_t t0 = tab[word & 0xFFu], t1 = tab[(word >> 8) & 0xFFu],
-                         t2 = tab[(word >> 16) & 0xFFu], t3 = tab[word >> 24];
-          const uint32_t lo32 = t0 | t1 << 10 | t2 << 20 | t3 << 30;
-          bits = __funnelshift_r(lo32, t3 >> 2, 2u * (uint32_t)a_off);
-          uint16_t sbits;
-          asm volatile("ld.shared.u16 %0, [%1];"
-                       : "=h"(sbits)
-                       : "r"(w_row + kWinRowCodes + s_off0 + 2u * (uint32_t)(g - w_lo)));
-          const float sf = __half2float(__ushort_as_half(sbits));
-          s_hi = bf16_bits_rn(sf);
-          s_lo = bf16_bits_rn(sf - __uint_as_float(s_hi << 16));
-          s_hi |= s_hi << 16;  // both halves of a pair
-          s_lo |= s_lo << 16;
-        }
-        if (g + 1 == w_hi) {  // this thread is done reading window wj
-          mbar_arrive(wempty0 + 8 * (wj % kWinSlots));
-          ++wj;
-          if (wj < n_win) {
-            w_lo = win_lo(wj);
-            w_hi = win_hi(wj);
+          tc_fence_after_sync();
+          ck_trace<CK>(trace, 2, t, it, 1);
+          const uint32_t xb = x_ring + (uint32_t)xs * P.x_stage_bytes;
+          const uint32_t a = tmem + kAStage0 + (uint32_t)as * kAStageCols;
+          if constexpr (CK) {
+            if ((d & 0xFFFFu) + (uint32_t)n_pad > 2 * kAccCols || (d >> 16) != 0u)
+              ck_record(8, d);
+            if ((a & 0xFFFFu) + 128u > kTmemCols || (a >> 16) != 0u) ck_record(9, a);
+            ck_smem<CK>(W, xb, P.x_stage_bytes, 10);
           }
+#pragma unroll
+          for (int k16 = 0; k16 < 8; ++k16) {
+            const uint64_t bd =
+                smem_desc_kmajor(xb + (uint32_t)(2 * k16) * lbo, lbo, 128u);
+            mma_bf16_ts(d, a + 8u * (uint32_t)k16, bd, idesc,
+                        (it > it0 || k16 > 0) ? 1u : 0u);
+            mma_bf16_ts(d, a + 64u + 8u * (uint32_t)k16, bd, idesc, 1u);
+          }
+          mma_commit(B0 + kBarXEmpty + 8 * xs);
+          mma_commit(B0 + kBarAEmpty + 8 * as);
+          ++ux;
+          xs = xs + 1 == P.x_stages ? 0 : xs + 1;
+          ++ua;
+          as = as + 1 == kAStages ? 0 : as + 1;
+        }
+        if (!ok) break;
+        ck_trace<CK>(trace, 2, t, 0, 2);
+        mma_commit(B0 + kBarAccFull + 8 * buf);
+        ++ca;
+        ck_trace<CK>(trace, 2, t, 0, 3);
+      }
+      // The arrives of tcgen05.commit land asynchronously, when the MMAs
+      // finish: before the CTA may leave (and its shared memory go to the
+      // next CTA), every arrive this thread caused must have landed. The
+      // drain commit covers every issued MMA; the last commit to each x and
+      // A stage is then observed on its own barrier (those barriers complete
+      // only through these commits). Bounded waits, also after a time-out.
+      mma_commit(B0 + kBarDrain);
+      mbar_wait(B0 + kBarDrain, 0u);
+      for (int j = ux > P.x_stages ? ux - P.x_stages : 0; j < ux; ++j)
+        mbar_wait(B0 + kBarXEmpty + 8 * (j % P.x_stages),
+                  (uint32_t)(j / P.x_stages) & 1u);
+      for (int j = ua > kAStages ? ua - kAStages : 0; j < ua; ++j)
+        mbar_wait(B0 + kBarAEmpty + 8 * (j % kAStages),
+                  (uint32_t)(j / kAStages) & 1u);
+      for (int j = ca > 2 ? ca - 2 : 0; j < ca; ++j)
+        mbar_wait(B0 + kBarAccFull + 8 * (j & 1), (uint32_t)(j >> 1) & 1u);
+    }
+  } else if (warp < kWarpDec) {
+    // ---- epilogue -----------------------------------------------------------
+    const int q = warp & 3;  // tensor-memory lane quarter
+    const int r = 32 * q + lane;
+    bool dead = false;
+    int i = 0;
+    for (int t = cid; t < P.tiles; t += nclusters, ++i) {
+      const int64_t row0 = (int64_t)t * kTileM;
+      const int buf = i & 1;
+      uint32_t v[64];
+#pragma unroll
+      for (int c = 0; c < 64; ++c) v[c] = 0x7FC00000u;  // NaN unless read
+      if (!dead) {
+        const bool got = mbar_wait(B0 + kBarAccFull + 8 * buf,
+                                   (uint32_t)(i >> 1) & 1u, abort_addr, lim);
+        if constexpr (CK) if (!got) ck_record(25, (uint64_t)i);
+        dead = !__all_sync(0xFFFFFFFFu, got);
+        if (!dead) {
+          tc_fence_after_sync();
+          if (lane == 0) ck_trace<CK>(trace, 3 + (q == 0 ? 0 : 1) * 0, t, 0, 1 + 16 * q);
+          const uint32_t ta =
+              tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)buf * kAccCols;
+          if constexpr (CK) ck_tmem<CK>(ta, (uint32_t)n_pad, (uint32_t)(32 * q), 11);
+          __syncwarp();  // converged for the warp-wide loads
+          tmem_ld16(ta, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
+          if (n_pad > 16)
+            tmem_ld16(ta + 16, *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
+          if (n_pad > 32)
+            tmem_ld16(ta + 32, *reinterpret_cast<uint32_t(*)[16]>(&v[32]));
+          if (n_pad > 48)
+            tmem_ld16(ta + 48, *reinterpret_cast<uint32_t(*)[16]>(&v[48]));
+          tmem_ld_wait();
+          if (lane == 0) ck_trace<CK>(trace, 4, t, 0, 2 + 16 * q);
+          tc_fence_before_sync();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(B0 + kBarAccEmpty + 8 * buf);
+        }
+      }
+      if (ks == 1) {
+        // the whole K: this thread's row goes straight to y (NaN after a
+        // time-out)
+        const int64_t row = row0 + r;
+        if (row < N) {
+          float scale = 1.0f;
+          if constexpr (FMT == TQ_FMT_B) {
+            if (w.scales != nullptr)
+              scale = __half2float(__ushort_as_half(w.scales[row / w.rps]));
+          }
+#pragma unroll
+          for (int b = 0; b < 64; ++b)
+            if (b < nb) {
+              if constexpr (CK) {
+                if (b >= batch) {
+                  ck_record(12, (uint64_t)row);
+                  continue;
+                }
+              }
+              y[(int64_t)b * ldy + row] = scale * __uint_as_float(v[b]);
+            }
         }
       } else {
-        const uint32_t src = code_ring + (uint32_t)cur * P.code_slot;
-        asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
-                     : "=r"(cw[0]), "=r"(cw[1]), "=r"(cw[2]), "=r"(cw[3])
-                     : "r"(src));
-        if (!row_ok) {
+        // a K slice (one tile per CTA): the partial row goes to this CTA's
+        // shared buffer; the owners add the cluster's partials after the
+        // cluster barrier at the end of the kernel
+        if constexpr (CK) ck_smem<CK>(W, P.red + delta + (uint32_t)(r * n_pad * 4), (uint32_t)n_pad * 4u, 14);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) cw[q] = 0x79797979u;  // weight 0
-        }
+        for (int c = 0; c < 64; ++c)
+          if (c < n_pad) part[r * n_pad + c] = __uint_as_float(v[c]);
       }
-      // decode this thread's kKPT k of its row: kKPT/2 hi and lo bf16 pairs
-      uint32_t hi[kKPT / 2], lo[kKPT / 2];
-#pragma unroll
-      for (int cc = 0; cc < kKPT / 8; ++cc) {
-        uint32_t h4[4], l4[4];
-        if constexpr (FMT == TQ_FMT_B)
-          decode8_b(cw[2 * cc], cw[2 * cc + 1], lut_base, lane8, h4, l4);
-        else
-          decode8_a(bits, cc, s_hi, s_lo, lut_base + 512, h4, l4);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          hi[4 * cc + q] = h4[q];
-          lo[4 * cc + q] = l4[q];
-        }
-      }
-      if (pending) arrive_prev();
-      if (it >= kStages) {
-        const bool ok = mbar_wait(empty0 + 8 * s, e_par);
-        if (!__all_sync(0xFFFFFFFFu, ok)) {
-          abort_flag = 1;
-          break;
-        }
-      }
-      tc_fence_after_sync();  // the stage's MMAs are done reading it
-      {
-        const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + kAccCols +
-                            (uint32_t)s * kStageCols +
-                            (uint32_t)(kKPT / 2) * (uint32_t)kp;
-        tmem_st_cols(ta, hi);
-        tmem_st_cols(ta + 32, lo);
-      }
-      uint8_t *st = smem + P.ring_off + s * P.stage_bytes;
-      // x tile: N rows x 64 k, 16 bytes per chunk, from this thread's ring
-      {
-        const uint32_t xs = x_ring(cur);
-#pragma unroll
-        for (int q = 0; q < kXPerThread; ++q) {
-          const int id = dt + q * kDecoderWarps * 32;
-          if (id < N * 8) {
-            uint4 v;
-            asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
-                         : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                         : "r"(xs + 16 * id));
-            *reinterpret_cast<uint4 *>(st + P.x_off +
-                                       tile_off(id >> 3, 8 * (id & 7), N)) = v;
-          }
-        }
-      }
-      fence_async_shared();   // x tile -> async proxy (MMA operand B)
-      s_prev = s;
-      pending = true;
-      if (++s == kStages) {
-        s = 0;
-        e_par ^= 1u;
-      }
-      cur = cur + 1 == kCodeDepth ? 0 : cur + 1;
     }
-    if (pending) arrive_prev();
-    cp_async_wait<0>();
-    // ---- epilogue: warps of the first half read their TMEM lane quarter ----
-    if (kp == 0) {
-      const bool ok = iters == 0 || mbar_wait(acc_bar, 0);
-      if (!ok) abort_flag = 1;
-      tc_fence_after_sync();
-      float scale = 1.0f;
-      if constexpr (FMT == TQ_FMT_B) {
-        if (row_ok && w.scales != nullptr)
-          scale = __half2float(__ushort_as_half(w.scales[grow / w.rps]));
-      }
-      float *part = reinterpret_cast<float *>(smem + P.ring_off);  // [128][N]
-      for (int cb = 0; cb < N / 16; ++cb) {
-        uint32_t v[16];
-        tmem_ld16(tmem + ((uint32_t)(quarter * 32) << 16) + cb * 16, v);
-        tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int b = cb * 16 + i;
-          float val = iters == 0 ? 0.0f : __uint_as_float(v[i]);
-          if (abort_flag) val = __int_as_float(0x7FC00000);
-          if (P.ks_count > 1) {
-            part[r * N + b] = val;  // summed across the cluster below
-          } else if (row_ok && b < batch) {
-            y[(int64_t)b * ldy + grow] = scale * val;
-          }
+  } else {
+    // ---- decoders -----------------------------------------------------------
+    const int q = warp & 3;
+    const int kp = (warp - kWarpDec) >> 2;  // which 64-k half of the block
+    const int r = 32 * q + lane;
+    const uint32_t lane_tab =
+        tab | (uint32_t)lane << (FMT == TQ_FMT_B ? 2 : 3);
+    const uint32_t t_hi =
+        tmem + ((uint32_t)(32 * q) << 16) + kAStage0 + 32u * (uint32_t)kp;
+    const bool skip_first = P.skip_first_arrive != 0;
+    int cs = 0, uc = 0, as = 0, ua = 0;
+    bool ok = true;
+    for (int t = cid; ok && t < P.tiles; t += nclusters) {
+      const int64_t row = (int64_t)t * kTileM + r;
+      const bool row_ok = row < N;
+      for (int ws = it0; ws < it1;) {
+        const int we = window_end(ws, it1, P.kblocks, kWin);
+        ok = __all_sync(0xFFFFFFFFu,
+                        mbar_wait(B0 + kBarCodeFull + 8 * cs,
+                                  (uint32_t)(uc / P.code_stages) & 1u,
+                                  abort_addr, lim));
+        if constexpr (CK) if (!ok && lane == 0) ck_record(28, (uint64_t)uc);
+        if (!ok) break;
+        const uint32_t slot =
+            code_stage(cs) + (uint32_t)r * (FMT == TQ_FMT_B ? kBRow : kARow);
+        // Format A: this row's byte skews inside its code and scale slots
+        uint32_t cskew = 0, sskew = 0;
+        int64_t g0 = 0;
+        if constexpr (FMT == TQ_FMT_A) {
+          const int plane = ws / P.kblocks;
+          g0 = 2 * (int64_t)(ws - plane * P.kblocks);
+          const int64_t gi = (row_ok ? row : 0) * gpr + g0;
+          cskew = (uint32_t)((reinterpret_cast<uintptr_t>(w.codes) +
+                              (uintptr_t)(plane * w.codes_plane_stride) +
+                              (uintptr_t)(gi * 13)) &
+                             15);
+          sskew = (uint32_t)((reinterpret_cast<uintptr_t>(w.scales) +
+                              (uintptr_t)(2 * (plane * w.scales_plane_stride +
+                                               gi))) &
+                             15);
         }
+        for (int it = ws; it < we; ++it) {
+          if (ua >= kAStages) {
+            ok = __all_sync(0xFFFFFFFFu,
+                            mbar_wait(B0 + kBarAEmpty + 8 * as,
+                                      (uint32_t)((ua / kAStages) + 1) & 1u,
+                                      abort_addr, lim));
+            if constexpr (CK) if (!ok && lane == 0) ck_record(29, (uint64_t)ua);
+            if (!ok) break;
+          }
+          tc_fence_after_sync();
+          if (lane == 0 && q == 0 && kp == 0) ck_trace<CK>(trace, 5, t, it, 1);
+          uint32_t hi[32], lo[32];
+          if constexpr (FMT == TQ_FMT_B) {
+            const uint32_t src = slot + 64u * (uint32_t)kp;
+            uint32_t cw[16];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const uint4 v4 = lds128(ck_smem<CK>(W, src + 16u * (uint32_t)j, 16u, 16));
+              cw[4 * j] = v4.x;
+              cw[4 * j + 1] = v4.y;
+              cw[4 * j + 2] = v4.z;
+              cw[4 * j + 3] = v4.w;
+            }
+            decode_b(cw, lane_tab, hi, lo);
+            // k past K (in the last block) and rows past N: zero weights
+            // (selects, no branch: the tcgen05.st below is warp-wide)
+            const int64_t kv = K - ((int64_t)it * kKB + 64 * kp);
+            if (__any_sync(0xFFFFFFFFu, kv < 64 || !row_ok)) {
+#pragma unroll
+              for (int m = 0; m < 32; ++m) {
+                const uint32_t keep = (row_ok && 2 * m < kv) ? 0xFFFFFFFFu : 0u;
+                hi[m] &= keep;
+                lo[m] &= keep;
+              }
+            }
+          } else {
+            const int gi = 2 * (it - ws) + kp;  // group inside the window
+            const bool valid = row_ok && g0 + gi < gpr;
+            const uint32_t o = cskew + 13u * (uint32_t)gi;
+            const uint32_t wa = slot + (o & ~3u);
+            const uint32_t sh = 8u * (o & 3u);
+            const uint32_t w0 = lds32(ck_smem<CK>(W, wa, 4u, 17)),
+                           w1 = lds32(ck_smem<CK>(W, wa + 4, 4u, 17)),
+                           w2 = lds32(ck_smem<CK>(W, wa + 8, 4u, 17)),
+                           w3 = lds32(ck_smem<CK>(W, wa + 12, 4u, 17));
+            const uint32_t b[4] = {__funnelshift_r(w0, w1, sh),
+                                   __funnelshift_r(w1, w2, sh),
+                                   __funnelshift_r(w2, w3, sh), w3 >> sh};
+            const uint32_t sa = slot + kARowCodes + sskew + 2u * (uint32_t)gi;
+            const uint32_t sbits =
+                (lds32(ck_smem<CK>(W, sa & ~3u, 4u, 18)) >> (8u * (sa & 2u))) & 0xFFFFu;
+            const float sf = __half2float(__ushort_as_half((unsigned short)sbits));
+            const uint32_t h = bf16_bits_rn(sf);
+            const uint32_t l = bf16_bits_rn(sf - __uint_as_float(h << 16));
+            decode_a(b, lane_tab, h ^ 0x8000u, h, l ^ 0x8000u, l, hi, lo);
+            if (__any_sync(0xFFFFFFFFu, !valid)) {
+              const uint32_t keep = valid ? 0xFFFFFFFFu : 0u;
+#pragma unroll
+              for (int m = 0; m < 32; ++m) {
+                hi[m] &= keep;
+                lo[m] &= keep;
+              }
+            }
+          }
+          uint32_t ta = t_hi + (uint32_t)as * kAStageCols;
+          if constexpr (CK) ta = ck_tmem<CK>(ta, 96u, (uint32_t)(32 * q), 19);
+          __syncwarp();  // converged for the warp-wide stores
+          tmem_st32(ta, hi);
+          tmem_st32(ta + 64u, lo);
+          tmem_st_wait();
+          if (lane == 0 && q == 0 && kp == 0) ck_trace<CK>(trace, 5, t, it, 2);
+          tc_fence_before_sync();
+          __syncwarp();
+          if (lane == 0 && !(skip_first && ua == 0))
+            mbar_arrive(B0 + kBarAFull + 8 * as);
+          ++ua;
+          as = as + 1 == kAStages ? 0 : as + 1;
+        }
+        if (!ok) break;
+        // this warp is done reading the window
+        __syncwarp();
+        if (lane == 0) mbar_arrive(B0 + kBarCodeEmpty + 8 * cs);
+        ws = we;
+        ++uc;
+        cs = cs + 1 == P.code_stages ? 0 : cs + 1;
       }
     }
   }
+
   tc_fence_before_sync();
   __syncthreads();
-  if (P.ks_count > 1) {
-    // Sum the cluster's partial tiles through distributed shared memory in
-    // rank order (deterministic); this CTA finishes its share of the rows.
+  if (threadIdx.x == 0) ck_trace<CK>(trace, 6, 0xFFFF, 0, 1);
+  if (ks > 1) {
+    // Add the cluster's partial tiles through distributed shared memory in
+    // rank order (deterministic); this CTA finishes the rows it owns. The
+    // second barrier keeps every CTA alive while peers read its partials.
     namespace cg = cooperative_groups;
     cg::cluster_group cluster = cg::this_cluster();
+    __syncwarp();
     cluster.sync();
-    const float *part = reinterpret_cast<const float *>(smem + P.ring_off);
-    const int r_lo = kTileM * ks / P.ks_count;
-    const int r_hi = kTileM * (ks + 1) / P.ks_count;
-    for (int i = threadIdx.x; i < (r_hi - r_lo) * N; i += blockDim.x) {
-      const int rr = r_lo + i / N, b = i % N;
-      const int64_t gr = row0 + rr;
-      if (gr >= w.n || b >= batch) continue;
-      float sum = 0.0f;
-      for (int q = 0; q < P.ks_count; ++q)
-        sum += cluster.map_shared_rank(part, q)[rr * N + b];
-      float scale = 1.0f;
-      if constexpr (FMT == TQ_FMT_B) {
-        if (w.scales != nullptr)
-          scale = __half2float(__ushort_as_half(w.scales[gr / w.rps]));
+    if (warp >= kWarpEpi && warp < kWarpDec && cid < P.tiles) {
+      const int et = (int)threadIdx.x - 32 * kWarpEpi;  // 0..127
+      const int64_t row0 = (int64_t)cid * kTileM;
+      const int own = r_hi - r_lo;
+      for (int idx = et; idx < own * nb; idx += 128) {
+        const int orr = idx % own, b = idx / own;
+        float sum = 0.0f;
+        for (int p = 0; p < ks; ++p)
+          sum += cluster.map_shared_rank(part, p)[(r_lo + orr) * n_pad + b];
+        const int64_t row = row0 + r_lo + orr;
+        if (row < N) {
+          float scale = 1.0f;
+          if constexpr (FMT == TQ_FMT_B) {
+            if (w.scales != nullptr)
+              scale = __half2float(__ushort_as_half(w.scales[row / w.rps]));
+          }
+          y[(int64_t)b * ldy + row] = scale * sum;
+        }
       }
-      y[(int64_t)b * ldy + gr] = scale * sum;
     }
-    cluster.sync();  // no CTA leaves while others read its partials
+    __syncwarp();
+    cluster.sync();
   }
-  if (warp == 0) {
+  if (warp == kWarpMma) {
+    __syncwarp();  // converged for the warp-wide free
     tc_fence_after_sync();
     tmem_dealloc(tmem, kTmemCols);
+    if (lane == 0) ck_trace<CK>(trace, 7, 0xFFFF, 0, 1);
   }
 }
 
-TcParams plan_tc(int fmt, int64_t batch) {
-  TcParams P{};
-  const int64_t b = batch < kMaxN ? batch : kMaxN;
-  P.n_pad = (int)((b + 15) / 16 * 16);
-  P.stage_bytes = P.n_pad * kBlockK * 2;
-  P.x_off = 0;
-  P.ring_off = 0;
-  P.code_slot = kTileM * (fmt == TQ_FMT_A ? kWinRowBytes : 64);
-  P.code_off = kStages * P.stage_bytes;
-  P.xring_off = P.code_off + (fmt == TQ_FMT_A ? kWinSlots : kCodeDepth) * P.code_slot;
-  P.lut_off = P.xring_off + kCodeDepth * P.n_pad * 128;
-  const int table = fmt == TQ_FMT_B ? kLutBytes : 512 + 128;
-  P.bar_off = P.lut_off + table;
-  P.tmem_slot_off = P.bar_off + (2 * kStages + 1 + 2 * kWinSlots) * 8 + 8;
-  P.smem = (size_t)P.tmem_slot_off + 16;
-  // one CTA per SM: each allocates the whole tensor memory
-  if (P.smem < 120 * 1024) P.smem = 120 * 1024;
-  return P;
+// ---- host side ---------------------------------------------------------------
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault,
+                                &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
 }
 
-// Cluster size (K slices per tile): the one that best fills whole waves of
-// one CTA per SM, preferring no split.
-int pick_ks(int64_t tiles, int iters, int sms) {
-  int best = 1;
-  double best_eff = 0.0;
+// Shared-memory plan for clusters of `ks`; false if it does not fit. The
+// dynamic window starts at `base` (the per-CTA reserved shared memory).
+bool plan_smem(int fmt, int n_pad, int ks, uint32_t base, TcPlan *P) {
+  P->n_pad = n_pad;
+  P->ks = ks;
+  P->base = base;
+  const uint32_t end = base + (uint32_t)kSmemMax;
+  const uint32_t tab = (base + 0xFFFFu) & ~0xFFFFu;
+  if (tab + 0x10000u > end) return false;
+  P->tab = tab;
+  P->code_stage_bytes = kTileM * (fmt == TQ_FMT_B ? kBRow : kARow);
+  P->x_stage_bytes = (uint32_t)n_pad * kKB * 2u;
+  P->x_stages = n_pad <= 32 ? kMaxXStages : 3;
+  // with a split of K, every CTA keeps its partial tile [128][n_pad] fp32
+  const uint32_t red_bytes = ks > 1 ? (uint32_t)(kTileM * n_pad * 4) : 0u;
+  // below the table: code stages
+  const uint32_t lo0 = (base + 127u) & ~127u;
+  P->code_lo = lo0;
+  P->code_lo_n = (int)((tab - lo0) / P->code_stage_bytes);
+  // above it: barriers, x ring, reduction buffer, further code stages
+  uint32_t a = tab + 0x10000u;
+  P->bars = a;
+  a += kBarBytes;
+  a = (a + 127u) & ~127u;
+  P->x_ring = a;
+  a += (uint32_t)P->x_stages * P->x_stage_bytes;
+  P->red = a;
+  a += red_bytes;
+  a = (a + 127u) & ~127u;
+  P->code_hi = a;
+  if (a > end) return false;
+  int hi_n = (int)((end - a) / P->code_stage_bytes);
+  if (P->code_lo_n > kMaxCodeStages) P->code_lo_n = kMaxCodeStages;
+  if (P->code_lo_n + hi_n > kMaxCodeStages) hi_n = kMaxCodeStages - P->code_lo_n;
+  P->code_stages = P->code_lo_n + hi_n;
+  if (P->code_stages < 2) return false;
+  const uint32_t top = hi_n > 0
+                           ? P->code_hi + (uint32_t)hi_n * P->code_stage_bytes
+                           : P->red + red_bytes;
+  P->smem = (size_t)(top - base);
+  return P->smem <= (size_t)kSmemMax;
+}
+
+// Clusters of `ks` CTAs (one per SM) that can be resident together.
+int resident_clusters(const void *kern, int ks, size_t smem) {
+  // An error already pending belongs to the caller: leave it and skip.
+  if (cudaPeekAtLastError() != cudaSuccess) return 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)ks, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)ks;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+    cudaGetLastError();  // the query's own error
+    return 0;
+  }
+  return n;
+}
+
+template <int FMT, bool CK>
+cudaError_t launch_tc_as(const WeightsView &w, const __nv_bfloat16 *x,
+                      int64_t batch, int64_t ldx, float *y, int64_t ldy,
+                      cudaStream_t stream) {
+  auto kern = gemm_tc_kernel<FMT, CK>;
+  cudaError_t e = ensure_smem_limit<gemm_tc_kernel<FMT, CK>>(kSmemMax);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 148, reserved = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  e = cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock,
+                             dev);
+  if (e != cudaSuccess) return e;
+  const int n_pad = (int)((batch + 15) / 16 * 16);
+  const int kblocks = (int)((w.k + kKB - 1) / kKB);
+  const int iters = (FMT == TQ_FMT_A ? w.planes : 1) * kblocks;
+  const int64_t tiles = (w.n + kTileM - 1) / kTileM;
+  if (tiles > (1 << 30) || iters < 1) return cudaErrorInvalidValue;
+
+  // Cluster size: the K split whose resident clusters finish the tiles with
+  // the fewest iterations per CTA (ceil(tiles / resident clusters) waves of
+  // ceil(iters / ks) blocks, plus a per-tile allowance), preferring no split.
+  static std::atomic<int> occ_cache[16][2][4][9];  // per instantiation
+  TcPlan best{};
+  int best_clusters = 0;
+  int64_t best_cost = -1;
   for (int ks = 1; ks <= 8 && ks <= iters; ++ks) {
-    const double ctas = (double)(tiles * ks);
-    const double waves = ctas / sms;
-    const double eff = waves / ceil(waves) - 0.02 * (ks - 1);
-    if (eff > best_eff + 1e-9) {
-      best_eff = eff;
-      best = ks;
+    TcPlan P{};
+    if (!plan_smem(FMT, n_pad, ks, (uint32_t)reserved, &P)) continue;
+    std::atomic<int> *slot =
+        dev < 16 ? &occ_cache[dev][FMT - 1][n_pad / 16 - 1][ks] : nullptr;
+    int c = slot ? slot->load() : 0;
+    if (c <= 0) {
+      c = resident_clusters(reinterpret_cast<const void *>(kern), ks, P.smem);
+      if (c <= 0 && ks == 1) c = sms;
+      if (slot && c > 0) slot->store(c);
+    }
+    if (c <= 0) continue;
+    // ks = 1: persistent CTAs walk the tiles; ks > 1: one tile per cluster
+    // (the partials are added at the end of the kernel), each wave paying
+    // the set-up again
+    const int64_t clusters = ks == 1 ? (c < tiles ? c : tiles) : tiles;
+    const int64_t waves = (tiles + c - 1) / c;
+    const int64_t cost =
+        waves * (((int64_t)iters + ks - 1) / ks + (ks == 1 ? 2 : 4));
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = P;
+      best_clusters = (int)clusters;
     }
   }
-  return best;
+  if (best_cost < 0) return cudaErrorInvalidConfiguration;
+  best.tiles = (int)tiles;
+  best.kblocks = kblocks;
+  best.iters = iters;
+  const uint64_t tw = g_test_wait_ns.load();
+  best.wait_ns = tw ? tw : kWaitLimitNs;
+  best.skip_first_arrive = g_test_skip_first_arrive.load();
+
+  // x as a 2-D tensor: K bf16 per row, `batch` rows ldx apart, boxes of
+  // 8 k x n_pad rows (rows past the batch and k past K read as zero).
+  auto encode = encode_fn();
+  if (encode == nullptr) return cudaErrorNotSupported;
+  CUtensorMap tmap;
+  cuuint64_t dims[2] = {(cuuint64_t)w.k, (cuuint64_t)batch};
+  cuuint64_t strides[1] = {(cuuint64_t)ldx * 2};
+  cuuint32_t box[2] = {8u, (cuuint32_t)n_pad};
+  cuuint32_t estr[2] = {1u, 1u};
+  if (encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+             const_cast<__nv_bfloat16 *>(x), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(best_clusters * best.ks), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = best.smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)best.ks;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  unsigned long long *trace =
+      CK ? reinterpret_cast<unsigned long long *>(g_test_trace.load()) : nullptr;
+  return cudaLaunchKernelEx(&cfg, kern, w, batch, y, ldy, best, tmap, trace);
 }
 
 template <int FMT>
 cudaError_t launch_tc(const WeightsView &w, const __nv_bfloat16 *x,
                       int64_t batch, int64_t ldx, float *y, int64_t ldy,
                       cudaStream_t stream) {
-  TcParams P = plan_tc(FMT, batch);
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t tiles = (w.n + kTileM - 1) / kTileM;
-  const int kblocks = (int)((w.k + kBlockK - 1) / kBlockK);
-  const int iters = (FMT == TQ_FMT_A ? w.planes : 1) * kblocks;
-  P.ks_count = pick_ks(tiles, iters, sms);
-  auto kern = gemm_tc_kernel<FMT>;
-  if (P.smem > 227 * 1024) return cudaErrorInvalidValue;
-  cudaError_t e = ensure_smem_limit<gemm_tc_kernel<FMT>>(227 * 1024);
-  if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(tiles * P.ks_count), 1, 1);
-  cfg.blockDim = dim3(TcCfg<FMT>::kThreads, 1, 1);
-  cfg.dynamicSmemBytes = P.smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)P.ks_count;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, w, x, batch, ldx, y, ldy, P);
+  if (g_test_self_check.load() != 0)
+    return launch_tc_as<FMT, true>(w, x, batch, ldx, y, ldy, stream);
+  return launch_tc_as<FMT, false>(w, x, batch, ldx, y, ldy, stream);
 }
 
 }  // namespace
 
+cudaError_t tc_check_record(uint64_t out[4], bool reset) {
+  cudaError_t e = cudaMemcpyFromSymbol(out, g_tc_check, sizeof(g_tc_check));
+  if (e != cudaSuccess || !reset) return e;
+  const unsigned long long zero[4] = {0, 0, 0, 0};
+  return cudaMemcpyToSymbol(g_tc_check, zero, sizeof(zero));
+}
+
 bool gemm_tc_supported(const WeightsView &w, int64_t batch) {
-  if (batch < 1) return false;
+  if (batch < 1 || w.k < 1) return false;
   if (w.format == TQ_FMT_B) return true;
   return w.format == TQ_FMT_A && w.group == 64;
 }

@@ -5,6 +5,16 @@
 
 namespace tq {
 
+// Test hooks of the tensor-core kernel (tq_testing.h).
+extern std::atomic<uint64_t> g_test_wait_ns;
+extern std::atomic<int> g_test_skip_first_arrive;
+// Kernel family forced by tq_testing_force_linear_path (0 = automatic).
+extern std::atomic<int> g_test_force_path;
+// Self-checking tensor-core kernel (tq_testing_tc_self_check) and its record.
+extern std::atomic<int> g_test_self_check;
+extern std::atomic<unsigned long long> g_test_trace;
+cudaError_t tc_check_record(uint64_t out[4], bool reset);
+
 // One warp per row; any shape the boundary accepts.
 cudaError_t linear_simple(const WeightsView &w, const __nv_bfloat16 *x,
                           int64_t batch, int64_t ldx, float *y, int64_t ldy,

@@ -1,10 +1,12 @@
-// sm_100 asynchronous-copy primitives used by the streaming kernels: shared
-// memory mbarriers and 1-D bulk copies (the TMA engine) global -> shared.
-// Written from the PTX ISA descriptions of mbarrier and cp.async.bulk.
+// sm_100 asynchronous-copy and synchronisation primitives used by the fused
+// GEMM: shared-memory mbarriers, 1-D bulk copies and 2-D tensor copies (the
+// TMA engine) global -> shared. Written from the PTX ISA descriptions of
+// mbarrier, cp.async.bulk and cp.async.bulk.tensor.
 //
 // Every wait is bounded: it polls with try_wait until the barrier phase
-// completes or a time limit (%globaltimer, nanoseconds) passes, and reports
-// which happened, so a kernel can never spin forever.
+// completes, a shared abort word becomes non-zero, or a time limit
+// (%globaltimer, nanoseconds) passes, and reports which happened, so a kernel
+// can never spin forever.
 #pragma once
 
 #include <stdint.h>
@@ -28,7 +30,7 @@ __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
                : "memory");
 }
 
-// Make barrier initialisation visible to the async (bulk-copy) proxy.
+// Make barrier initialisation visible to the async proxy and to the cluster.
 __device__ __forceinline__ void mbar_init_fence() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
@@ -38,6 +40,7 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
                : "memory");
 }
 
+// Arrive and add `bytes` to the transaction count of the current phase.
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar,
                                                       uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(
@@ -58,7 +61,37 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait for the phase with the given parity to complete; false on time-out.
+__device__ __forceinline__ int ld_volatile_s32(uint32_t addr) {
+  int v;
+  asm volatile("ld.volatile.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr)
+               : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_volatile_s32(uint32_t addr, int v) {
+  asm volatile("st.volatile.shared.u32 [%0], %1;" ::"r"(addr), "r"(v)
+               : "memory");
+}
+
+// Wait for the phase with the given parity to complete. Returns false when
+// the wait gave up: the word at `abort_addr` became non-zero, or `limit_ns`
+// passed (then the abort word is set, so that the CTA's other roles stop).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
+                                          uint32_t abort_addr,
+                                          uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (;;) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (ld_volatile_s32(abort_addr) != 0) return false;
+    if (global_ns() - t0 > limit_ns) {
+      st_volatile_s32(abort_addr, 1);
+      return false;
+    }
+  }
+}
+
+// Wait without an abort word (kernels with a single waiting role).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
@@ -78,6 +111,26 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src,
       "[%0], [%1], %2, [%3];" ::"r"(dst),
       "l"(src), "r"(bytes), "r"(bar)
       : "memory");
+}
+
+// 2-D tensor copy of one box (coordinates c0 innermost, c1) into this CTA's
+// shared memory, completing on `bar`; out-of-range elements read as zero.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap,
+                                            int32_t c0, int32_t c1,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::"
+      "bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(tmap), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+
+// ---- thread-block clusters -------------------------------------------------
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
 }
 
 }  // namespace tq

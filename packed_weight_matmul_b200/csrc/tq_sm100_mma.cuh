@@ -1,6 +1,7 @@
 // sm_100 fifth-generation tensor-core primitives (tcgen05) used by the
-// fused GEMM: tensor-memory allocation, MMA issue with shared-memory operand
-// descriptors, commit to an mbarrier, and tensor-memory loads. Written from
+// fused GEMM: tensor-memory allocation, MMA issue with the A operand in
+// tensor memory and B described in shared memory, commit to an mbarrier, and
+// tensor-memory loads and stores. Written from
 // the PTX ISA descriptions of tcgen05 (field layouts cross-checked against the
 // CUTLASS UMMA descriptor definitions).
 #pragma once
@@ -62,19 +63,6 @@ __device__ __forceinline__ void fence_async_shared() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// D[tmem] (+)= A[smem desc] * B[smem desc]^T, one thread issues.
-__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc,
-                                         uint64_t b_desc, uint32_t idesc,
-                                         uint32_t accumulate) {
-  asm volatile(
-      "{\n .reg .pred p;\n"
-      " setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(
-          d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
 // D[tmem] (+)= A[tmem] * B[smem desc]^T, one thread issues. A (M = 128 rows
 // on the 128 lanes) sits in tensor memory with K along the columns, two
 // 16-bit elements per 32-bit column, the lower k in the low half.
@@ -121,6 +109,23 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr,
       "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]),
       "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]),
       "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+
+// Warp-wide: store 32 consecutive 32-bit columns of this warp's 32 lanes.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr,
+                                          const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(
+          taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]),
+      "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]),
+      "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]),
+      "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]),
+      "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]),
+      "r"(v[30]), "r"(v[31])
       : "memory");
 }
 

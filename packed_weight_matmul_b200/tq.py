@@ -23,7 +23,10 @@ TQ_FMT_A, TQ_FMT_B = 1, 2
 
 # Every entry point declared in include/tq.h.
 ENTRY_POINTS = ("tq_packed_bytes", "tq_build_lut", "tq_quantize_pack",
-                "tq_unpack", "tq_linear", "tq_status_string")
+                "tq_unpack", "tq_linear", "tq_status_string",
+                "tq_encode_b", "tq_testing_linear_wait_fault",
+                "tq_testing_force_linear_path", "tq_testing_tc_self_check",
+                "tq_testing_tc_trace")
 
 
 class TqError(RuntimeError):
@@ -59,8 +62,18 @@ def _load():
     L.tq_unpack.argtypes = [C.POINTER(tq_weights), P, P, P]
     L.tq_linear.restype = C.c_int
     L.tq_linear.argtypes = [C.POINTER(tq_weights), P, i64, i64, P, i64, P]
+    L.tq_encode_b.restype = C.c_int
+    L.tq_encode_b.argtypes = [P, i64, i64, P, C.c_float, i32, P, P, P, P, P]
     L.tq_status_string.restype = C.c_char_p
     L.tq_status_string.argtypes = [C.c_int]
+    L.tq_testing_linear_wait_fault.restype = C.c_int
+    L.tq_testing_linear_wait_fault.argtypes = [i32, C.c_uint64]
+    L.tq_testing_force_linear_path.restype = C.c_int
+    L.tq_testing_force_linear_path.argtypes = [i32]
+    L.tq_testing_tc_self_check.restype = C.c_int
+    L.tq_testing_tc_self_check.argtypes = [i32, P, i32]
+    L.tq_testing_tc_trace.restype = C.c_int
+    L.tq_testing_tc_trace.argtypes = [P]
     return L
 
 
@@ -108,6 +121,41 @@ def tq_build_lut(alpha: float, ladder) -> np.ndarray:
                              lad.ctypes.data_as(C.c_void_p),
                              out.ctypes.data_as(C.c_void_p)), "tq_build_lut")
     return out
+
+
+def tq_testing_linear_wait_fault(withhold_first_arrive: bool,
+                                 wait_limit_ns: int = 0) -> None:
+    """Test hook (include/tq_testing.h): make the tensor-core tq_linear
+    kernels time out on purpose, with a short wait limit."""
+    _check(_lib.tq_testing_linear_wait_fault(int(bool(withhold_first_arrive)),
+                                             int(wait_limit_ns)),
+           "tq_testing_linear_wait_fault")
+
+
+def tq_testing_force_linear_path(path: int) -> None:
+    """Test hook (include/tq_testing.h): 0 automatic dispatch, 1 CUDA-core
+    kernels, 2 tensor-core kernel."""
+    _check(_lib.tq_testing_force_linear_path(int(path)),
+           "tq_testing_force_linear_path")
+
+
+def tq_testing_tc_self_check(enable: bool, read: bool = False,
+                             reset: bool = False):
+    """Test hook (include/tq_testing.h): select the self-checking
+    tensor-core kernel; with read=True return its record (4 integers)."""
+    rec = np.zeros(4, np.uint64)
+    _check(_lib.tq_testing_tc_self_check(
+        int(bool(enable)), rec.ctypes.data_as(C.c_void_p) if read else None,
+        int(bool(reset))), "tq_testing_tc_self_check")
+    return [int(v) for v in rec] if read else None
+
+
+def tq_testing_tc_trace(buffer) -> None:
+    """Test hook (include/tq_testing.h): progress trace of the self-checking
+    tensor-core kernel into a pinned host tensor (int64), or None."""
+    _check(_lib.tq_testing_tc_trace(None if buffer is None else
+                                    buffer.data_ptr()),
+           "tq_testing_tc_trace")
 
 
 def tq_status_string(status: int) -> str:
@@ -163,6 +211,25 @@ def tq_quantize_pack(W, group, planes, codes_out, scales_out, dev_status=None,
                                _stream(stream))
     if check:
         _check(st, "tq_quantize_pack")
+    return st
+
+
+def tq_encode_b(W, ladder, zeta, rows_per_scale, codes_out, rho_out,
+                alpha_out, dev_status=None, stream=None, n=None, k=None,
+                check=True):
+    """Format B encoder: W bf16 [n][k] (device) -> codes_out uint8 [n][k],
+    rho_out fp16 [ceil(n / rows_per_scale)] (None when rows_per_scale = 0),
+    alpha_out fp32 [1] (all device). `ladder` is 5 host floats."""
+    if n is None:
+        n, k = W.shape
+    lad = np.ascontiguousarray(np.asarray(ladder, np.float32))
+    assert lad.shape == (5,)
+    st = _lib.tq_encode_b(_ptr(W), n, k, lad.ctypes.data_as(C.c_void_p),
+                          C.c_float(zeta), rows_per_scale, _ptr(codes_out),
+                          _ptr(rho_out), _ptr(alpha_out), _ptr(dev_status),
+                          _stream(stream))
+    if check:
+        _check(st, "tq_encode_b")
     return st
 
 

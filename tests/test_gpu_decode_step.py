@@ -3,10 +3,11 @@
 The decode step (Gemma-4-31B-shaped linear layers of "A Discrete Weight
 Language for Large Language Models", section 6.1) runs q/k/v 8192 x 5376,
 o 5376 x 8192, gate/up 21504 x 5376 and down 5376 x 21504 in Format B with the
-3^-(k-1) ladder, at batch 1, 4, 16 and 64. One layer of each shape, with the
-codes the bench draws for it, is checked on 64 seeded rows (the last row
-included) against the fp64 oracle, in the launch configuration the bench
-times."""
+3^-(k-1) ladder, at batch 1, 4, 16 and 64. One layer of each shape, with
+uniform seeded codes drawn here on the host (the bench draws its codes on the
+device, from the same distribution), is checked on 64 seeded rows (the last
+row included) against the fp64 oracle, through the same dispatch and launch
+configuration the bench times at that shape and batch."""
 import numpy as np
 import pytest
 import torch
