@@ -11,13 +11,17 @@
 // y^T: tile t, t + CTAs, ... With a split, a cluster of `ks` CTAs takes one
 // tile, each CTA a slice of K. For each 128-wide k block ("iteration"):
 //   - the code producer warp copies the tile's codes into a shared-memory
-//     ring with 1-D bulk copies, one per row (Format B: the block's 128
-//     codes; Format A: windows of 4 blocks = 8 groups of 13 bytes plus their
-//     fp16 scales, as aligned 16-byte supersets of each row's run);
+//     ring with tensor copies (TMA): Format B one 128-row x 128-code box
+//     per block; Format A one box of codes and one of fp16 scales per window
+//     of 4 blocks = 8 groups of 13 bytes, from the 16-byte boundary at or
+//     below the window (when rows start on 16-byte boundaries; otherwise one
+//     1-D bulk copy of each row's aligned run). Code boxes use the 128-byte
+//     swizzle, so the decoders' row-wise reads spread over the banks. Few
+//     large copies matter: the copy engine spends tens of cycles on each;
 //   - the x producer copies the x tile (batch rounded up to 16 rows = N of
-//     the MMA, 128 k) with 2-D tensor copies in the canonical K-major layout
-//     (core matrices of 8 rows x 16 bytes); rows past the batch and k past K
-//     read as zero;
+//     the MMA, 128 k) with one 3-D tensor copy in the canonical K-major
+//     layout (core matrices of 8 rows x 16 bytes); rows past the batch and
+//     k past K read as zero;
 //   - 8 decoder warps (two per tensor-memory lane quarter; a thread owns one
 //     row and 64 k) turn the codes into bf16 operands and store them straight
 //     into tensor memory (tcgen05.st): A never passes through shared memory.
@@ -55,6 +59,7 @@
 
 #include <cooperative_groups.h>
 
+#include <cstring>
 #include <mutex>
 
 #include "tq_common.cuh"
@@ -94,10 +99,13 @@ constexpr int kWarpCodes = 0, kWarpX = 1, kWarpMma = 2, kWarpEpi = 3,
 constexpr int kThreads = 32 * (kWarpDec + kDecWarps);  // 480
 constexpr int kMaxCodeStages = 8;
 constexpr int kMaxXStages = 4;
-constexpr uint32_t kBRow = 144;          // Format B row slot: 128 codes + pad
+constexpr uint32_t kBRow = 128;          // Format B row: 128 codes, swizzled
 constexpr int kAWin = 4;                 // Format A window: 4 blocks, 8 groups
 constexpr uint32_t kARowCodes = 128;     // 104 code bytes + <= 15 skew
-constexpr uint32_t kARow = 160;          // + 16 scale bytes + <= 15 skew
+constexpr uint32_t kARow = 160;          // per-row copies: + 16 scale bytes
+                                         // + <= 15 skew
+constexpr uint32_t kAMapScales = kTileM * kARowCodes;  // tensor copies: the
+constexpr uint32_t kAMapSRow = 32;       // scale rows (16 fp16) follow the codes
 constexpr int kSmemMax = 227 * 1024;
 
 // Barrier block (byte offsets).
@@ -117,6 +125,8 @@ struct TcPlan {
   int x_stages;
   uint32_t red;  // partial tile [128][n_pad] fp32 (split of K only)
   uint32_t bars;
+  int a_map;    // Format A windows by tensor copies (else one copy per row)
+  int x_boxes;  // tensor copies per x stage: 1 (3-D map) or 16 (2-D map)
   uint64_t wait_ns;
   int skip_first_arrive;
   size_t smem;
@@ -311,6 +321,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const WeightsView w, int64_t batch, float *__restrict__ y,
                    int64_t ldy, const TcPlan P,
                    const __grid_constant__ CUtensorMap tmap_x,
+                   const __grid_constant__ CUtensorMap tmap_c,
+                   const __grid_constant__ CUtensorMap tmap_s,
                    unsigned long long *trace) {
   constexpr int kWin = FMT == TQ_FMT_A ? kAWin : 1;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -413,6 +425,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (warp == kWarpX && lane == 0)
     asm volatile("prefetch.tensormap [%0];" ::"l"(&tmap_x) : "memory");
+  if (warp == kWarpCodes && lane == 0 && (FMT == TQ_FMT_B || P.a_map)) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&tmap_c) : "memory");
+    if (FMT == TQ_FMT_A)
+      asm volatile("prefetch.tensormap [%0];" ::"l"(&tmap_s) : "memory");
+  }
   // the lane-replicated table
   if constexpr (FMT == TQ_FMT_B) {
     for (int i = threadIdx.x; i < 256 * 8; i += blockDim.x) {
@@ -440,7 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                : "memory");
 
   if (warp == kWarpCodes) {
-    // ---- code producer: bulk copies of each window's rows -------------------
+    // ---- code producer: each window's codes (and scales) ---------------------
     int s = 0, u = 0;  // ring slot, windows issued so far
     bool ok = true;
     for (int t = cid; ok && t < P.tiles; t += nclusters) {
@@ -459,22 +476,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t dst0 = code_stage(s);
         if (lane == 0) ck_trace<CK>(trace, 0, t, ws, 1);
         if constexpr (FMT == TQ_FMT_B) {
-          const int64_t k0 = (int64_t)ws * kKB;
-          const uint32_t sz = (uint32_t)(K - k0 < kKB ? K - k0 : kKB);
-          if (lane == 0) mbar_arrive_expect_tx(full, sz * (uint32_t)rows);
-          __syncwarp();
-          for (int r = lane; r < rows; r += 32) {
-            uint32_t d = dst0 + (uint32_t)r * kBRow;
-            const uint8_t *src = w.codes + (row0 + r) * K + k0;
-            if constexpr (CK) {
-              d = ck_smem<CK>(W, d, sz, 2);
-              if (row0 + r >= N || k0 + sz > K) {
-                ck_record(3, (uint64_t)((row0 + r) * K + k0));
-                src = w.codes;
-              }
-            }
-            bulk_g2s(d, src, sz, full);
+          // one box of 128 rows x 128 codes, 128-byte swizzle (16-byte chunk
+          // c of row r lands at chunk c ^ (r & 7)); rows past N and codes
+          // past K read as zero, and the decoders mask them
+          if (lane == 0) {
+            uint32_t d = dst0;
+            if constexpr (CK) d = ck_smem<CK>(W, d, kTileM * kBRow, 2);
+            mbar_arrive_expect_tx(full, kTileM * kBRow);
+            tma_load_2d(d, &tmap_c, ws * kKB, (int)row0, full);
           }
+          __syncwarp();
+        } else if (P.a_map) {
+          // the window's 8 groups of every row: codes from the 16-byte
+          // boundary at or below the first byte (128 bytes, 128-byte
+          // swizzle), scales from the 8-scale boundary (16 fp16)
+          const int plane = ws / P.kblocks;
+          const int g0 = 2 * (ws - plane * P.kblocks);
+          if (lane == 0) {
+            uint32_t d = dst0;
+            if constexpr (CK) d = ck_smem<CK>(W, d, P.code_stage_bytes, 4);
+            mbar_arrive_expect_tx(full, kTileM * (kARowCodes + kAMapSRow));
+            tma_load_3d(d, &tmap_c, (13 * g0) & ~15, (int)row0, plane, full);
+            tma_load_3d(d + kAMapScales, &tmap_s, g0 & ~7, (int)row0, plane,
+                        full);
+          }
+          __syncwarp();
         } else {
           const int plane = ws / P.kblocks;
           const int64_t g0 = 2 * (int64_t)(ws - plane * P.kblocks);
@@ -528,7 +554,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                   (uint32_t)(j / P.code_stages) & 1u);
     }
   } else if (warp == kWarpX) {
-    // ---- x producer: 16 tensor copies of 8 k x n_pad rows per iteration -----
+    // ---- x producer: the 128 k x n_pad tile of each iteration ---------------
+    // (one 3-D copy: 16 core-matrix columns of 8 k x n_pad rows; or 16 2-D
+    // copies of one column each)
     if (lane == 0) {
       int s = 0, u = 0;
       bool ok = true;
@@ -548,14 +576,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int k0 = (it % P.kblocks) * kKB;
           ck_trace<CK>(trace, 1, t, it, 1);
           mbar_arrive_expect_tx(full, 16u * box);
+          if (P.x_boxes == 1) {
+            uint32_t d = dst;
+            if constexpr (CK) d = ck_smem<CK>(W, d, 16u * box, 6);
+            tma_load_3d(d, &tmap_x, 0, 0, k0 / 8, full);
+          } else {
 #pragma unroll 1
-          for (int c = 0; c < 16; ++c) {
-            uint32_t d = dst + (uint32_t)c * box;
-            if constexpr (CK) {
-              d = ck_smem<CK>(W, d, box, 6);
-              if ((d & 127u) != 0u) ck_record(7, d);
+            for (int c = 0; c < 16; ++c) {
+              uint32_t d = dst + (uint32_t)c * box;
+              if constexpr (CK) {
+                d = ck_smem<CK>(W, d, box, 6);
+                if ((d & 127u) != 0u) ck_record(7, d);
+              }
+              tma_load_2d(d, &tmap_x, k0 + 8 * c, 0, full);
             }
-            tma_load_2d(d, &tmap_x, k0 + 8 * c, 0, full);
           }
           ++u;
           s = s + 1 == P.x_stages ? 0 : s + 1;
@@ -735,23 +769,37 @@ __global__ void __launch_bounds__(kThreads, 1)
                                   abort_addr, lim));
         if constexpr (CK) if (!ok && lane == 0) ck_record(28, (uint64_t)uc);
         if (!ok) break;
-        const uint32_t slot =
-            code_stage(cs) + (uint32_t)r * (FMT == TQ_FMT_B ? kBRow : kARow);
-        // Format A: this row's byte skews inside its code and scale slots
+        // this row's codes (crow) and scales (srow) in the stage; a row
+        // written by a tensor copy is swizzled: logical byte o is at o ^ sw
+        const bool swz = FMT == TQ_FMT_B || P.a_map;
+        const uint32_t sw = swz ? (uint32_t)(r & 7) << 4 : 0u;
+        const uint32_t crow =
+            code_stage(cs) + (uint32_t)r * (FMT == TQ_FMT_B ? kBRow
+                                            : swz ? kARowCodes : kARow);
+        const uint32_t srow = swz ? code_stage(cs) + kAMapScales +
+                                        (uint32_t)r * kAMapSRow
+                                  : crow + kARowCodes;
+        // Format A: byte skews of the window's first group inside the code and
+        // scale rows (the same for every row with tensor copies)
         uint32_t cskew = 0, sskew = 0;
         int64_t g0 = 0;
         if constexpr (FMT == TQ_FMT_A) {
           const int plane = ws / P.kblocks;
           g0 = 2 * (int64_t)(ws - plane * P.kblocks);
-          const int64_t gi = (row_ok ? row : 0) * gpr + g0;
-          cskew = (uint32_t)((reinterpret_cast<uintptr_t>(w.codes) +
-                              (uintptr_t)(plane * w.codes_plane_stride) +
-                              (uintptr_t)(gi * 13)) &
-                             15);
-          sskew = (uint32_t)((reinterpret_cast<uintptr_t>(w.scales) +
-                              (uintptr_t)(2 * (plane * w.scales_plane_stride +
-                                               gi))) &
-                             15);
+          if (swz) {
+            cskew = (uint32_t)(13 * g0) & 15u;
+            sskew = 2u * ((uint32_t)g0 & 7u);
+          } else {
+            const int64_t gi = (row_ok ? row : 0) * gpr + g0;
+            cskew = (uint32_t)((reinterpret_cast<uintptr_t>(w.codes) +
+                                (uintptr_t)(plane * w.codes_plane_stride) +
+                                (uintptr_t)(gi * 13)) &
+                               15);
+            sskew = (uint32_t)((reinterpret_cast<uintptr_t>(w.scales) +
+                                (uintptr_t)(2 * (plane * w.scales_plane_stride +
+                                                 gi))) &
+                               15);
+          }
         }
         for (int it = ws; it < we; ++it) {
           if (ua >= kAStages) {
@@ -766,11 +814,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0 && q == 0 && kp == 0) ck_trace<CK>(trace, 5, t, it, 1);
           uint32_t hi[32], lo[32];
           if constexpr (FMT == TQ_FMT_B) {
-            const uint32_t src = slot + 64u * (uint32_t)kp;
             uint32_t cw[16];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              const uint4 v4 = lds128(ck_smem<CK>(W, src + 16u * (uint32_t)j, 16u, 16));
+              const uint32_t a =
+                  crow + ((64u * (uint32_t)kp + 16u * (uint32_t)j) ^ sw);
+              const uint4 v4 = lds128(ck_smem<CK>(W, a, 16u, 16));
               cw[4 * j] = v4.x;
               cw[4 * j + 1] = v4.y;
               cw[4 * j + 2] = v4.z;
@@ -792,16 +841,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int gi = 2 * (it - ws) + kp;  // group inside the window
             const bool valid = row_ok && g0 + gi < gpr;
             const uint32_t o = cskew + 13u * (uint32_t)gi;
-            const uint32_t wa = slot + (o & ~3u);
+            const uint32_t wl = o & ~3u;  // logical offsets wl .. wl + 15
             const uint32_t sh = 8u * (o & 3u);
-            const uint32_t w0 = lds32(ck_smem<CK>(W, wa, 4u, 17)),
-                           w1 = lds32(ck_smem<CK>(W, wa + 4, 4u, 17)),
-                           w2 = lds32(ck_smem<CK>(W, wa + 8, 4u, 17)),
-                           w3 = lds32(ck_smem<CK>(W, wa + 12, 4u, 17));
+            const uint32_t w0 = lds32(ck_smem<CK>(W, crow + (wl ^ sw), 4u, 17)),
+                           w1 = lds32(ck_smem<CK>(W, crow + ((wl + 4) ^ sw), 4u, 17)),
+                           w2 = lds32(ck_smem<CK>(W, crow + ((wl + 8) ^ sw), 4u, 17)),
+                           w3 = lds32(ck_smem<CK>(W, crow + ((wl + 12) ^ sw), 4u, 17));
             const uint32_t b[4] = {__funnelshift_r(w0, w1, sh),
                                    __funnelshift_r(w1, w2, sh),
                                    __funnelshift_r(w2, w3, sh), w3 >> sh};
-            const uint32_t sa = slot + kARowCodes + sskew + 2u * (uint32_t)gi;
+            const uint32_t sa = srow + sskew + 2u * (uint32_t)gi;
             const uint32_t sbits =
                 (lds32(ck_smem<CK>(W, sa & ~3u, 4u, 18)) >> (8u * (sa & 2u))) & 0xFFFFu;
             const float sf = __half2float(__ushort_as_half((unsigned short)sbits));
@@ -915,8 +964,9 @@ bool plan_smem(int fmt, int n_pad, int ks, uint32_t base, TcPlan *P) {
   P->x_stages = n_pad <= 32 ? kMaxXStages : 3;
   // with a split of K, every CTA keeps its partial tile [128][n_pad] fp32
   const uint32_t red_bytes = ks > 1 ? (uint32_t)(kTileM * n_pad * 4) : 0u;
-  // below the table: code stages
-  const uint32_t lo0 = (base + 127u) & ~127u;
+  // below the table: code stages (1024-byte aligned: the 128-byte swizzle
+  // of tensor copies repeats every 8 rows of 128 bytes)
+  const uint32_t lo0 = (base + 1023u) & ~1023u;
   P->code_lo = lo0;
   P->code_lo_n = (int)((tab - lo0) / P->code_stage_bytes);
   // above it: barriers, x ring, reduction buffer, further code stages
@@ -928,7 +978,7 @@ bool plan_smem(int fmt, int n_pad, int ks, uint32_t base, TcPlan *P) {
   a += (uint32_t)P->x_stages * P->x_stage_bytes;
   P->red = a;
   a += red_bytes;
-  a = (a + 127u) & ~127u;
+  a = (a + 1023u) & ~1023u;
   P->code_hi = a;
   if (a > end) return false;
   int hi_n = (int)((end - a) / P->code_stage_bytes);
@@ -1025,21 +1075,85 @@ cudaError_t launch_tc_as(const WeightsView &w, const __nv_bfloat16 *x,
   best.wait_ns = tw ? tw : kWaitLimitNs;
   best.skip_first_arrive = g_test_skip_first_arrive.load();
 
-  // x as a 2-D tensor: K bf16 per row, `batch` rows ldx apart, boxes of
-  // 8 k x n_pad rows (rows past the batch and k past K read as zero).
   auto encode = encode_fn();
   if (encode == nullptr) return cudaErrorNotSupported;
-  CUtensorMap tmap;
-  cuuint64_t dims[2] = {(cuuint64_t)w.k, (cuuint64_t)batch};
-  cuuint64_t strides[1] = {(cuuint64_t)ldx * 2};
-  cuuint32_t box[2] = {8u, (cuuint32_t)n_pad};
-  cuuint32_t estr[2] = {1u, 1u};
-  if (encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
-             const_cast<__nv_bfloat16 *>(x), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return cudaErrorInvalidValue;
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  // x: K bf16 per row, `batch` rows ldx apart. As a 3-D tensor {8 k, row,
+  // k / 8} one box {8, n_pad, 16} is the whole 128 k x n_pad tile in the
+  // canonical K-major layout (16 columns of n_pad rows x 16 bytes); if the
+  // driver declines that view, 2-D boxes {8, n_pad} of one column each.
+  // Rows past the batch and k past K read as zero.
+  CUtensorMap tmap_x;
+  {
+    const cuuint64_t dims[3] = {8u, (cuuint64_t)batch, (cuuint64_t)(w.k / 8)};
+    const cuuint64_t strides[2] = {(cuuint64_t)ldx * 2, 16u};
+    const cuuint32_t box[3] = {8u, (cuuint32_t)n_pad, 16u};
+    best.x_boxes = 1;
+    if (encode(&tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+               const_cast<__nv_bfloat16 *>(x), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS) {
+      const cuuint64_t dims2[2] = {(cuuint64_t)w.k, (cuuint64_t)batch};
+      const cuuint64_t strides2[1] = {(cuuint64_t)ldx * 2};
+      const cuuint32_t box2[2] = {8u, (cuuint32_t)n_pad};
+      best.x_boxes = 16;
+      if (encode(&tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                 const_cast<__nv_bfloat16 *>(x), dims2, strides2, box2, estr,
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                 CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    }
+  }
+  // codes (and Format A scales)
+  CUtensorMap tmap_c, tmap_s;
+  memset(&tmap_c, 0, sizeof(tmap_c));
+  memset(&tmap_s, 0, sizeof(tmap_s));
+  best.a_map = 0;
+  if (FMT == TQ_FMT_B) {
+    // [N][K] bytes; boxes of 128 rows x 128 codes, 128-byte swizzle
+    const cuuint64_t dims[2] = {(cuuint64_t)w.k, (cuuint64_t)w.n};
+    const cuuint64_t strides[1] = {(cuuint64_t)w.k};
+    const cuuint32_t box[2] = {kBRow, (cuuint32_t)kTileM};
+    if (encode(&tmap_c, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+               const_cast<uint8_t *>(w.codes), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  } else {
+    // [plane][N][13 K/64] bytes and [plane][N][K/64] fp16 as 3-D tensors,
+    // when every row and plane starts on a 16-byte boundary (K a multiple
+    // of 1024); otherwise the producer copies each row's run by itself
+    const int64_t gpr = w.k / 64;
+    const int64_t cpitch = 13 * gpr, spitch = 2 * gpr;
+    const int64_t cps = w.codes_plane_stride, sps = 2 * w.scales_plane_stride;
+    if (cpitch % 16 == 0 && spitch % 16 == 0 &&
+        (w.planes == 1 || (cps % 16 == 0 && sps % 16 == 0))) {
+      const cuuint64_t cd[3] = {(cuuint64_t)cpitch, (cuuint64_t)w.n,
+                                (cuuint64_t)w.planes};
+      const cuuint64_t cs[2] = {(cuuint64_t)cpitch,
+                                (cuuint64_t)(w.planes > 1 ? cps : cpitch * w.n)};
+      const cuuint32_t cb[3] = {kARowCodes, (cuuint32_t)kTileM, 1u};
+      const cuuint64_t sd[3] = {(cuuint64_t)gpr, (cuuint64_t)w.n,
+                                (cuuint64_t)w.planes};
+      const cuuint64_t ss[2] = {(cuuint64_t)spitch,
+                                (cuuint64_t)(w.planes > 1 ? sps : spitch * w.n)};
+      const cuuint32_t sb[3] = {kAMapSRow / 2, (cuuint32_t)kTileM, 1u};
+      if (encode(&tmap_c, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3,
+                 const_cast<uint8_t *>(w.codes), cd, cs, cb, estr,
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS &&
+          encode(&tmap_s, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3,
+                 const_cast<uint16_t *>(w.scales), sd, ss, sb, estr,
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                 CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS)
+        best.a_map = 1;
+    }
+  }
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(best_clusters * best.ks), 1, 1);
@@ -1055,7 +1169,8 @@ cudaError_t launch_tc_as(const WeightsView &w, const __nv_bfloat16 *x,
   cfg.numAttrs = 1;
   unsigned long long *trace =
       CK ? reinterpret_cast<unsigned long long *>(g_test_trace.load()) : nullptr;
-  return cudaLaunchKernelEx(&cfg, kern, w, batch, y, ldy, best, tmap, trace);
+  return cudaLaunchKernelEx(&cfg, kern, w, batch, y, ldy, best, tmap_x, tmap_c,
+                            tmap_s, trace);
 }
 
 template <int FMT>
@@ -1077,7 +1192,9 @@ cudaError_t tc_check_record(uint64_t out[4], bool reset) {
 }
 
 bool gemm_tc_supported(const WeightsView &w, int64_t batch) {
-  if (batch < 1 || w.k < 1) return false;
+  // tensor-copy coordinates are 32-bit
+  if (batch < 1 || w.k < 1 || w.n >= (1ll << 31) || w.k >= (1ll << 31))
+    return false;
   if (w.format == TQ_FMT_B) return true;
   return w.format == TQ_FMT_A && w.group == 64;
 }

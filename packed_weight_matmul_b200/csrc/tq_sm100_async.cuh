@@ -125,6 +125,19 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap,
       : "memory");
 }
 
+// 3-D tensor copy of one box (coordinates c0 innermost, c1, c2) into this
+// CTA's shared memory, completing on `bar`; out-of-range elements read as
+// zero.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *tmap,
+                                            int32_t c0, int32_t c1, int32_t c2,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::"
+      "bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(tmap), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
+      : "memory");
+}
+
 // ---- thread-block clusters -------------------------------------------------
 
 __device__ __forceinline__ uint32_t cluster_rank() {
