@@ -35,7 +35,10 @@ tq_status tq_testing_linear_wait_fault(int32_t withhold_first_arrive,
  *   0  automatic (the default dispatch by format and batch);
  *   1  the CUDA-core kernels (GEMV where it takes the batch, else the
  *      one-warp-per-row kernel);
- *   2  the tensor-core kernel.
+ *   2  the tensor-core kernel;
+ *   3  the tensor-core kernel with every Format B code-book entry split
+ *      into a bf16 hi + lo operand pair, even where the code book allows
+ *      the single-operand path (integer multiples of one unit).
  * A family that cannot take the call falls back to the automatic choice.
  * Returns TQ_ERR_INVALID_ARG for other values. */
 tq_status tq_testing_force_linear_path(int32_t path);

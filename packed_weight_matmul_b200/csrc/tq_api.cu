@@ -189,7 +189,7 @@ tq_status tq_testing_linear_wait_fault(int32_t withhold_first_arrive,
 }
 
 tq_status tq_testing_force_linear_path(int32_t path) {
-  if (path < 0 || path > 2) return TQ_ERR_INVALID_ARG;
+  if (path < 0 || path > 3) return TQ_ERR_INVALID_ARG;
   tq::g_test_force_path.store(path);
   return TQ_OK;
 }

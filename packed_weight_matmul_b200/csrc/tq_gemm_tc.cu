@@ -112,7 +112,8 @@ constexpr int kSmemMax = 227 * 1024;
 constexpr uint32_t kBarCodeFull = 0, kBarCodeEmpty = 64, kBarXFull = 128,
                    kBarXEmpty = 160, kBarAFull = 192, kBarAEmpty = 216,
                    kBarAccFull = 240, kBarAccEmpty = 256, kBarDrain = 296,
-                   kTmemSlot = 304, kAbort = 308, kBarBytes = 320;
+                   kTmemSlot = 304, kAbort = 308, kUnit = 312,
+                   kBarBytes = 320;
 
 struct TcPlan {
   int n_pad, ks, tiles, kblocks, iters;
@@ -123,12 +124,13 @@ struct TcPlan {
   uint32_t code_stage_bytes;
   uint32_t x_ring, x_stage_bytes;
   int x_stages;
-  uint32_t red;  // partial tile [128][n_pad] fp32 (split of K only)
+  uint32_t red;  // partial tile [n_pad][128] fp32 (split of K only)
   uint32_t bars;
   int a_map;    // Format A windows by tensor copies (else one copy per row)
   int x_boxes;  // tensor copies per x stage: 1 (3-D map) or 16 (2-D map)
   uint64_t wait_ns;
   int skip_first_arrive;
+  int grid_ok;  // Format B: the single-operand code-book path may be used
   size_t smem;
 };
 
@@ -217,6 +219,21 @@ __device__ __forceinline__ void decode_b(const uint32_t (&cw)[16],
     lo[2 * j] = prmt(v0, v1, 0x7632u);
     hi[2 * j + 1] = prmt(v2, v3, 0x5410u);
     lo[2 * j + 1] = prmt(v2, v3, 0x7632u);
+  }
+}
+
+// Format B, single operand: 64 codes of one row -> 32 bf16 pairs.
+__device__ __forceinline__ void decode_b_hi(const uint32_t (&cw)[16],
+                                            uint32_t lane_tab,
+                                            uint32_t (&hi)[32]) {
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const uint32_t v0 = lut32(prmt(cw[j], lane_tab, 0x7604u));
+    const uint32_t v1 = lut32(prmt(cw[j], lane_tab, 0x7614u));
+    const uint32_t v2 = lut32(prmt(cw[j], lane_tab, 0x7624u));
+    const uint32_t v3 = lut32(prmt(cw[j], lane_tab, 0x7634u));
+    hi[2 * j] = prmt(v0, v1, 0x5410u);
+    hi[2 * j + 1] = prmt(v2, v3, 0x5410u);
   }
 }
 
@@ -417,6 +434,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(B0 + kBarAccEmpty + 8 * b, 4);
     }
     mbar_init(B0 + kBarDrain, 1);
+    st_volatile_s32(B0 + kUnit, 0x7F800000);  // +inf
     mbar_init_fence();
   }
   if (warp == kWarpMma) {
@@ -430,14 +448,51 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (FMT == TQ_FMT_A)
       asm volatile("prefetch.tensormap [%0];" ::"l"(&tmap_s) : "memory");
   }
+  // Format B: when every code-book entry is an integer multiple m of one
+  // unit u (|m| <= 256, to 2^-20 of the entry; e.g. the balanced-ternary
+  // ladder 3^-(i-1), whose 243 words are the integers -121..121 in units of
+  // alpha / 81), the operand is bf16(m), exact: one MMA per k step, and u
+  // multiplies the accumulator in the epilogue. The representation error,
+  // 2^-20, is below that of the hi + lo split (2^-17). Otherwise each entry
+  // becomes bf16 hi + lo (two MMAs). u is the smallest non-zero |entry|; the
+  // test runs in every CTA on the same table, so all CTAs agree.
+  bool grid = false;
+  float unit = 1.0f;
+  if constexpr (FMT == TQ_FMT_B) {
+    __syncthreads();  // the unit word is initialised
+    float lv = 0.0f;
+    if (threadIdx.x < 243) {
+      lv = __ldg(w.lut + threadIdx.x);
+      const float a = fabsf(lv);
+      if (a > 0.0f && a <= 3.4028235e38f)
+        atom_min_shared_u32(B0 + kUnit, __float_as_uint(a));
+    }
+    __syncthreads();
+    const float u = __int_as_float(ld_volatile_s32(B0 + kUnit));
+    bool ok = true;
+    if (threadIdx.x < 243) {
+      const float m = rintf(__fdiv_rn(lv, u));
+      ok = u <= 3.4028235e38f && fabsf(m) <= 256.0f &&
+           fabs((double)lv - (double)u * (double)m) <=
+               ldexp(fabs((double)lv), -20);
+    }
+    grid = __syncthreads_and(ok) != 0 && P.grid_ok != 0;
+    if (grid) unit = u;
+  }
   // the lane-replicated table
   if constexpr (FMT == TQ_FMT_B) {
     for (int i = threadIdx.x; i < 256 * 8; i += blockDim.x) {
       const int e = i >> 3, j = i & 7;
       const float v = __ldg(w.lut + e);
-      const uint32_t h = bf16_bits_rn(v);
-      const uint32_t l = bf16_bits_rn(v - __uint_as_float(h << 16));
-      const uint32_t word = h | l << 16;
+      uint32_t word;
+      if (grid) {
+        // bf16(m) in the low half; entries 243..255 stay NaN
+        word = e < 243 ? bf16_bits_rn(rintf(__fdiv_rn(v, unit))) : 0x7FC0u;
+      } else {
+        const uint32_t h = bf16_bits_rn(v);
+        const uint32_t l = bf16_bits_rn(v - __uint_as_float(h << 16));
+        word = h | l << 16;
+      }
       sts128(tab + (uint32_t)e * 256u + (uint32_t)j * 16u, word, word, word,
              word);
     }
@@ -644,7 +699,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 smem_desc_kmajor(xb + (uint32_t)(2 * k16) * lbo, lbo, 128u);
             mma_bf16_ts(d, a + 8u * (uint32_t)k16, bd, idesc,
                         (it > it0 || k16 > 0) ? 1u : 0u);
-            mma_bf16_ts(d, a + 64u + 8u * (uint32_t)k16, bd, idesc, 1u);
+            if (!grid)
+              mma_bf16_ts(d, a + 64u + 8u * (uint32_t)k16, bd, idesc, 1u);
           }
           mma_commit(B0 + kBarXEmpty + 8 * xs);
           mma_commit(B0 + kBarAEmpty + 8 * as);
@@ -733,17 +789,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                   continue;
                 }
               }
-              y[(int64_t)b * ldy + row] = scale * __uint_as_float(v[b]);
+              y[(int64_t)b * ldy + row] = scale * (unit * __uint_as_float(v[b]));
             }
         }
       } else {
         // a K slice (one tile per CTA): the partial row goes to this CTA's
         // shared buffer; the owners add the cluster's partials after the
         // cluster barrier at the end of the kernel
-        if constexpr (CK) ck_smem<CK>(W, P.red + delta + (uint32_t)(r * n_pad * 4), (uint32_t)n_pad * 4u, 14);
+        // (batch column c of the tile at part[c * 128 ..]: a warp's stores
+        // and the owners' reads are 32 consecutive words, conflict-free)
+        if constexpr (CK) ck_smem<CK>(W, P.red + delta, (uint32_t)(kTileM * n_pad * 4), 14);
 #pragma unroll
         for (int c = 0; c < 64; ++c)
-          if (c < n_pad) part[r * n_pad + c] = __uint_as_float(v[c]);
+          if (c < n_pad) part[c * kTileM + r] = __uint_as_float(v[c]);
       }
     }
   } else {
@@ -825,7 +883,10 @@ __global__ void __launch_bounds__(kThreads, 1)
               cw[4 * j + 2] = v4.z;
               cw[4 * j + 3] = v4.w;
             }
-            decode_b(cw, lane_tab, hi, lo);
+            if (grid)
+              decode_b_hi(cw, lane_tab, hi);
+            else
+              decode_b(cw, lane_tab, hi, lo);
             // k past K (in the last block) and rows past N: zero weights
             // (selects, no branch: the tcgen05.st below is warp-wide)
             const int64_t kv = K - ((int64_t)it * kKB + 64 * kp);
@@ -834,7 +895,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int m = 0; m < 32; ++m) {
                 const uint32_t keep = (row_ok && 2 * m < kv) ? 0xFFFFFFFFu : 0u;
                 hi[m] &= keep;
-                lo[m] &= keep;
+                if (!grid) lo[m] &= keep;
               }
             }
           } else {
@@ -870,7 +931,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if constexpr (CK) ta = ck_tmem<CK>(ta, 96u, (uint32_t)(32 * q), 19);
           __syncwarp();  // converged for the warp-wide stores
           tmem_st32(ta, hi);
-          tmem_st32(ta + 64u, lo);
+          if (!grid) tmem_st32(ta + 64u, lo);
           tmem_st_wait();
           if (lane == 0 && q == 0 && kp == 0) ck_trace<CK>(trace, 5, t, it, 2);
           tc_fence_before_sync();
@@ -910,7 +971,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int orr = idx % own, b = idx / own;
         float sum = 0.0f;
         for (int p = 0; p < ks; ++p)
-          sum += cluster.map_shared_rank(part, p)[(r_lo + orr) * n_pad + b];
+          sum += cluster.map_shared_rank(part, p)[b * kTileM + r_lo + orr];
         const int64_t row = row0 + r_lo + orr;
         if (row < N) {
           float scale = 1.0f;
@@ -918,7 +979,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (w.scales != nullptr)
               scale = __half2float(__ushort_as_half(w.scales[row / w.rps]));
           }
-          y[(int64_t)b * ldy + row] = scale * sum;
+          y[(int64_t)b * ldy + row] = scale * (unit * sum);
         }
       }
     }
@@ -962,7 +1023,7 @@ bool plan_smem(int fmt, int n_pad, int ks, uint32_t base, TcPlan *P) {
   P->code_stage_bytes = kTileM * (fmt == TQ_FMT_B ? kBRow : kARow);
   P->x_stage_bytes = (uint32_t)n_pad * kKB * 2u;
   P->x_stages = n_pad <= 32 ? kMaxXStages : 3;
-  // with a split of K, every CTA keeps its partial tile [128][n_pad] fp32
+  // with a split of K, every CTA keeps its partial tile [n_pad][128] fp32
   const uint32_t red_bytes = ks > 1 ? (uint32_t)(kTileM * n_pad * 4) : 0u;
   // below the table: code stages (1024-byte aligned: the 128-byte swizzle
   // of tensor copies repeats every 8 rows of 128 bytes)
@@ -1074,6 +1135,7 @@ cudaError_t launch_tc_as(const WeightsView &w, const __nv_bfloat16 *x,
   const uint64_t tw = g_test_wait_ns.load();
   best.wait_ns = tw ? tw : kWaitLimitNs;
   best.skip_first_arrive = g_test_skip_first_arrive.load();
+  best.grid_ok = g_test_force_path.load() == 3 ? 0 : 1;
 
   auto encode = encode_fn();
   if (encode == nullptr) return cudaErrorNotSupported;

@@ -9,7 +9,7 @@ cudaError_t launch_linear(const WeightsView &w, const __nv_bfloat16 *x,
                           int64_t batch, int64_t ldx, float *y, int64_t ldy,
                           cudaStream_t stream) {
   const int force = g_test_force_path.load();
-  if (force == 2 && gemm_tc_supported(w, batch))
+  if ((force == 2 || force == 3) && gemm_tc_supported(w, batch))
     return gemm_tc(w, x, batch, ldx, y, ldy, stream);
   if (force == 1) {
     if (gemv_b_supported(w, batch))

@@ -73,6 +73,11 @@ __device__ __forceinline__ void st_volatile_s32(uint32_t addr, int v) {
                : "memory");
 }
 
+__device__ __forceinline__ void atom_min_shared_u32(uint32_t addr, uint32_t v) {
+  asm volatile("atom.shared.min.u32 _, [%0], %1;" ::"r"(addr), "r"(v)
+               : "memory");
+}
+
 // Wait for the phase with the given parity to complete. Returns false when
 // the wait gave up: the word at `abort_addr` became non-zero, or `limit_ns`
 // passed (then the abort word is set, so that the CTA's other roles stop).

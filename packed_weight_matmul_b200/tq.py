@@ -134,7 +134,8 @@ def tq_testing_linear_wait_fault(withhold_first_arrive: bool,
 
 def tq_testing_force_linear_path(path: int) -> None:
     """Test hook (include/tq_testing.h): 0 automatic dispatch, 1 CUDA-core
-    kernels, 2 tensor-core kernel."""
+    kernels, 2 tensor-core kernel, 3 tensor-core kernel with the Format B
+    code book always split into bf16 hi + lo operands."""
     _check(_lib.tq_testing_force_linear_path(int(path)),
            "tq_testing_force_linear_path")
 

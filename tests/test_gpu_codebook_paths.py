@@ -1,0 +1,93 @@
+"""GPU parity of the two Format B operand paths of the tensor-core kernel.
+
+A code book whose entries are all integer multiples m of one unit u (|m| <=
+256, to 2^-20 of each entry) is decoded to the single exact operand bf16(m),
+with u applied to the accumulator; any other code book is split into a bf16
+hi + lo pair. These tests run both paths against the fp64 oracle (same
+tolerance as test_gpu_linear), force the hi + lo path on a code book that
+would take the single path (tq_testing_force_linear_path(3)), and check that
+an entry just off the grid is not forced onto it: with every code of a row
+equal and x all ones, an entry rounded onto the grid would miss by about
+1e-3 * K * |w|, far outside the tolerance."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import oref
+from packed_weight_matmul_b200 import inputs as I
+from tests import gpu_util as U
+
+pytestmark = pytest.mark.gpu
+
+BATCHES = (5, 16, 33, 64)
+# a ladder whose 243 sums are not on one grid (the encoder's test ladder)
+LADDER_FREE = np.array([1.0, 0.33, 0.115, 0.037, 0.012], np.float32)
+
+
+@pytest.fixture
+def force_path():
+    def set_path(p):
+        U.tq().tq_testing_force_linear_path(p)
+    yield set_path
+    U.tq().tq_testing_force_linear_path(0)
+
+
+def _run(codes, lut, rho=None, rps=0, batches=BATCHES, seed=0, label=""):
+    rho_bits = I.bits(rho) if rho is not None else None
+    w = U.weights_b_dev(codes, lut, rho, rps)
+    absmax = U.absmax_rows_b(codes.numpy(), lut, rho_bits, rps)
+    for batch in batches:
+        x = I.x_normal(batch, codes.shape[1], seed + batch)
+        xb = U.x_bits(x)
+        y, _ = U.linear(w, x)
+        ref = oref.linear_B(codes.numpy(), lut, xb, rho_bits, rps)
+        U.check_tolerance(y, ref, xb, absmax, f"{label} b={batch}")
+
+
+@pytest.mark.parametrize("n,k,rps", [(130, 5376, 1), (300, 2064, 0),
+                                     (257, 4096, 128)])
+def test_off_grid_ladder_uses_hi_lo(n, k, rps):
+    lut = oref.build_lut(I.ALPHA, LADDER_FREE)
+    codes = I.codes_uniform(n, k, n + k)
+    rho = I.rho_uniform(I.rho_count(n, rps), 3) if rps else None
+    _run(codes, lut, rho, rps, label=f"free ladder {n}x{k}")
+
+
+@pytest.mark.parametrize("path", [2, 3])
+def test_grid_ladder_both_paths(force_path, path):
+    lut = oref.build_lut(I.ALPHA, I.ladder_pow3().numpy())
+    codes = I.codes_uniform(300, 4224, 77)
+    force_path(path)
+    _run(codes, lut, label=f"pow3 path {path}")
+
+
+@pytest.mark.parametrize("path", [0, 3])
+def test_entry_off_grid_is_not_rounded_onto_it(force_path, path):
+    lut = oref.build_lut(I.ALPHA, I.ladder_pow3().numpy()).copy()
+    lut[200] = np.float32(lut[200] * np.float32(1.001))
+    n, k = 256, 4096
+    codes = I.codes_uniform(n, k, 5)
+    codes[7, :] = 200  # one row of a single code
+    force_path(path)
+    w = U.weights_b_dev(codes, lut)
+    absmax = U.absmax_rows_b(codes.numpy(), lut)
+    for batch in (8, 64):
+        x = torch.ones(batch, k, dtype=torch.bfloat16)
+        xb = U.x_bits(x)
+        y, _ = U.linear(w, x)
+        ref = oref.linear_B(codes.numpy(), lut, xb)
+        U.check_tolerance(y, ref, xb, absmax, f"off-grid entry b={batch}")
+
+
+def test_integer_ladder_and_zero_book():
+    # ladder 81, 27, 9, 3, 1: the entries are the integers -121..121 * alpha
+    lut = oref.build_lut(np.float32(0.75),
+                         np.array([81, 27, 9, 3, 1], np.float32))
+    codes = I.codes_uniform(200, 1040, 9)
+    _run(codes, lut, batches=(6, 64), label="integer ladder")
+    # alpha = 0: every entry is zero, and so is every output
+    zero = oref.build_lut(np.float32(0.0), I.ladder_pow3().numpy())
+    w = U.weights_b_dev(codes, zero)
+    for batch in (6, 64):
+        y, _ = U.linear(w, I.x_normal(batch, 1040, batch))
+        assert np.all(y == 0.0)
