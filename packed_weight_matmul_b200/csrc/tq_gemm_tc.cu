@@ -19,9 +19,10 @@
 //     swizzle, so the decoders' row-wise reads spread over the banks. Few
 //     large copies matter: the copy engine spends tens of cycles on each;
 //   - the x producer copies the x tile (batch rounded up to 16 rows = N of
-//     the MMA, 128 k) with one 3-D tensor copy in the canonical K-major
-//     layout (core matrices of 8 rows x 16 bytes); rows past the batch and
-//     k past K read as zero;
+//     the MMA, 128 k) with two tensor copies of 64 k, 128-byte rows in the
+//     K-major 128-byte-swizzle layout; rows past the batch and k past K read
+//     as zero (boxes of 16-byte rows cost the copy engine about 20 cycles a
+//     row, which made x the slowest input);
 //   - 8 decoder warps (two per tensor-memory lane quarter; a thread owns one
 //     row and 64 k) turn the codes into bf16 operands and store them straight
 //     into tensor memory (tcgen05.st): A never passes through shared memory.
@@ -127,7 +128,6 @@ struct TcPlan {
   uint32_t red;  // partial tile [n_pad][128] fp32 (split of K only)
   uint32_t bars;
   int a_map;    // Format A windows by tensor copies (else one copy per row)
-  int x_boxes;  // tensor copies per x stage: 1 (3-D map) or 16 (2-D map)
   uint64_t wait_ns;
   int skip_first_arrive;
   int grid_ok;  // Format B: the single-operand code-book path may be used
@@ -610,12 +610,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kWarpX) {
     // ---- x producer: the 128 k x n_pad tile of each iteration ---------------
-    // (one 3-D copy: 16 core-matrix columns of 8 k x n_pad rows; or 16 2-D
-    // copies of one column each)
+    // (two copies of 64 k x n_pad rows, 128-byte rows with the 128-byte
+    // swizzle: the K-major layout the MMA reads)
     if (lane == 0) {
       int s = 0, u = 0;
       bool ok = true;
-      const uint32_t box = (uint32_t)n_pad * 16u;
+      const uint32_t half = (uint32_t)n_pad * 128u;
       for (int t = cid; ok && t < P.tiles; t += nclusters) {
         for (int it = it0; it < it1; ++it) {
           if (u >= P.x_stages &&
@@ -630,21 +630,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t dst = x_ring + (uint32_t)s * P.x_stage_bytes;
           const int k0 = (it % P.kblocks) * kKB;
           ck_trace<CK>(trace, 1, t, it, 1);
-          mbar_arrive_expect_tx(full, 16u * box);
-          if (P.x_boxes == 1) {
-            uint32_t d = dst;
-            if constexpr (CK) d = ck_smem<CK>(W, d, 16u * box, 6);
-            tma_load_3d(d, &tmap_x, 0, 0, k0 / 8, full);
-          } else {
-#pragma unroll 1
-            for (int c = 0; c < 16; ++c) {
-              uint32_t d = dst + (uint32_t)c * box;
-              if constexpr (CK) {
-                d = ck_smem<CK>(W, d, box, 6);
-                if ((d & 127u) != 0u) ck_record(7, d);
-              }
-              tma_load_2d(d, &tmap_x, k0 + 8 * c, 0, full);
+          mbar_arrive_expect_tx(full, 2u * half);
+          for (int h = 0; h < 2; ++h) {
+            uint32_t d = dst + (uint32_t)h * half;
+            if constexpr (CK) {
+              d = ck_smem<CK>(W, d, half, 6);
+              if ((d & 1023u) != 0u) ck_record(7, d);
             }
+            tma_load_2d(d, &tmap_x, k0 + 64 * h, 0, full);
           }
           ++u;
           s = s + 1 == P.x_stages ? 0 : s + 1;
@@ -658,7 +651,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- MMA issuer ---------------------------------------------------------
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(kTileM, n_pad);
-      const uint32_t lbo = (uint32_t)n_pad * 16u;  // next 8 k of the x tile
+      const uint32_t xhalf = (uint32_t)n_pad * 128u;  // k 64..127 of the tile
       int xs = 0, ux = 0, as = 0, ua = 0;
       int ca = 0;  // accumulator commits
       bool ok = true;
@@ -695,8 +688,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
 #pragma unroll
           for (int k16 = 0; k16 < 8; ++k16) {
-            const uint64_t bd =
-                smem_desc_kmajor(xb + (uint32_t)(2 * k16) * lbo, lbo, 128u);
+            const uint64_t bd = smem_desc_kmajor_sw128(
+                xb + (uint32_t)(k16 >> 2) * xhalf + 32u * (uint32_t)(k16 & 3));
             mma_bf16_ts(d, a + 8u * (uint32_t)k16, bd, idesc,
                         (it > it0 || k16 > 0) ? 1u : 0u);
             if (!grid)
@@ -1034,7 +1027,7 @@ bool plan_smem(int fmt, int n_pad, int ks, uint32_t base, TcPlan *P) {
   uint32_t a = tab + 0x10000u;
   P->bars = a;
   a += kBarBytes;
-  a = (a + 127u) & ~127u;
+  a = (a + 1023u) & ~1023u;  // 128-byte swizzle atoms
   P->x_ring = a;
   a += (uint32_t)P->x_stages * P->x_stage_bytes;
   P->red = a;
@@ -1140,33 +1133,20 @@ cudaError_t launch_tc_as(const WeightsView &w, const __nv_bfloat16 *x,
   auto encode = encode_fn();
   if (encode == nullptr) return cudaErrorNotSupported;
   const cuuint32_t estr[3] = {1u, 1u, 1u};
-  // x: K bf16 per row, `batch` rows ldx apart. As a 3-D tensor {8 k, row,
-  // k / 8} one box {8, n_pad, 16} is the whole 128 k x n_pad tile in the
-  // canonical K-major layout (16 columns of n_pad rows x 16 bytes); if the
-  // driver declines that view, 2-D boxes {8, n_pad} of one column each.
-  // Rows past the batch and k past K read as zero.
+  // x: K bf16 per row, `batch` rows ldx apart; boxes of 64 k x n_pad rows
+  // (128-byte rows, 128-byte swizzle). Rows past the batch and k past K
+  // read as zero.
   CUtensorMap tmap_x;
   {
-    const cuuint64_t dims[3] = {8u, (cuuint64_t)batch, (cuuint64_t)(w.k / 8)};
-    const cuuint64_t strides[2] = {(cuuint64_t)ldx * 2, 16u};
-    const cuuint32_t box[3] = {8u, (cuuint32_t)n_pad, 16u};
-    best.x_boxes = 1;
-    if (encode(&tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+    const cuuint64_t dims[2] = {(cuuint64_t)w.k, (cuuint64_t)batch};
+    const cuuint64_t strides[1] = {(cuuint64_t)ldx * 2};
+    const cuuint32_t box[2] = {64u, (cuuint32_t)n_pad};
+    if (encode(&tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
                const_cast<__nv_bfloat16 *>(x), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS) {
-      const cuuint64_t dims2[2] = {(cuuint64_t)w.k, (cuuint64_t)batch};
-      const cuuint64_t strides2[1] = {(cuuint64_t)ldx * 2};
-      const cuuint32_t box2[2] = {8u, (cuuint32_t)n_pad};
-      best.x_boxes = 16;
-      if (encode(&tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
-                 const_cast<__nv_bfloat16 *>(x), dims2, strides2, box2, estr,
-                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                 CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return cudaErrorInvalidValue;
-    }
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
   }
   // codes (and Format A scales)
   CUtensorMap tmap_c, tmap_s;

@@ -30,6 +30,18 @@ __device__ __forceinline__ uint64_t smem_desc_kmajor(uint32_t addr, uint32_t lbo
          ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
 }
 
+// Shared-memory matrix descriptor for a K-major operand in the 128-byte
+// swizzle layout (as a tensor copy with the 128-byte swizzle writes it):
+// rows of 64 16-bit elements (128 bytes) 128 bytes apart, 16-byte chunk c of
+// row r stored at chunk c ^ (r & 7), groups of 8 rows 1024 bytes apart (SBO),
+// the atom 1024-byte aligned. A k16 step inside the 64-element row starts
+// 32 bytes further. LBO is unused for this layout (encoded as 1); layout
+// type 2 (128-byte swizzle) at bits 61-63, version 1 at bits 46-47.
+__device__ __forceinline__ uint64_t smem_desc_kmajor_sw128(uint32_t addr) {
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | (1ull << 16) |
+         ((uint64_t)(1024u >> 4) << 32) | (1ull << 46) | (2ull << 61);
+}
+
 // Warp-wide: allocate `cols` tensor-memory columns (power of two >= 32); the
 // base address is written to shared memory at `dst`.
 __device__ __forceinline__ void tmem_alloc(uint32_t dst, uint32_t cols) {
