@@ -1050,7 +1050,7 @@ def main():
                     help="layer workload: columns")
     ap.add_argument("--planes", type=int, default=1,
                     help="layer workload: Format A planes")
-    ap.add_argument("--force-path", type=int, default=0, choices=[0, 1, 2],
+    ap.add_argument("--force-path", type=int, default=0, choices=[0, 1, 2, 3],
                     help="kernel family for comparisons: 0 automatic, "
                          "1 CUDA cores, 2 tensor cores")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
