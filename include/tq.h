@@ -201,6 +201,48 @@ tq_status tq_unpack(const tq_weights *w, void *W_bf16_out, int32_t *dev_status,
 tq_status tq_linear(const tq_weights *w, const void *x_bf16, int64_t batch,
                     int64_t ldx, float *y, int64_t ldy, void *cuda_stream);
 
+/* Expert-indexed Format A weights (FUCINA README, "The method": hot experts
+ * carry both ternary planes W ~ d1 T1 + d2 T2, cold experts one; the experts
+ * are stored hot-first, so the second plane covers the prefix 0 .. n_hot - 1).
+ * Every expert is an n_rows x k_cols Format A matrix with group G = 64.
+ *   codes / scales    plane 1 of every expert: expert e at
+ *                     codes + e * n * (k/64) * 13 bytes and
+ *                     scales + e * n * (k/64) fp16 (the Format A layout of
+ *                     one plane); device, 16-byte aligned.
+ *   codes2 / scales2  plane 2 of experts 0 .. n_hot - 1, same layout and
+ *                     strides; NULL when n_hot = 0. */
+typedef struct {
+  int32_t n_experts;       /* E >= 1 */
+  int32_t n_hot;           /* 0 .. E: experts with a second plane */
+  int32_t group;           /* G: must be 64 */
+  int32_t reserved;        /* 0 */
+  int64_t n_rows;          /* N of every expert */
+  int64_t k_cols;          /* K of every expert, a multiple of 64 */
+  const uint8_t *codes;
+  const uint16_t *scales;
+  const uint8_t *codes2;
+  const uint16_t *scales2;
+} tq_experts;
+
+/* Expert-indexed packed matmul (the mixture-of-experts product of the FUCINA
+ * README; a token routed to k experts appears once per expert):
+ *   y[t][n] = sum_k w_{ids[t]}[n][k] x[t][k],  w_e = s1 t1 + s2 t2 for
+ *   e < n_hot, s1 t1 otherwise, for t = 0 .. n_tokens - 1.
+ *   ids       device int32 [n_tokens], 4-byte aligned.
+ *   x         device bf16 [n_tokens][ldx], 16-byte aligned, ldx >= k,
+ *             ldx % 8 == 0.
+ *   y         device fp32 [n_tokens][ldy], 4-byte aligned, ldy >= n.
+ *   n_tokens  0 .. 65535 (0: nothing to do).
+ *   dev_status device int32 or NULL: TQ_ERR_INVALID_ARG when an id lies
+ *             outside 0 .. E - 1; that token's row of y is then NaN.
+ * Same accuracy bound as tq_linear. The ids stay on the device: one launch,
+ * no host synchronisation. Expert-indexed calls have no counterpart of the
+ * tensor-core path: each token is one batch-1 product. */
+tq_status tq_linear_experts(const tq_experts *w, const int32_t *ids,
+                            int64_t n_tokens, const void *x_bf16, int64_t ldx,
+                            float *y, int64_t ldy, int32_t *dev_status,
+                            void *cuda_stream);
+
 /* Static description of a status value. */
 const char *tq_status_string(tq_status status);
 

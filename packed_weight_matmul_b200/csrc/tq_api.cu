@@ -181,6 +181,62 @@ tq_status tq_linear(const tq_weights *w, const void *x_bf16, int64_t batch,
       stream));
 }
 
+tq_status tq_linear_experts(const tq_experts *w, const int32_t *ids,
+                            int64_t n_tokens, const void *x_bf16, int64_t ldx,
+                            float *y, int64_t ldy, int32_t *dev_status,
+                            void *cuda_stream) {
+  if (w == nullptr || n_tokens < 0) return TQ_ERR_INVALID_ARG;
+  if (w->n_experts < 1 || w->n_hot < 0 || w->n_hot > w->n_experts ||
+      w->reserved != 0)
+    return TQ_ERR_INVALID_ARG;
+  if (w->group != 64) return TQ_ERR_UNSUPPORTED;
+  if (w->n_rows < 1 || w->k_cols < 64) return TQ_ERR_SHAPE;
+  if (w->k_cols % 64 != 0) return TQ_ERR_SHAPE;
+  if (w->codes == nullptr || w->scales == nullptr) return TQ_ERR_INVALID_ARG;
+  if (w->n_hot > 0 && (w->codes2 == nullptr || w->scales2 == nullptr))
+    return TQ_ERR_INVALID_ARG;
+  if (!aligned(w->codes, 16) || !aligned(w->scales, 16)) return TQ_ERR_ALIGNMENT;
+  if (w->n_hot > 0 && (!aligned(w->codes2, 16) || !aligned(w->scales2, 16)))
+    return TQ_ERR_ALIGNMENT;
+  if (n_tokens > 65535) return TQ_ERR_UNSUPPORTED;
+  if (n_tokens == 0) return TQ_OK;
+  if (ids == nullptr || x_bf16 == nullptr || y == nullptr)
+    return TQ_ERR_INVALID_ARG;
+  if (ldx < w->k_cols || ldy < w->n_rows) return TQ_ERR_SHAPE;
+  if (!aligned(ids, 4) || !aligned(x_bf16, 16) || ldx % 8 != 0 ||
+      !aligned(y, 4))
+    return TQ_ERR_ALIGNMENT;
+  if (dev_status != nullptr && !aligned(dev_status, 4)) return TQ_ERR_ALIGNMENT;
+  tq::WeightsView v = {};
+  v.format = TQ_FMT_A;
+  v.group = 64;
+  v.planes = w->n_hot > 0 ? 2 : 1;
+  v.rps = 0;
+  v.n = w->n_rows;
+  v.k = w->k_cols;
+  v.codes = w->codes;
+  v.scales = w->scales;
+  v.lut = nullptr;
+  if (!tq::gemv_a_supported(v, 1)) return TQ_ERR_UNSUPPORTED;
+  const int64_t groups = w->n_rows * (w->k_cols / 64);
+  tq::ExpertsView E = {};
+  E.ids = ids;
+  E.n_experts = w->n_experts;
+  E.n_hot = w->n_hot;
+  E.codes = w->codes;
+  E.scales = w->scales;
+  E.codes2 = w->codes2;
+  E.scales2 = w->scales2;
+  E.codes_stride = groups * 13;
+  E.scales_stride = groups;
+  E.ldx = ldx;
+  E.ldy = ldy;
+  E.status = dev_status;
+  return from_cuda(tq::gemv_a_experts(
+      v, E, n_tokens, static_cast<const __nv_bfloat16 *>(x_bf16), y,
+      static_cast<cudaStream_t>(cuda_stream)));
+}
+
 tq_status tq_testing_linear_wait_fault(int32_t withhold_first_arrive,
                                        uint64_t wait_limit_ns) {
   tq::g_test_skip_first_arrive.store(withhold_first_arrive != 0 ? 1 : 0);

@@ -35,6 +35,21 @@ struct WeightsView {
   int64_t scales_plane_stride;  // elements
 };
 
+// Expert-indexed Format A call (tq_linear_experts): token t uses expert
+// ids[t]; ids == nullptr marks a plain call.
+struct ExpertsView {
+  const int32_t *ids;
+  int n_experts, n_hot;
+  const uint8_t *codes;    // plane 1 of every expert
+  const uint16_t *scales;
+  const uint8_t *codes2;   // plane 2 of experts 0 .. n_hot - 1
+  const uint16_t *scales2;
+  int64_t codes_stride;    // bytes between experts
+  int64_t scales_stride;   // elements between experts
+  int64_t ldx, ldy;
+  int32_t *status;
+};
+
 // Raise a kernel's dynamic shared-memory limit to `bytes` once per device.
 // The attribute is one value per function and context; every caller asks for
 // the same (largest) value, so concurrent callers cannot lower it under one

@@ -51,6 +51,7 @@ struct GemvAParams {
   int ks_count;      // CTAs per cluster (K slices)
   int rb_count;      // row blocks
   int rows_max;      // rows of the largest row block
+  int planes_max;    // planes the partial-sum buffer holds
   int64_t ng;        // groups per row
 };
 
@@ -101,13 +102,42 @@ __device__ __forceinline__ float butterfly8(float *v, int lane) {
 
 __global__ void __launch_bounds__(kThreads, 1)
     gemv_a_kernel(WeightsView w, const __nv_bfloat16 *__restrict__ x,
-                  float *__restrict__ y, GemvAParams P) {
+                  float *__restrict__ y, GemvAParams P, ExpertsView E) {
   namespace cg = cooperative_groups;
   extern __shared__ __align__(16) uint8_t smem[];
   const uint32_t tab = (uint32_t)__cvta_generic_to_shared(smem);
   // [planes][rows_max] partial sums, then the CTA's x slice as fp32
   float *red = reinterpret_cast<float *>(smem + kTabBytes);
-  float *xs_all = red + w.planes * P.rows_max;
+  float *xs_all = red + P.planes_max * P.rows_max;
+
+  // Expert-indexed calls: token t = blockIdx.z multiplies x row t by the
+  // matrix of expert ids[t] (plane 2 for the hot prefix e < n_hot) into y
+  // row t. An id outside 0 .. n_experts - 1 computes on expert 0, reports
+  // TQ_ERR_INVALID_ARG and leaves NaN in the row (every CTA of the cluster
+  // reads the same id, so all take the same path).
+  bool bad_id = false;
+  if (E.ids != nullptr) {
+    const int64_t t = blockIdx.z;
+    int e = __ldg(E.ids + t);
+    if (e < 0 || e >= E.n_experts) {
+      bad_id = true;
+      e = 0;
+    }
+    w.codes = E.codes + (int64_t)e * E.codes_stride;
+    w.scales = E.scales + (int64_t)e * E.scales_stride;
+    w.planes = e < E.n_hot ? 2 : 1;
+    if (w.planes == 2) {
+      // plane 2 lives in its own arrays: express it as an offset
+      w.codes_plane_stride =
+          (int64_t)(E.codes2 + (int64_t)e * E.codes_stride - w.codes);
+      w.scales_plane_stride =
+          (int64_t)(E.scales2 + (int64_t)e * E.scales_stride - w.scales);
+    }
+    x += t * E.ldx;
+    y += t * E.ldy;
+    if (bad_id && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0)
+      report(E.status, TQ_ERR_INVALID_ARG);
+  }
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ks = blockIdx.x;  // rank in the cluster = K slice
@@ -121,7 +151,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int r_lo = rows * warp / kWarps;
   const int r_n = rows * (warp + 1) / kWarps - r_lo;
 
-  for (int i = threadIdx.x; i < w.planes * P.rows_max; i += kThreads)
+  for (int i = threadIdx.x; i < P.planes_max * P.rows_max; i += kThreads)
     red[i] = 0.0f;
   // Clear the tables once: a byte >= 243 then reads a finite value (a
   // neighbouring table's entry or the pad).
@@ -270,7 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float *rr = cluster.map_shared_rank(red, q);
       for (int pl = 0; pl < w.planes; ++pl) sum += rr[pl * P.rows_max + r];
     }
-    y[row_lo + r] = sum;
+    y[row_lo + r] = bad_id ? __int_as_float(0x7FC00000) : sum;
   }
   cluster.sync();  // no CTA leaves while others read its partial sums
 }
@@ -326,34 +356,46 @@ int max_clusters(int dev, int ks, size_t smem) {
 
 }  // namespace
 
-cudaError_t gemv_a(const WeightsView &w, const __nv_bfloat16 *x, float *y,
-                   cudaStream_t stream) {
+namespace {
+
+// One launch for `tokens` independent GEMVs (1 for a plain call): grid
+// (K slices, row blocks, tokens), clusters along the K slices.
+cudaError_t launch_gemv_a(const WeightsView &w, const __nv_bfloat16 *x,
+                          float *y, const ExpertsView &E, int64_t tokens,
+                          int planes_max, cudaStream_t stream) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (tokens < 1 || tokens > 65535) return cudaErrorInvalidValue;
   GemvAParams P;
   P.ng = w.k / kG;
+  P.planes_max = planes_max;
   const size_t big = 160 * 1024;  // any request of one CTA per SM
   cudaError_t e = ensure_smem_limit<gemv_a_kernel>(kSmemMax);
   if (e != cudaSuccess) return e;
   // K slices: at most 8 (portable cluster), at least one full window each.
   // Each CTA owns an SM; its time is about windows x (its rows' lookups +
-  // one table build), so take the split with the least of that, counting
-  // only the clusters that are resident together.
+  // one table build). The resident clusters are shared by the tokens: take
+  // the split with the least of (waves x that), waves counted over the
+  // row blocks of every token.
   int best_ks = 1;
   int64_t best_rb = 1, best_ctas = 0;
   double best_cost = 0.0;
   for (int ks = 8; ks >= 1; ks /= 2) {
     if (ks > 1 && (P.ng + kWinGroups - 1) / kWinGroups < ks) continue;
     if ((P.ng + ks - 1) / ks > kMaxSliceGroups) break;
-    int64_t rb = max_clusters(dev, ks, big);
-    if (rb < 1) rb = sms / ks;
+    int64_t res = max_clusters(dev, ks, big);
+    if (res < 1) res = sms / ks;
+    if (res < 1) res = 1;
+    int64_t rb = res / tokens;
     if (rb < 1) rb = 1;
     if (rb > w.n) rb = w.n;
     const int64_t rows = (w.n + rb - 1) / rb;
+    const int64_t waves = (rb * tokens + res - 1) / res;
     const int64_t wins = ((P.ng + ks - 1) / ks + kWinGroups - 1) / kWinGroups;
     const double cost =
-        (double)wins * ((double)((rows + kWarps - 1) / kWarps) * w.planes * 40.0 + 300.0);
+        (double)waves * (double)wins *
+        ((double)((rows + kWarps - 1) / kWarps) * planes_max * 40.0 + 300.0);
     if (best_ctas == 0 || cost < best_cost) {
       best_cost = cost;
       best_ctas = rb * ks;
@@ -367,14 +409,15 @@ cudaError_t gemv_a(const WeightsView &w, const __nv_bfloat16 *x, float *y,
   const int64_t slice = (P.ng + best_ks - 1) / best_ks;
   const int64_t fixed = (int64_t)kTabBytes + slice * kG * 4;
   // the partial sums must fit next to the tables and the x slice
-  const int64_t red_cap = (kSmemMax - fixed) / (4 * w.planes);
+  const int64_t red_cap = (kSmemMax - fixed) / (4 * planes_max);
   if ((w.n + rb - 1) / rb > red_cap) rb = (w.n + red_cap - 1) / red_cap;
   if (rb > 65535) return cudaErrorInvalidConfiguration;
   P.rb_count = (int)rb;
   P.rows_max = (int)((w.n + rb - 1) / rb);
-  const size_t smem = (size_t)fixed + (size_t)w.planes * P.rows_max * 4;
+  const size_t smem = (size_t)fixed + (size_t)planes_max * P.rows_max * 4;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)P.ks_count, (unsigned)P.rb_count, 1);
+  cfg.gridDim = dim3((unsigned)P.ks_count, (unsigned)P.rb_count,
+                     (unsigned)tokens);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
@@ -385,7 +428,21 @@ cudaError_t gemv_a(const WeightsView &w, const __nv_bfloat16 *x, float *y,
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemv_a_kernel, w, x, y, P);
+  return cudaLaunchKernelEx(&cfg, gemv_a_kernel, w, x, y, P, E);
+}
+
+}  // namespace
+
+cudaError_t gemv_a(const WeightsView &w, const __nv_bfloat16 *x, float *y,
+                   cudaStream_t stream) {
+  ExpertsView E = {};
+  return launch_gemv_a(w, x, y, E, 1, w.planes, stream);
+}
+
+cudaError_t gemv_a_experts(const WeightsView &w, const ExpertsView &E,
+                           int64_t tokens, const __nv_bfloat16 *x, float *y,
+                           cudaStream_t stream) {
+  return launch_gemv_a(w, x, y, E, tokens, E.n_hot > 0 ? 2 : 1, stream);
 }
 
 }  // namespace tq

@@ -30,6 +30,12 @@ cudaError_t gemv_b(const WeightsView &w, const __nv_bfloat16 *x, int64_t batch,
 bool gemv_a_supported(const WeightsView &w, int64_t batch);
 cudaError_t gemv_a(const WeightsView &w, const __nv_bfloat16 *x, float *y,
                    cudaStream_t stream);
+// Expert-indexed batch-1 GEMVs (tq_linear_experts): `w` describes one
+// expert's matrix (n, k, group); token t multiplies x row t by expert
+// E.ids[t] into y row t.
+cudaError_t gemv_a_experts(const WeightsView &w, const ExpertsView &E,
+                           int64_t tokens, const __nv_bfloat16 *x, float *y,
+                           cudaStream_t stream);
 
 // Batches that are a real contraction: tcgen05 MMAs on decoded bf16 hi/lo
 // operands, accumulator in tensor memory.

@@ -26,7 +26,7 @@ ENTRY_POINTS = ("tq_packed_bytes", "tq_build_lut", "tq_quantize_pack",
                 "tq_unpack", "tq_linear", "tq_status_string",
                 "tq_encode_b", "tq_testing_linear_wait_fault",
                 "tq_testing_force_linear_path", "tq_testing_tc_self_check",
-                "tq_testing_tc_trace")
+                "tq_testing_tc_trace", "tq_linear_experts")
 
 
 class TqError(RuntimeError):
@@ -43,6 +43,14 @@ class tq_weights(C.Structure):
                 ("codes", C.c_void_p), ("scales", C.c_void_p),
                 ("lut", C.c_void_p), ("codes_plane_stride", C.c_int64),
                 ("scales_plane_stride", C.c_int64)]
+
+
+class tq_experts(C.Structure):
+    _fields_ = [("n_experts", C.c_int32), ("n_hot", C.c_int32),
+                ("group", C.c_int32), ("reserved", C.c_int32),
+                ("n_rows", C.c_int64), ("k_cols", C.c_int64),
+                ("codes", C.c_void_p), ("scales", C.c_void_p),
+                ("codes2", C.c_void_p), ("scales2", C.c_void_p)]
 
 
 def _load():
@@ -74,6 +82,9 @@ def _load():
     L.tq_testing_tc_self_check.argtypes = [i32, P, i32]
     L.tq_testing_tc_trace.restype = C.c_int
     L.tq_testing_tc_trace.argtypes = [P]
+    L.tq_linear_experts.restype = C.c_int
+    L.tq_linear_experts.argtypes = [C.POINTER(tq_experts), P, i64, P, i64, P,
+                                    i64, P, P]
     return L
 
 
@@ -121,6 +132,22 @@ def tq_build_lut(alpha: float, ladder) -> np.ndarray:
                              lad.ctypes.data_as(C.c_void_p),
                              out.ctypes.data_as(C.c_void_p)), "tq_build_lut")
     return out
+
+
+def tq_linear_experts(w: "Experts", ids, x, y, n_tokens=None, ldx=None,
+                      ldy=None, status=None, stream=None, check=True):
+    if n_tokens is None:
+        n_tokens = ids.shape[0]
+    if ldx is None:
+        ldx = x.stride(0)
+    if ldy is None:
+        ldy = y.stride(0)
+    st = _lib.tq_linear_experts(C.byref(w.desc), _ptr(ids), n_tokens, _ptr(x),
+                                ldx, _ptr(y), ldy, _ptr(status),
+                                _stream(stream))
+    if check:
+        _check(st, "tq_linear_experts")
+    return st
 
 
 def tq_testing_linear_wait_fault(withhold_first_arrive: bool,
@@ -189,6 +216,33 @@ def weights_a(codes, scales, n, k, group=64, planes=1, codes_plane_stride=0,
                    codes_plane_stride=codes_plane_stride,
                    scales_plane_stride=scales_plane_stride)
     return Weights(d, (codes, scales))
+
+
+class Experts:
+    """A tq_experts descriptor that keeps its tensors alive."""
+
+    def __init__(self, desc: tq_experts, keep):
+        self.desc = desc
+        self._keep = keep
+
+    @property
+    def n(self):
+        return self.desc.n_rows
+
+    @property
+    def k(self):
+        return self.desc.k_cols
+
+
+def experts_a(codes, scales, n_experts, n, k, n_hot=0, codes2=None,
+              scales2=None, group=64) -> Experts:
+    """Plane 1 of every expert in codes / scales ([E][N][K/G][13] bytes,
+    [E][N][K/G] fp16); plane 2 of experts 0 .. n_hot - 1 in codes2 /
+    scales2 (same layout)."""
+    d = tq_experts(n_experts=n_experts, n_hot=n_hot, group=group, reserved=0,
+                   n_rows=n, k_cols=k, codes=_ptr(codes), scales=_ptr(scales),
+                   codes2=_ptr(codes2), scales2=_ptr(scales2))
+    return Experts(d, (codes, scales, codes2, scales2))
 
 
 def weights_b(codes, lut, rho=None, rows_per_scale=0, n=None, k=None) -> Weights:

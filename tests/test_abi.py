@@ -142,3 +142,46 @@ def test_validation_before_launch(tq):
         E.TQ_ERR_INVALID_ARG
     assert L.tq_unpack(C.byref(_wa(tq).desc), 0x60008, None, None) == \
         E.TQ_ERR_ALIGNMENT
+
+
+def _we(tq, **kw):
+    f = dict(n_experts=4, n_hot=1, group=64, reserved=0, n_rows=8, k_cols=128,
+             codes=0x10000, scales=0x20000, codes2=0x30000, scales2=0x40000)
+    f.update(kw)
+    return tq.tq_experts(**f)
+
+
+def _experts(tq, w, ids=0x50000, tokens=3, x=0x60000, ldx=128, y=0x70000,
+             ldy=8, status=None):
+    return tq.lib().tq_linear_experts(C.byref(w), ids, tokens, x, ldx, y, ldy,
+                                      status, None)
+
+
+def test_experts_validation_before_launch(tq):
+    """tq_linear_experts rejects every bad argument on the host (fake,
+    never dereferenced addresses: no GPU is touched)."""
+    E = tq
+    assert tq.lib().tq_linear_experts(None, 0x50000, 1, 0x60000, 128, 0x70000,
+                                      8, None, None) == E.TQ_ERR_INVALID_ARG
+    assert _experts(tq, _we(tq, n_experts=0)) == E.TQ_ERR_INVALID_ARG
+    assert _experts(tq, _we(tq, n_hot=5)) == E.TQ_ERR_INVALID_ARG
+    assert _experts(tq, _we(tq, n_hot=-1)) == E.TQ_ERR_INVALID_ARG
+    assert _experts(tq, _we(tq, reserved=1)) == E.TQ_ERR_INVALID_ARG
+    assert _experts(tq, _we(tq, group=128)) == E.TQ_ERR_UNSUPPORTED
+    assert _experts(tq, _we(tq, k_cols=96)) == E.TQ_ERR_SHAPE
+    assert _experts(tq, _we(tq, n_rows=0)) == E.TQ_ERR_SHAPE
+    assert _experts(tq, _we(tq, codes=None)) == E.TQ_ERR_INVALID_ARG
+    assert _experts(tq, _we(tq, codes2=None)) == E.TQ_ERR_INVALID_ARG
+    assert _experts(tq, _we(tq, codes2=None, scales2=None, n_hot=0), ids=None,
+                    tokens=0) == E.TQ_OK
+    assert _experts(tq, _we(tq, codes=0x10008)) == E.TQ_ERR_ALIGNMENT
+    assert _experts(tq, _we(tq, scales2=0x40004)) == E.TQ_ERR_ALIGNMENT
+    assert _experts(tq, _we(tq), tokens=-1) == E.TQ_ERR_INVALID_ARG
+    assert _experts(tq, _we(tq), tokens=70000) == E.TQ_ERR_UNSUPPORTED
+    assert _experts(tq, _we(tq), ids=None) == E.TQ_ERR_INVALID_ARG
+    assert _experts(tq, _we(tq), ldx=64) == E.TQ_ERR_SHAPE
+    assert _experts(tq, _we(tq), ldy=4) == E.TQ_ERR_SHAPE
+    assert _experts(tq, _we(tq), ids=0x50002) == E.TQ_ERR_ALIGNMENT
+    assert _experts(tq, _we(tq), x=0x60002) == E.TQ_ERR_ALIGNMENT
+    assert _experts(tq, _we(tq), ldx=132) == E.TQ_ERR_ALIGNMENT
+    assert _experts(tq, _we(tq), status=0x80002) == E.TQ_ERR_ALIGNMENT
