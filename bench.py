@@ -764,6 +764,94 @@ class EncodeB(Workload):
         return f"{min(rows, 256)} rows of each encoder layer shape"
 
 
+class ExpertsA(Workload):
+    """Expert-indexed Format A layer (tq_linear_experts): 128 experts of
+    768 x 2048 (a mixture-of-experts FFN projection), G = 64, the 32 hot
+    experts 0..31 with a second plane; 64 routed rows per call (8 tokens x
+    8 experts), ids seeded uniform on 0..127; weights bf16 0.02*StudentT(5)
+    quantized on the GPU. Algorithmic bytes: the packages (codes + scales,
+    both planes of hot experts) of the distinct experts a call touches."""
+    name = "experts_a"
+    MAX_ROWS = 64
+    E, N, K, HOT, TOKENS = 128, 768, 2048, 32, 64
+    BATCHES = (64,)
+    SOURCES = ("tq_gemv_a.cu", "tq_api.cu")
+
+    def __init__(self):
+        gpr = self.K // 64
+        self.per = self.N * gpr  # groups per expert plane
+        self.pkg = (self.E + self.HOT) * self.per * 15
+        self.copies = max(1, -(-3 * L2_BYTES // self.pkg))
+        g = torch.Generator().manual_seed(41)
+        self.ids_h = torch.randint(0, self.E, (self.TOKENS,), generator=g,
+                                   dtype=torch.int32)
+        used = sorted(set(self.ids_h.tolist()))
+        self.call_bytes = sum((2 if e < self.HOT else 1) * self.per * 15
+                              for e in used)
+
+    def describe(self):
+        return {"workload": f"{self.name}: {self.E} Format A experts of "
+                f"{self.N}x{self.K}, G=64, experts 0..{self.HOT - 1} with two "
+                f"planes, {self.TOKENS} routed rows per call (ids uniform), "
+                "weights bf16 0.02*StudentT(5); x bf16 N(0,1)",
+                "layers_rotated": self.copies,
+                "bytes_resident": self.copies * self.pkg,
+                "l2": "rotating distinct copies, resident bytes > 3x L2",
+                "batches": [self.TOKENS], "parallelism": "replicas"}
+
+    def setup(self, tq, dev):
+        E, N, K, H = self.E, self.N, self.K, self.HOT
+        W = I.student_t_bf16(E * N, K, seed=43).to(dev)
+        ng = E * N * (K // 64)
+        c = torch.empty(2 * ng * 13, dtype=torch.uint8, device=dev)
+        s = torch.empty(2 * ng + 8, dtype=torch.int16, device=dev)
+        st = torch.zeros(1, dtype=torch.int32, device=dev)
+        tq.tq_quantize_pack(W, 64, 2, c, s, st)
+        del W
+        c1, s1 = c[:ng * 13], s[:ng]
+        c2, s2 = c[ng * 13:ng * 13 + H * self.per * 13], s[ng:ng + H * self.per]
+        self.keep = [(c1.clone(), s1.clone(), c2.clone(), s2.clone())
+                     for _ in range(self.copies)]
+        del c, s
+        self.w = [tq.experts_a(a, b, E, N, K, H, cc, d)
+                  for a, b, cc, d in self.keep]
+        self.ids = self.ids_h.to(dev)
+        self.x = I.x_normal(self.TOKENS, K, 47).to(dev)
+        self.y = torch.zeros(self.TOKENS, N, device=dev)
+        self.pin_io([self.x], [self.y])
+
+    def capture(self, tq):
+        calls = [lambda i=i: tq.tq_linear_experts(self.w[i], self.ids, self.x,
+                                                  self.y)
+                 for i in range(self.copies)]
+        return [Step(f"tokens{self.TOKENS}", capture_graph(calls),
+                     self.copies * self.call_bytes, self.copies,
+                     f"linear_experts_a_tokens{self.TOKENS}",
+                     2.0 * self.TOKENS * self.N * self.K * self.copies)]
+
+    def oracle_setup(self):
+        from oracle import oref
+        self.oref = oref
+        # rows 0..63 of a hot and of a cold expert (both planes of the hot)
+        rows, K = 64, self.K
+        c, s = oref.quantize_pack_A(
+            I.bits(I.student_t_bf16(2 * rows, K, seed=43)), 64, 2)
+        c, s = np.asarray(c).reshape(2, -1), np.asarray(s).reshape(2, -1)
+        per = rows * (K // 64)
+        self.pkg_h = (c[0], s[0], c[1][:per * 13], s[1][:per])
+        self.xb = I.bits(I.x_normal(2, K, 47))
+
+    def oracle_jobs(self, rows, r0=0):
+        c1, s1, c2, s2 = self.pkg_h
+        ids = np.array([0, 1], np.int32)
+        return [(lambda: self.oref.linear_experts_A(
+            c1, s1, c2, s2, 2, 1, 64, self.K, ids, self.xb),
+            3 * 64 * (self.K // 64) * 15)]
+
+    def sample_desc(self, rows):
+        return "64 rows of a hot and of a cold expert, one token each"
+
+
 def make_workload(args):
     batches = tuple(args.batch) if args.batch else None
     if args.workload == "decode_step":
@@ -775,7 +863,8 @@ def make_workload(args):
 
 WORKLOADS = {"fmt_b_4096": FmtB4096, "fmt_b_gemma": FmtBGemma,
              "fmt_a_large": FmtALarge, "decode_step": DecodeStep,
-             "fmt_a_small": FmtASmall, "layer": Layer, "encode_b": EncodeB}
+             "fmt_a_small": FmtASmall, "layer": Layer, "encode_b": EncodeB,
+             "experts_a": ExpertsA}
 
 
 # ---- the oracle on the host cores ---------------------------------------------------
