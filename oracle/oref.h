@@ -128,6 +128,21 @@ int oref_linear_B(const uint8_t *codes, int64_t n, int64_t k, const float *lut,
                   int64_t nrows, const uint16_t *x, int64_t batch, int64_t ldx,
                   double *y);
 
+/* Adaptive alphabets (section 8.3): the same with one code book per block of
+ * lut_rows rows (row n uses lut + 256 * (n / lut_rows)); lut_rows = 0 is the
+ * layer's single code book (the functions above). */
+int oref_unpack_Bx(const uint8_t *codes, int64_t n, int64_t k,
+                   const float *lut, int64_t lut_rows, const uint16_t *rho,
+                   int32_t rps, uint16_t *W_out);
+int oref_weights_Bx(const uint8_t *codes, int64_t n, int64_t k,
+                    const float *lut, int64_t lut_rows, const uint16_t *rho,
+                    int32_t rps, const int64_t *rows, int64_t nrows,
+                    double *w_out);
+int oref_linear_Bx(const uint8_t *codes, int64_t n, int64_t k,
+                   const float *lut, int64_t lut_rows, const uint16_t *rho,
+                   int32_t rps, const int64_t *rows, int64_t nrows,
+                   const uint16_t *x, int64_t batch, int64_t ldx, double *y);
+
 /* Encoder (section 3.1; per-row / per-head scale, section 3.3): the greedy
  * 5-step ternary path of every weight over the ladder with zero-bias zeta,
  * r_0 = W / a with a = alpha = max |W| (rps = 0) or a = max |W| over the

@@ -92,6 +92,13 @@ def _declare(L):
     L.oref_weights_B.argtypes = [P, i64, i64, P, P, i32, P, i64, P]
     L.oref_encode_B.restype = C.c_int
     L.oref_encode_B.argtypes = [P, i64, i64, P, C.c_float, i32, P, P, P]
+    L.oref_unpack_Bx.restype = C.c_int
+    L.oref_unpack_Bx.argtypes = [P, i64, i64, P, i64, P, i32, P]
+    L.oref_weights_Bx.restype = C.c_int
+    L.oref_weights_Bx.argtypes = [P, i64, i64, P, i64, P, i32, P, i64, P]
+    L.oref_linear_Bx.restype = C.c_int
+    L.oref_linear_Bx.argtypes = [P, i64, i64, P, i64, P, i32, P, i64, P, i64,
+                                 i64, P]
     L.oref_linear_B.restype = C.c_int
     L.oref_linear_B.argtypes = [P, i64, i64, P, P, i32, P, i64, P, i64, i64,
                                 P]
@@ -232,29 +239,32 @@ def build_lut(alpha: float, ladder, check=True, L=None):
     return _ret(lut, st, check)
 
 
-def unpack_B(codes, lut, rho=None, rps=0, check=True, L=None):
+def unpack_B(codes, lut, rho=None, rps=0, check=True, L=None, lut_rows=0):
+    """lut: one code book [256], or with lut_rows > 0 one per block of
+    lut_rows rows ([ceil(n / lut_rows)][256], section 8.3)."""
     codes = _c(codes, np.uint8)
     n, k = codes.shape
     lut, rho = _c(lut, np.float32), _c(rho, np.uint16)
     out = np.zeros((n, k), np.uint16)
-    st = (L or lib()).oref_unpack_B(_p(codes), n, k, _p(lut), _p(rho), rps,
-                                    _p(out))
+    st = (L or lib()).oref_unpack_Bx(_p(codes), n, k, _p(lut), lut_rows,
+                                     _p(rho), rps, _p(out))
     return _ret(out, st, check)
 
 
-def weights_B(codes, lut, rho=None, rps=0, rows=None, check=True, L=None):
+def weights_B(codes, lut, rho=None, rps=0, rows=None, check=True, L=None,
+              lut_rows=0):
     codes = _c(codes, np.uint8)
     n, k = codes.shape
     lut, rho, rows = _c(lut, np.float32), _c(rho, np.uint16), _c(rows, np.int64)
     nr = n if rows is None else len(rows)
     out = np.zeros((nr, k), np.float64)
-    st = (L or lib()).oref_weights_B(_p(codes), n, k, _p(lut), _p(rho), rps,
-                                     _p(rows), nr, _p(out))
+    st = (L or lib()).oref_weights_Bx(_p(codes), n, k, _p(lut), lut_rows,
+                                      _p(rho), rps, _p(rows), nr, _p(out))
     return _ret(out, st, check)
 
 
 def linear_B(codes, lut, x_bits, rho=None, rps=0, rows=None, check=True,
-             L=None):
+             L=None, lut_rows=0):
     codes = _c(codes, np.uint8)
     n, k = codes.shape
     lut, rho, rows = _c(lut, np.float32), _c(rho, np.uint16), _c(rows, np.int64)
@@ -262,8 +272,9 @@ def linear_B(codes, lut, x_bits, rho=None, rps=0, rows=None, check=True,
     batch, ldx = x.shape
     nr = n if rows is None else len(rows)
     y = np.zeros((batch, nr), np.float64)
-    st = (L or lib()).oref_linear_B(_p(codes), n, k, _p(lut), _p(rho), rps,
-                                    _p(rows), nr, _p(x), batch, ldx, _p(y))
+    st = (L or lib()).oref_linear_Bx(_p(codes), n, k, _p(lut), lut_rows,
+                                     _p(rho), rps, _p(rows), nr, _p(x), batch,
+                                     ldx, _p(y))
     return _ret(y, st, check)
 
 

@@ -24,6 +24,12 @@
  *   B4 unpack yields bf16(fp32(rho * LUT[code])), or bf16(LUT[code]) without
  *      rho; codes >= 243 are OREF_ERR_BAD_CODE;
  *   B5 the matmul uses the exact weight rho * LUT[code] (fp64).
+ *
+ * Adaptive alphabets (section 8.3 "Adaptive alphabets": one ladder per row
+ * or per block of 32 rows instead of one per layer), read as one code book
+ * per block of lut_rows rows: row n decodes with the table
+ * lut + 256 * (n / lut_rows), each built from its block's ladder as above;
+ * lut_rows = 0 is the single code book of the layer.
  */
 #include <math.h>
 #include <stdlib.h>
@@ -47,25 +53,33 @@ int oref_build_lut(float alpha, const float ladder[5], float lut[256]) {
 }
 
 static int check_B(const uint8_t *codes, int64_t n, int64_t k,
-                   const float *lut, const uint16_t *rho, int32_t rps) {
+                   const float *lut, int64_t lut_rows, const uint16_t *rho,
+                   int32_t rps) {
   if (!codes || !lut || n < 0 || k < 0) return OREF_ERR_INVALID_ARG;
-  if (rps < 0) return OREF_ERR_INVALID_ARG;
+  if (rps < 0 || lut_rows < 0) return OREF_ERR_INVALID_ARG;
   if (rps > 0 && !rho) return OREF_ERR_INVALID_ARG;
   return OREF_OK;
 }
 
-int oref_unpack_B(const uint8_t *codes, int64_t n, int64_t k, const float *lut,
-                  const uint16_t *rho, int32_t rps, uint16_t *W_out) {
-  int st = check_B(codes, n, k, lut, rho, rps);
+/* the code book of row r */
+static const float *row_lut(const float *lut, int64_t lut_rows, int64_t r) {
+  return lut_rows > 0 ? lut + 256 * (r / lut_rows) : lut;
+}
+
+int oref_unpack_Bx(const uint8_t *codes, int64_t n, int64_t k,
+                   const float *lut, int64_t lut_rows, const uint16_t *rho,
+                   int32_t rps, uint16_t *W_out) {
+  int st = check_B(codes, n, k, lut, lut_rows, rho, rps);
   if (st != OREF_OK) return st;
   if (!W_out) return OREF_ERR_INVALID_ARG;
   int status = OREF_OK;
   for (int64_t r = 0; r < n; ++r) {
     double scale = (rps > 0) ? oref_f16_to_f64(rho[r / rps]) : 1.0;
+    const float *L = row_lut(lut, lut_rows, r);
     for (int64_t j = 0; j < k; ++j) {
       uint8_t c = codes[r * k + j];
       if (c >= 243 && status == OREF_OK) status = OREF_ERR_BAD_CODE;
-      double v = (double)lut[c];
+      double v = (double)L[c];
       /* rho * LUT: fp16 x fp32 is exact in fp64, then rounded to fp32 */
       float f = (rps > 0) ? oref_f64_to_f32(scale * v) : (float)v;
       W_out[r * k + j] = oref_f32_to_bf16(f);
@@ -74,10 +88,16 @@ int oref_unpack_B(const uint8_t *codes, int64_t n, int64_t k, const float *lut,
   return status;
 }
 
-int oref_weights_B(const uint8_t *codes, int64_t n, int64_t k, const float *lut,
-                   const uint16_t *rho, int32_t rps, const int64_t *rows,
-                   int64_t nrows, double *w_out) {
-  int st = check_B(codes, n, k, lut, rho, rps);
+int oref_unpack_B(const uint8_t *codes, int64_t n, int64_t k, const float *lut,
+                  const uint16_t *rho, int32_t rps, uint16_t *W_out) {
+  return oref_unpack_Bx(codes, n, k, lut, 0, rho, rps, W_out);
+}
+
+int oref_weights_Bx(const uint8_t *codes, int64_t n, int64_t k,
+                    const float *lut, int64_t lut_rows, const uint16_t *rho,
+                    int32_t rps, const int64_t *rows, int64_t nrows,
+                    double *w_out) {
+  int st = check_B(codes, n, k, lut, lut_rows, rho, rps);
   if (st != OREF_OK) return st;
   if (!w_out) return OREF_ERR_INVALID_ARG;
   if (!rows) nrows = n;
@@ -86,20 +106,27 @@ int oref_weights_B(const uint8_t *codes, int64_t n, int64_t k, const float *lut,
     int64_t r = rows ? rows[i] : i;
     if (r < 0 || r >= n) return OREF_ERR_INVALID_ARG;
     double scale = (rps > 0) ? oref_f16_to_f64(rho[r / rps]) : 1.0;
+    const float *L = row_lut(lut, lut_rows, r);
     for (int64_t j = 0; j < k; ++j) {
       uint8_t c = codes[r * k + j];
       if (c >= 243 && status == OREF_OK) status = OREF_ERR_BAD_CODE;
-      w_out[i * k + j] = scale * (double)lut[c]; /* exact (B5) */
+      w_out[i * k + j] = scale * (double)L[c]; /* exact (B5) */
     }
   }
   return status;
 }
 
-int oref_linear_B(const uint8_t *codes, int64_t n, int64_t k, const float *lut,
-                  const uint16_t *rho, int32_t rps, const int64_t *rows,
-                  int64_t nrows, const uint16_t *x, int64_t batch, int64_t ldx,
-                  double *y) {
-  int st = check_B(codes, n, k, lut, rho, rps);
+int oref_weights_B(const uint8_t *codes, int64_t n, int64_t k, const float *lut,
+                   const uint16_t *rho, int32_t rps, const int64_t *rows,
+                   int64_t nrows, double *w_out) {
+  return oref_weights_Bx(codes, n, k, lut, 0, rho, rps, rows, nrows, w_out);
+}
+
+int oref_linear_Bx(const uint8_t *codes, int64_t n, int64_t k,
+                   const float *lut, int64_t lut_rows, const uint16_t *rho,
+                   int32_t rps, const int64_t *rows, int64_t nrows,
+                   const uint16_t *x, int64_t batch, int64_t ldx, double *y) {
+  int st = check_B(codes, n, k, lut, lut_rows, rho, rps);
   if (st != OREF_OK) return st;
   if (!x || !y || batch < 0 || ldx < k) return OREF_ERR_INVALID_ARG;
   if (!rows) nrows = n;
@@ -111,7 +138,7 @@ int oref_linear_B(const uint8_t *codes, int64_t n, int64_t k, const float *lut,
       status = OREF_ERR_INVALID_ARG;
       break;
     }
-    int s = oref_weights_B(codes, n, k, lut, rho, rps, &r, 1, w);
+    int s = oref_weights_Bx(codes, n, k, lut, lut_rows, rho, rps, &r, 1, w);
     if (s != OREF_OK && status == OREF_OK) status = s;
     for (int64_t b = 0; b < batch; ++b) {
       const uint16_t *xb = x + b * ldx;
@@ -122,6 +149,14 @@ int oref_linear_B(const uint8_t *codes, int64_t n, int64_t k, const float *lut,
   }
   free(w);
   return status;
+}
+
+int oref_linear_B(const uint8_t *codes, int64_t n, int64_t k, const float *lut,
+                  const uint16_t *rho, int32_t rps, const int64_t *rows,
+                  int64_t nrows, const uint16_t *x, int64_t batch, int64_t ldx,
+                  double *y) {
+  return oref_linear_Bx(codes, n, k, lut, 0, rho, rps, rows, nrows, x, batch,
+                        ldx, y);
 }
 
 /* ---- encoder (section 3.1 "Encoding", section 3.3 "Per-row scale") -------

@@ -46,11 +46,17 @@ MUTATIONS = {
     "lut_digit_sign": ("oref_format_b.c", "int c = rest % 3 - 1;",
                        "int c = 1 - rest % 3;"),
     "rho_row_index": ("oref_format_b.c",
-                      "double scale = (rps > 0) ? oref_f16_to_f64(rho[r / rps]) : 1.0;\n    for (int64_t j = 0; j < k; ++j) {\n      uint8_t c = codes[r * k + j];\n      if (c >= 243 && status == OREF_OK) status = OREF_ERR_BAD_CODE;\n      w_out",
-                      "double scale = (rps > 0) ? oref_f16_to_f64(rho[r % rps]) : 1.0;\n    for (int64_t j = 0; j < k; ++j) {\n      uint8_t c = codes[r * k + j];\n      if (c >= 243 && status == OREF_OK) status = OREF_ERR_BAD_CODE;\n      w_out"),
+                      "double scale = (rps > 0) ? oref_f16_to_f64(rho[r / rps]) : 1.0;\n    const float *L = row_lut(lut, lut_rows, r);\n    for (int64_t j = 0; j < k; ++j) {\n      uint8_t c = codes[r * k + j];\n      if (c >= 243 && status == OREF_OK) status = OREF_ERR_BAD_CODE;\n      w_out",
+                      "double scale = (rps > 0) ? oref_f16_to_f64(rho[r % rps]) : 1.0;\n    const float *L = row_lut(lut, lut_rows, r);\n    for (int64_t j = 0; j < k; ++j) {\n      uint8_t c = codes[r * k + j];\n      if (c >= 243 && status == OREF_OK) status = OREF_ERR_BAD_CODE;\n      w_out"),
     "dropped_rho_in_matmul": ("oref_format_b.c",
-                              "w_out[i * k + j] = scale * (double)lut[c];",
-                              "w_out[i * k + j] = (double)lut[c];"),
+                              "w_out[i * k + j] = scale * (double)L[c];",
+                              "w_out[i * k + j] = (double)L[c];"),
+    "lut_block_index_off_by_one_row": ("oref_format_b.c",
+                                       "lut + 256 * (r / lut_rows)",
+                                       "lut + 256 * ((r + 1) / lut_rows)"),
+    "lut_block_ignored": ("oref_format_b.c",
+                          "return lut_rows > 0 ? lut + 256 * (r / lut_rows) : lut;",
+                          "return lut;"),
     "encode_tie_to_nonzero": ("oref_format_b.c",
                               "if (fabsf(rn) < ar) {", "if (fabsf(rn) <= ar) {"),
     "encode_zero_bias_ignored": ("oref_format_b.c",

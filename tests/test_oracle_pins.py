@@ -550,3 +550,52 @@ def test_linear_experts_A_brute_force(oref):
                                   np.array([5], np.int32), xb[:1], G,
                                   check=False)
     assert st == oref.ERR_INVALID_ARG
+
+
+# ---- adaptive alphabets (one code book per block of rows, section 8.3) -------
+
+def _block_weights_numpy(codes, alpha, ladders, lut_rows):
+    """fp32(alpha * sum_i c_i a_{b,i}) per weight, from the code's base-3
+    digits (first digit least significant) and the ladder of the row's
+    block b = n // lut_rows; the sum in fp64 over ascending i."""
+    c = codes.astype(np.int64)
+    blk = np.arange(codes.shape[0]) // lut_rows
+    lad = ladders.astype(np.float64)[blk]  # [n][5]
+    s = np.zeros(codes.shape, np.float64)
+    for i in range(5):
+        s = s + ((c // 3 ** i) % 3 - 1) * lad[:, i:i + 1]
+    return (np.float64(alpha) * s).astype(np.float32).astype(np.float64)
+
+
+@pytest.mark.parametrize("n,lut_rows", [(70, 32), (64, 32), (5, 1), (9, 4)])
+def test_adaptive_alphabet_per_block_code_books(oref, n, lut_rows):
+    rng = np.random.default_rng(n * 7 + lut_rows)
+    k = 48
+    nb = -(-n // lut_rows)
+    ladders = rng.uniform(0.01, 1.0, (nb, 5)).astype(np.float32)
+    alpha = np.float32(0.03)
+    luts = np.stack([oref.build_lut(alpha, ladders[b]) for b in range(nb)])
+    codes = rng.integers(0, 243, (n, k)).astype(np.uint8)
+    want = _block_weights_numpy(codes, alpha, ladders, lut_rows)
+    got = oref.weights_B(codes, luts, lut_rows=lut_rows)
+    assert np.array_equal(got, want)
+    # unpack: bf16 of the same weights
+    ub = oref.unpack_B(codes, luts, lut_rows=lut_rows)
+    ref = torch.from_numpy(want.astype(np.float32)).to(torch.bfloat16)
+    assert np.array_equal(ub, ref.view(torch.int16).numpy().view(np.uint16))
+    # matmul against numpy over the same exact weights
+    x = I.x_normal(3, k, 5)
+    xb = I.bits(x)
+    y = oref.linear_B(codes, luts, xb, lut_rows=lut_rows)
+    x64 = x.double().numpy()
+    np.testing.assert_allclose(y, x64 @ want.T, rtol=1e-12, atol=1e-15)
+
+
+def test_adaptive_alphabet_equal_books_match_single_book(oref):
+    rng = np.random.default_rng(2)
+    codes = rng.integers(0, 243, (40, 32)).astype(np.uint8)
+    lut = oref.build_lut(np.float32(0.02), I.ladder_pow3().numpy())
+    luts = np.stack([lut] * 4)
+    x = I.bits(I.x_normal(2, 32, 1))
+    assert np.array_equal(oref.linear_B(codes, luts, x, lut_rows=10),
+                          oref.linear_B(codes, lut, x))
