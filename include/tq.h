@@ -102,6 +102,12 @@ typedef struct {
                               aligned. A: ignored */
   int64_t codes_plane_stride;  /* A: bytes between planes; 0 = dense */
   int64_t scales_plane_stride; /* A: elements between planes; 0 = dense */
+  int64_t lut_rows;        /* B: 0 = one code book for every row; r > 0 =
+                              adaptive alphabet (alphaneural.io page,
+                              section 8.3): row n decodes with the code book
+                              lut + 256 * (n / r), lut holding ceil(n / r)
+                              books of 256 fp32 (one tq_build_lut per
+                              block's ladder). A: must be 0 */
 } tq_weights;
 
 /* Bytes of a package: A = planes * n * (k/G) * (ceil(G/5) + 2) (codes and

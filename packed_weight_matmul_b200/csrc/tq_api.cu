@@ -34,7 +34,10 @@ tq_status check_weights(const tq_weights *w, tq::WeightsView *v) {
   v->rps = w->rows_per_scale;
   v->codes_plane_stride = 0;
   v->scales_plane_stride = 0;
+  v->lut_rows = w->lut_rows;
+  if (w->lut_rows < 0) return TQ_ERR_INVALID_ARG;
   if (w->format == TQ_FMT_A) {
+    if (w->lut_rows != 0) return TQ_ERR_INVALID_ARG;
     if (w->scales == nullptr) return TQ_ERR_INVALID_ARG;
     if (w->planes < 1 || w->planes > 2) return TQ_ERR_INVALID_ARG;
     if (w->group != 64 && w->group != 128) return TQ_ERR_UNSUPPORTED;
@@ -217,6 +220,7 @@ tq_status tq_linear_experts(const tq_experts *w, const int32_t *ids,
   v.codes = w->codes;
   v.scales = w->scales;
   v.lut = nullptr;
+  v.lut_rows = 0;
   if (!tq::gemv_a_supported(v, 1)) return TQ_ERR_UNSUPPORTED;
   const int64_t groups = w->n_rows * (w->k_cols / 64);
   tq::ExpertsView E = {};

@@ -33,6 +33,7 @@ struct WeightsView {
   const float *lut;
   int64_t codes_plane_stride;   // bytes
   int64_t scales_plane_stride;  // elements
+  int64_t lut_rows;             // B: rows per code book (0: one for all)
 };
 
 // Expert-indexed Format A call (tq_linear_experts): token t uses expert

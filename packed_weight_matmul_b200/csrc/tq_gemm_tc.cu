@@ -237,6 +237,26 @@ __device__ __forceinline__ void decode_b_hi(const uint32_t (&cw)[16],
   }
 }
 
+// Format B with a code book per block of rows (adaptive alphabet): 64 codes
+// of one row -> 32 hi and 32 lo bf16 pairs through the warp's compact book
+// (256 words bf16 hi | lo << 16 at ctab).
+__device__ __forceinline__ void decode_b_compact(const uint32_t (&cw)[16],
+                                                 uint32_t ctab,
+                                                 uint32_t (&hi)[32],
+                                                 uint32_t (&lo)[32]) {
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const uint32_t v0 = lut32(ctab + ((cw[j] << 2) & 0x3FCu));
+    const uint32_t v1 = lut32(ctab + ((cw[j] >> 6) & 0x3FCu));
+    const uint32_t v2 = lut32(ctab + ((cw[j] >> 14) & 0x3FCu));
+    const uint32_t v3 = lut32(ctab + ((cw[j] >> 22) & 0x3FCu));
+    hi[2 * j] = prmt(v0, v1, 0x5410u);
+    lo[2 * j] = prmt(v0, v1, 0x7632u);
+    hi[2 * j + 1] = prmt(v2, v3, 0x5410u);
+    lo[2 * j + 1] = prmt(v2, v3, 0x7632u);
+  }
+}
+
 // Format A: one group (13 code bytes, realigned into b[0..3]) -> 32 hi and
 // 32 lo bf16 pairs of s*t. (nh, ph) = (-s_hi with a zero upper half, +s_hi)
 // are the byte sources of the selecting permute; (nl, pl) the same for s_lo.
@@ -458,7 +478,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   // test runs in every CTA on the same table, so all CTAs agree.
   bool grid = false;
   float unit = 1.0f;
-  if constexpr (FMT == TQ_FMT_B) {
+  // adaptive alphabet: every decoder warp builds its rows' compact book per
+  // tile in the table region; no shared table, no single-operand path
+  const bool adaptive = FMT == TQ_FMT_B && w.lut_rows > 0;
+  if (FMT == TQ_FMT_B && !adaptive) {
     __syncthreads();  // the unit word is initialised
     float lv = 0.0f;
     if (threadIdx.x < 243) {
@@ -480,7 +503,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (grid) unit = u;
   }
   // the lane-replicated table
-  if constexpr (FMT == TQ_FMT_B) {
+  if (FMT == TQ_FMT_B && !adaptive) {
     for (int i = threadIdx.x; i < 256 * 8; i += blockDim.x) {
       const int e = i >> 3, j = i & 7;
       const float v = __ldg(w.lut + e);
@@ -496,7 +519,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       sts128(tab + (uint32_t)e * 256u + (uint32_t)j * 16u, word, word, word,
              word);
     }
-  } else {
+  } else if (FMT == TQ_FMT_A) {
     for (int i = threadIdx.x; i < 256 * 16; i += blockDim.x) {
       const int e = i >> 4, j = i & 15;
       const uint2 v = selector_entry((uint32_t)e);
@@ -809,9 +832,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool skip_first = P.skip_first_arrive != 0;
     int cs = 0, uc = 0, as = 0, ua = 0;
     bool ok = true;
+    // this warp's compact book (adaptive alphabet)
+    const uint32_t ctab = tab + (uint32_t)(warp - kWarpDec) * 1024u;
     for (int t = cid; ok && t < P.tiles; t += nclusters) {
       const int64_t row = (int64_t)t * kTileM + r;
       const bool row_ok = row < N;
+      if (adaptive) {
+        // rows t * 128 + 32 q .. + 31 share one book (lut_rows % 32 == 0);
+        // a warp wholly past N reads book 0 (its weights are masked)
+        const int64_t r0w = (int64_t)t * kTileM + 32 * q;
+        const float *bl = w.lut + ((r0w < N ? r0w : 0) / w.lut_rows) * 256;
+        __syncwarp();  // this warp's lookups of the previous tile are done
+        for (int e = lane; e < 256; e += 32) {
+          const float v = __ldg(bl + e);
+          const uint32_t h = bf16_bits_rn(v);
+          const uint32_t l = bf16_bits_rn(v - __uint_as_float(h << 16));
+          asm volatile("st.shared.u32 [%0], %1;" ::"r"(ctab + 4u * (uint32_t)e),
+                       "r"(h | l << 16)
+                       : "memory");
+        }
+        __syncwarp();
+      }
       for (int ws = it0; ws < it1;) {
         const int we = window_end(ws, it1, P.kblocks, kWin);
         ok = __all_sync(0xFFFFFFFFu,
@@ -876,7 +917,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               cw[4 * j + 2] = v4.z;
               cw[4 * j + 3] = v4.w;
             }
-            if (grid)
+            if (adaptive)
+              decode_b_compact(cw, ctab, hi, lo);
+            else if (grid)
               decode_b_hi(cw, lane_tab, hi);
             else
               decode_b(cw, lane_tab, hi, lo);
@@ -1237,7 +1280,8 @@ bool gemm_tc_supported(const WeightsView &w, int64_t batch) {
   // tensor-copy coordinates are 32-bit
   if (batch < 1 || w.k < 1 || w.n >= (1ll << 31) || w.k >= (1ll << 31))
     return false;
-  if (w.format == TQ_FMT_B) return true;
+  // adaptive alphabet: a decoder warp's 32 rows must share a code book
+  if (w.format == TQ_FMT_B) return w.lut_rows % 32 == 0;
   return w.format == TQ_FMT_A && w.group == 64;
 }
 

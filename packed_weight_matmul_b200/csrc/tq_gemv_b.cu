@@ -448,7 +448,8 @@ int device_sms() {
 }  // namespace
 
 bool gemv_b_supported(const WeightsView &w, int64_t batch) {
-  return w.format == TQ_FMT_B && batch >= 1 && batch <= 4;
+  // one code book per layer: the kernel keeps it lane-replicated on chip
+  return w.format == TQ_FMT_B && w.lut_rows == 0 && batch >= 1 && batch <= 4;
 }
 
 cudaError_t gemv_b(const WeightsView &w, const __nv_bfloat16 *x, int64_t batch,

@@ -11,6 +11,13 @@ cudaError_t launch_linear(const WeightsView &w, const __nv_bfloat16 *x,
   const int force = g_test_force_path.load();
   if ((force == 2 || force == 3) && gemm_tc_supported(w, batch))
     return gemm_tc(w, x, batch, ldx, y, ldy, stream);
+  if (w.format == TQ_FMT_B && w.lut_rows > 0) {
+    // adaptive alphabet: the tensor-core kernel when every warp's 32 rows
+    // share a code book (any batch), else the one-warp-per-row kernel
+    if (gemm_tc_supported(w, batch))
+      return gemm_tc(w, x, batch, ldx, y, ldy, stream);
+    return linear_simple(w, x, batch, ldx, y, ldy, stream);
+  }
   if (force == 1) {
     if (gemv_b_supported(w, batch))
       return gemv_b(w, x, batch, ldx, y, ldy, stream);

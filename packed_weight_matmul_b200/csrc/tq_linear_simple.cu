@@ -29,19 +29,24 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 &v, float *f) {
   }
 }
 
+// One warp per row. The code book sits in shared memory: the layer's one
+// book, or with one book per block of lut_rows rows (adaptive alphabet)
+// each warp's copy of its row's book.
 template <int BT>
 __global__ void __launch_bounds__(kWarps * 32)
     linear_b_simple(const uint8_t *__restrict__ codes, int64_t n, int64_t k,
-                    const float *__restrict__ lut,
+                    const float *__restrict__ lut, int64_t lut_rows,
                     const uint16_t *__restrict__ rho, int rps,
                     const __nv_bfloat16 *__restrict__ x, int64_t ldx,
                     float *__restrict__ y, int64_t ldy) {
-  __shared__ float sL[kLutEntries];
-  for (int i = threadIdx.x; i < kLutEntries; i += blockDim.x) sL[i] = lut[i];
-  __syncthreads();
+  __shared__ float sLw[kWarps][kLutEntries];
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int64_t row = (int64_t)blockIdx.x * kWarps + warp;
   if (row >= n) return;
+  float *sL = sLw[warp];
+  const float *rl = lut_rows > 0 ? lut + (row / lut_rows) * kLutEntries : lut;
+  for (int i = lane; i < kLutEntries; i += 32) sL[i] = rl[i];
+  __syncwarp();
   float acc[BT];
 #pragma unroll
   for (int b = 0; b < BT; ++b) acc[b] = 0.0f;
@@ -126,7 +131,7 @@ cudaError_t launch_b(const WeightsView &w, const __nv_bfloat16 *x, int64_t ldx,
                      float *y, int64_t ldy, cudaStream_t stream) {
   const unsigned blocks = (unsigned)((w.n + kWarps - 1) / kWarps);
   linear_b_simple<BT><<<blocks, kWarps * 32, 0, stream>>>(
-      w.codes, w.n, w.k, w.lut, w.scales, w.rps, x, ldx, y, ldy);
+      w.codes, w.n, w.k, w.lut, w.lut_rows, w.scales, w.rps, x, ldx, y, ldy);
   return cudaGetLastError();
 }
 

@@ -98,10 +98,11 @@ __global__ void __launch_bounds__(kGroupsPerBlock)
 }
 
 // Format B: one thread per 16 codes (k % 16 == 0, so a chunk never crosses a
-// row).
+// row). With one code book per block of lut_rows rows (adaptive alphabet)
+// the row's book is read through the read-only cache.
 __global__ void __launch_bounds__(256)
     unpack_b_kernel(const uint8_t *__restrict__ codes, int64_t n, int64_t k,
-                    const float *__restrict__ lut,
+                    const float *__restrict__ lut, int64_t lut_rows,
                     const uint16_t *__restrict__ rho, int rps,
                     uint16_t *__restrict__ out, int32_t *status) {
   __shared__ float sL[kLutEntries];
@@ -113,6 +114,7 @@ __global__ void __launch_bounds__(256)
        c += (int64_t)gridDim.x * blockDim.x) {
     const int64_t row = (c * 16) / k;
     const float r = rho ? __half2float(__ushort_as_half(rho[row / rps])) : 1.0f;
+    const float *rl = lut_rows > 0 ? lut + (row / lut_rows) * kLutEntries : nullptr;
     const uint4 cv = __ldcs(reinterpret_cast<const uint4 *>(codes) + c);
     const uint32_t words[4] = {cv.x, cv.y, cv.z, cv.w};
     uint32_t o[8];
@@ -123,7 +125,7 @@ __global__ void __launch_bounds__(256)
       for (int e = 0; e < 4; ++e) {
         const uint32_t code = (words[q] >> (8 * e)) & 0xFFu;
         bad |= code >= 243u;
-        float v = sL[code];
+        float v = rl != nullptr ? __ldg(rl + code) : sL[code];
         if (rho) v = __fmul_rn(r, v);  // fp16 x fp32 rounded once to fp32
         h[e] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
       }
@@ -165,8 +167,8 @@ cudaError_t launch_unpack(const WeightsView &w, uint16_t *out,
   const int64_t chunks = w.n * (w.k / 16);
   const int64_t want = (chunks + 255) / 256;
   const int blocks = (int)(want < (int64_t)sms * 8 ? want : (int64_t)sms * 8);
-  unpack_b_kernel<<<blocks, 256, 0, stream>>>(w.codes, w.n, w.k, w.lut,
-                                              w.scales, w.rps, out, status);
+  unpack_b_kernel<<<blocks, 256, 0, stream>>>(
+      w.codes, w.n, w.k, w.lut, w.lut_rows, w.scales, w.rps, out, status);
   return cudaGetLastError();
 }
 

@@ -42,7 +42,8 @@ class tq_weights(C.Structure):
                 ("n_rows", C.c_int64), ("k_cols", C.c_int64),
                 ("codes", C.c_void_p), ("scales", C.c_void_p),
                 ("lut", C.c_void_p), ("codes_plane_stride", C.c_int64),
-                ("scales_plane_stride", C.c_int64)]
+                ("scales_plane_stride", C.c_int64),
+                ("lut_rows", C.c_int64)]
 
 
 class tq_experts(C.Structure):
@@ -245,13 +246,17 @@ def experts_a(codes, scales, n_experts, n, k, n_hot=0, codes2=None,
     return Experts(d, (codes, scales, codes2, scales2))
 
 
-def weights_b(codes, lut, rho=None, rows_per_scale=0, n=None, k=None) -> Weights:
+def weights_b(codes, lut, rho=None, rows_per_scale=0, n=None, k=None,
+              lut_rows=0) -> Weights:
+    """lut: one code book (256 fp32), or with lut_rows > 0 one per block of
+    lut_rows rows ([ceil(n / lut_rows)][256], the adaptive alphabet)."""
     if n is None:
         n, k = codes.shape
     d = tq_weights(format=TQ_FMT_B, group=0, planes=1,
                    rows_per_scale=rows_per_scale if rho is not None else 0,
                    n_rows=n, k_cols=k, codes=_ptr(codes), scales=_ptr(rho),
-                   lut=_ptr(lut), codes_plane_stride=0, scales_plane_stride=0)
+                   lut=_ptr(lut), codes_plane_stride=0, scales_plane_stride=0,
+                   lut_rows=lut_rows)
     return Weights(d, (codes, lut, rho))
 
 

@@ -185,3 +185,12 @@ def test_experts_validation_before_launch(tq):
     assert _experts(tq, _we(tq), x=0x60002) == E.TQ_ERR_ALIGNMENT
     assert _experts(tq, _we(tq), ldx=132) == E.TQ_ERR_ALIGNMENT
     assert _experts(tq, _we(tq), status=0x80002) == E.TQ_ERR_ALIGNMENT
+
+
+def test_lut_rows_validation(tq):
+    """lut_rows: negative is rejected, and Format A must leave it 0."""
+    E = tq
+    assert _linear(tq, _wb(tq, lut_rows=-1)) == E.TQ_ERR_INVALID_ARG
+    assert _linear(tq, _wa(tq, lut_rows=32)) == E.TQ_ERR_INVALID_ARG
+    # a zero-row call with per-block books is valid and launches nothing
+    assert _linear(tq, _wb(tq, n_rows=0, lut_rows=32), ldy=0) == E.TQ_OK
