@@ -552,21 +552,27 @@ class Layer(Workload):
     name = "layer"
     MAX_ROWS = 256
 
-    def __init__(self, fmt="B", n=8192, k=5376, batches=(1,), planes=1):
+    def __init__(self, fmt="B", n=8192, k=5376, batches=(1,), planes=1,
+                 lut_rows=0):
         self.fmt, self.n, self.k = fmt.upper(), n, k
         self.BATCHES = tuple(batches)
         self.planes = planes
+        self.lut_rows = lut_rows if self.fmt == "B" else 0
+        self.books = -(-n // lut_rows) if self.lut_rows else 1
         if self.fmt == "A":
             self.pkg = planes * n * (k // 64) * 15
         else:
-            self.pkg = n * k + 972
+            self.pkg = n * k + 972 * self.books
         self.copies = max(1, -(-3 * L2_BYTES // self.pkg))
 
     def describe(self):
         what = (f"Format A {self.n}x{self.k}, G=64, {self.planes} plane(s), "
                 "quantized from bf16 0.02*StudentT(5)" if self.fmt == "A" else
                 f"Format B {self.n}x{self.k}, codes uniform 0..242, ladder "
-                "a_k=3^-(k-1), alpha=0.02, no rho")
+                "a_k=3^-(k-1), alpha=0.02, no rho" if not self.lut_rows else
+                f"Format B {self.n}x{self.k}, codes uniform 0..242, adaptive "
+                f"alphabet: one code book per {self.lut_rows} rows (ladder "
+                "amplitudes U(0.01, 1) per block, seeded), alpha=0.02, no rho")
         return {"workload": f"{self.name}: {what}; x bf16 N(0,1) at batch "
                 f"{', '.join(map(str, self.BATCHES))}",
                 "layers_rotated": self.copies,
@@ -588,14 +594,22 @@ class Layer(Workload):
             self.w = [tq.weights_a(c, s, n, k, 64, self.planes)
                       for c, s in self.keep]
         else:
-            lut = tq.tq_build_lut(I.ALPHA, I.ladder_pow3().numpy())
-            self.lut_d = torch.from_numpy(lut).to(dev)
+            self.lut_d = torch.from_numpy(self.book_array(tq.tq_build_lut)).to(dev)
             self.keep = [I.codes_uniform(n, k, 5 + i, device=dev)
                          for i in range(self.copies)]
-            self.w = [tq.weights_b(c, self.lut_d) for c in self.keep]
+            self.w = [tq.weights_b(c, self.lut_d, lut_rows=self.lut_rows)
+                      for c in self.keep]
         self.x = {b: I.x_normal(b, k, 60 + b).to(dev) for b in self.BATCHES}
         self.y = {b: torch.zeros(b, n, device=dev) for b in self.BATCHES}
         self.pin_io(list(self.x.values()), list(self.y.values()))
+
+    def book_array(self, build):
+        """The layer's code book, or one per block (seeded ladders)."""
+        if not self.lut_rows:
+            return build(I.ALPHA, I.ladder_pow3().numpy())
+        rng = np.random.default_rng(17)
+        lad = rng.uniform(0.01, 1.0, (self.books, 5)).astype(np.float32)
+        return np.stack([build(I.ALPHA, lad[b]) for b in range(self.books)])
 
     def capture(self, tq):
         steps = []
@@ -619,7 +633,7 @@ class Layer(Workload):
             self.pkg_h = oref.quantize_pack_A(Wh, 64, self.planes)
         else:
             self.codes_h = I.codes_uniform(rows, self.k, 5).numpy()
-            self.lut_h = oref.build_lut(I.ALPHA, I.ladder_pow3().numpy())
+            self.lut_h = self.book_array(oref.build_lut)
         self.xb = {b: I.bits(I.x_normal(b, self.k, 60 + b))
                    for b in self.BATCHES}
 
@@ -635,8 +649,12 @@ class Layer(Workload):
                     self.planes * rows * (self.k // 64) * 15))
             else:
                 c = self.codes_h[r0:r0 + rows]
-                jobs.append((lambda b=b, c=c: self.oref.linear_B(
-                    c, self.lut_h, self.xb[b]), rows * self.k))
+                # the sample's rows r0.. decode with their own books
+                lr = self.lut_rows
+                L = self.lut_h if not lr else \
+                    self.lut_h[r0 // lr:][:-(-rows // lr) + 1]
+                jobs.append((lambda b=b, c=c, L=L: self.oref.linear_B(
+                    c, L, self.xb[b], lut_rows=lr), rows * self.k))
         return jobs
 
     def sample_desc(self, rows):
@@ -857,7 +875,8 @@ def make_workload(args):
     if args.workload == "decode_step":
         return DecodeStep(batches=batches or I.DECODE_BATCHES)
     if args.workload == "layer":
-        return Layer(args.fmt, args.n, args.k, batches or (1,), args.planes)
+        return Layer(args.fmt, args.n, args.k, batches or (1,), args.planes,
+                     args.lut_rows)
     return WORKLOADS[args.workload]()
 
 
@@ -1142,6 +1161,9 @@ def main():
     ap.add_argument("--force-path", type=int, default=0, choices=[0, 1, 2, 3],
                     help="kernel family for comparisons: 0 automatic, "
                          "1 CUDA cores, 2 tensor cores")
+    ap.add_argument("--lut-rows", type=int, default=0,
+                    help="layer workload, Format B: rows per code book "
+                         "(adaptive alphabet); 0 = one code book")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-seconds", type=float, default=90.0,
