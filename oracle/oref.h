@@ -143,6 +143,15 @@ int oref_linear_Bx(const uint8_t *codes, int64_t n, int64_t k,
                    int32_t rps, const int64_t *rows, int64_t nrows,
                    const uint16_t *x, int64_t batch, int64_t ldx, double *y);
 
+/* 7-bit truncated alphabet (section 8.1): `used` = the distinct codes in
+ * ascending order (<= 128, else OREF_ERR_RANGE; padded with 121), 16 indices
+ * into it per 14 bytes, little-endian (index j at bits 7j .. 7j+6), rows of
+ * 14 k / 16 bytes (k % 16 == 0). unpack7_codes inverts pack7 to codes. */
+int oref_pack7(const uint8_t *codes, int64_t n, int64_t k, uint8_t used[128],
+               int32_t *n_used, uint8_t *packed);
+int oref_unpack7_codes(const uint8_t *packed, const uint8_t used[128],
+                       int64_t n, int64_t k, uint8_t *codes);
+
 /* Encoder (section 3.1; per-row / per-head scale, section 3.3): the greedy
  * 5-step ternary path of every weight over the ladder with zero-bias zeta,
  * r_0 = W / a with a = alpha = max |W| (rps = 0) or a = max |W| over the

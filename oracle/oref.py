@@ -99,6 +99,10 @@ def _declare(L):
     L.oref_linear_Bx.restype = C.c_int
     L.oref_linear_Bx.argtypes = [P, i64, i64, P, i64, P, i32, P, i64, P, i64,
                                  i64, P]
+    L.oref_pack7.restype = C.c_int
+    L.oref_pack7.argtypes = [P, i64, i64, P, P, P]
+    L.oref_unpack7_codes.restype = C.c_int
+    L.oref_unpack7_codes.argtypes = [P, P, i64, i64, P]
     L.oref_linear_B.restype = C.c_int
     L.oref_linear_B.argtypes = [P, i64, i64, P, P, i32, P, i64, P, i64, i64,
                                 P]
@@ -309,3 +313,40 @@ def linear_experts_A(codes1, scales1, codes2, scales2, n_experts, n_hot, n, k,
         _p(codes1), _p(scales1), _p(codes2), _p(scales2), n_experts, n_hot,
         n, k, G, _p(ids), tokens, _p(x), ldx, _p(y))
     return _ret(y, st, check)
+
+
+# ---- 7-bit truncated alphabet (section 8.1) ---------------------------------
+
+def pack7(codes, check=True, L=None):
+    """codes uint8 [n][k] (k % 16 == 0) -> (used uint8 [128], n_used,
+    packed uint8 [n][14 k / 16])."""
+    codes = _c(codes, np.uint8)
+    n, k = codes.shape
+    used = np.zeros(128, np.uint8)
+    cnt = np.zeros(1, np.int32)
+    packed = np.zeros((n, 14 * (k // 16)), np.uint8)
+    st = (L or lib()).oref_pack7(_p(codes), n, k, _p(used), _p(cnt),
+                                 _p(packed))
+    return _ret((used, int(cnt[0]), packed), st, check)
+
+
+def unpack7_codes(packed, used, n, k, check=True, L=None):
+    packed, used = _c(packed, np.uint8), _c(used, np.uint8)
+    codes = np.zeros((n, k), np.uint8)
+    st = (L or lib()).oref_unpack7_codes(_p(packed), _p(used), n, k,
+                                         _p(codes))
+    return _ret(codes, st, check)
+
+
+def linear_B7(packed, used, n, k, lut, x_bits, rho=None, rps=0, rows=None,
+              check=True, L=None):
+    """The 7-bit layer's matmul: index i is the code used[i], then Format
+    B's matmul over the same code book."""
+    codes = unpack7_codes(packed, used, n, k, L=L)
+    return linear_B(codes, lut, x_bits, rho, rps, rows, check, L)
+
+
+def unpack_B7(packed, used, n, k, lut, rho=None, rps=0, check=True, L=None):
+    codes = unpack7_codes(packed, used, n, k, L=L)
+    return unpack_B(codes, lut, rho, rps, check, L)
+

@@ -251,3 +251,76 @@ int oref_encode_B(const uint16_t *W, int64_t n, int64_t k,
   }
   return status;
 }
+
+/* ---- 7-bit truncated alphabet (section 8.1 "Variable-depth words") --------
+ *
+ * When a layer uses only a few of the 243 words, a code fits in 7 bits
+ * next to a per-layer table of the words in use. Readings where the page
+ * leaves a step open:
+ *   T1 the table `used` lists the distinct codes of the layer in ascending
+ *      order, at most 128 of them (more is OREF_ERR_RANGE); entries past the
+ *      count hold 121, the all-zero word;
+ *   T2 a weight stores the index of its code in that table;
+ *   T3 16 indices are packed little-endian into 14 bytes: index j of a
+ *      chunk occupies bits 7j .. 7j + 6 of the chunk read as a 112-bit
+ *      integer whose byte 0 holds bits 0 .. 7; a row of k codes (k a multiple
+ *      of 16) takes 14 k / 16 bytes, rows back to back;
+ *   T4 index i decodes to the code used[i], so the weight is LUT[used[i]]
+ *      (times rho as in Format B) and the matmul is Format B's.
+ */
+int oref_pack7(const uint8_t *codes, int64_t n, int64_t k, uint8_t used[128],
+               int32_t *n_used, uint8_t *packed) {
+  if (!codes || !used || !n_used || !packed || n < 0 || k < 0 || k % 16 != 0)
+    return OREF_ERR_INVALID_ARG;
+  int present[256] = {0};
+  for (int64_t i = 0; i < n * k; ++i) present[codes[i]] = 1;
+  int count = 0;
+  int index_of[256];
+  for (int c = 0; c < 256; ++c) {
+    index_of[c] = -1;
+    if (present[c]) {
+      if (count == 128) return OREF_ERR_RANGE;
+      index_of[c] = count;
+      used[count++] = (uint8_t)c;
+    }
+  }
+  for (int i = count; i < 128; ++i) used[i] = 121;
+  *n_used = count;
+  const int64_t row_bytes = 14 * (k / 16);
+  for (int64_t r = 0; r < n; ++r) {
+    for (int64_t ch = 0; ch < k / 16; ++ch) {
+      uint8_t *out = packed + r * row_bytes + 14 * ch;
+      for (int b = 0; b < 14; ++b) out[b] = 0;
+      for (int j = 0; j < 16; ++j) {
+        const int idx = index_of[codes[r * k + 16 * ch + j]];
+        for (int bit = 0; bit < 7; ++bit) /* bit 7j + bit of the chunk */
+          if ((idx >> bit) & 1) {
+            const int pos = 7 * j + bit;
+            out[pos / 8] |= (uint8_t)(1u << (pos % 8));
+          }
+      }
+    }
+  }
+  return OREF_OK;
+}
+
+int oref_unpack7_codes(const uint8_t *packed, const uint8_t used[128],
+                       int64_t n, int64_t k, uint8_t *codes) {
+  if (!packed || !used || !codes || n < 0 || k < 0 || k % 16 != 0)
+    return OREF_ERR_INVALID_ARG;
+  const int64_t row_bytes = 14 * (k / 16);
+  for (int64_t r = 0; r < n; ++r) {
+    for (int64_t ch = 0; ch < k / 16; ++ch) {
+      const uint8_t *in = packed + r * row_bytes + 14 * ch;
+      for (int j = 0; j < 16; ++j) {
+        int idx = 0;
+        for (int bit = 0; bit < 7; ++bit) {
+          const int pos = 7 * j + bit;
+          idx |= ((in[pos / 8] >> (pos % 8)) & 1) << bit;
+        }
+        codes[r * k + 16 * ch + j] = used[idx];
+      }
+    }
+  }
+  return OREF_OK;
+}

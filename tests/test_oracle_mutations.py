@@ -80,6 +80,15 @@ MUTATIONS = {
                                  "int s = oref_weights_A(codes1,"),
     "experts_drop_second_plane": ("oref_format_a.c",
                                   "? w1[j] + w2[j] : w1[j];", "? w1[j] : w1[j];"),
+    "pack7_bits_msb_first": ("oref_format_b.c",
+                             "const int pos = 7 * j + bit;\n            out[pos / 8]",
+                             "const int pos = 7 * j + (6 - bit);\n            out[pos / 8]"),
+    "pack7_pad_word_zero": ("oref_format_b.c",
+                            "for (int i = count; i < 128; ++i) used[i] = 121;",
+                            "for (int i = count; i < 128; ++i) used[i] = 0;"),
+    "unpack7_index_off_by_one": ("oref_format_b.c",
+                                 "codes[r * k + 16 * ch + j] = used[idx];",
+                                 "codes[r * k + 16 * ch + j] = used[(idx + 1) & 127];"),
     "round_ties_up": ("oref_fp.c",
                       "return (fmod(f, 2.0) == 0.0) ? f : f + 1.0;",
                       "return f + 1.0;"),

@@ -599,3 +599,59 @@ def test_adaptive_alphabet_equal_books_match_single_book(oref):
     x = I.bits(I.x_normal(2, 32, 1))
     assert np.array_equal(oref.linear_B(codes, luts, x, lut_rows=10),
                           oref.linear_B(codes, lut, x))
+
+
+# ---- 7-bit truncated alphabet (section 8.1) ---------------------------------
+
+def _pack7_python(codes):
+    """Independent restatement: the used table is np.unique (padded with the
+    all-zero word 121), and each 16-index chunk is the little-endian 14-byte
+    image of sum_j idx_j * 2^(7 j)."""
+    used = np.unique(codes)
+    idx = np.searchsorted(used, codes)
+    n, k = codes.shape
+    out = bytearray()
+    for r in range(n):
+        for ch in range(k // 16):
+            v = 0
+            for j in range(16):
+                v |= int(idx[r, 16 * ch + j]) << (7 * j)
+            out += v.to_bytes(14, "little")
+    table = np.full(128, 121, np.uint8)
+    table[:len(used)] = used
+    return table, len(used), np.frombuffer(bytes(out), np.uint8).reshape(n, -1)
+
+
+@pytest.mark.parametrize("n,k,distinct", [(3, 32, 45), (7, 64, 128), (1, 16, 1),
+                                          (5, 48, 18)])
+def test_pack7_layout_and_round_trip(oref, n, k, distinct):
+    rng = np.random.default_rng(n * 100 + distinct)
+    words = rng.choice(243, distinct, replace=False)
+    codes = rng.choice(words, (n, k)).astype(np.uint8)
+    codes.reshape(-1)[:distinct] = words  # every word present
+    used, cnt, packed = oref.pack7(codes)
+    t_used, t_cnt, t_packed = _pack7_python(codes)
+    assert cnt == t_cnt == distinct
+    assert np.array_equal(used, t_used)
+    assert np.array_equal(packed, t_packed)
+    assert np.array_equal(oref.unpack7_codes(packed, used, n, k), codes)
+
+
+def test_pack7_too_many_words_and_shape(oref):
+    codes = np.arange(129, dtype=np.uint8).repeat(16).reshape(129, 16)
+    _, st = oref.pack7(codes, check=False)
+    assert st == oref.ERR_RANGE
+    codes = np.zeros((2, 24), np.uint8)
+    _, st = oref.pack7(codes, check=False)
+    assert st == oref.ERR_INVALID_ARG
+
+
+def test_linear_b7_equals_format_b(oref):
+    rng = np.random.default_rng(4)
+    words = rng.choice(243, 45, replace=False)
+    codes = rng.choice(words, (20, 64)).astype(np.uint8)
+    lut = oref.build_lut(np.float32(0.02), I.ladder_pow3().numpy())
+    used, _, packed = oref.pack7(codes)
+    x = I.bits(I.x_normal(3, 64, 8))
+    assert np.array_equal(oref.linear_B7(packed, used, 20, 64, lut, x),
+                          oref.linear_B(codes, lut, x))
