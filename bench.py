@@ -561,6 +561,8 @@ class Layer(Workload):
         self.books = -(-n // lut_rows) if self.lut_rows else 1
         if self.fmt == "A":
             self.pkg = planes * n * (k // 64) * 15
+        elif self.fmt == "B7":
+            self.pkg = n * 14 * (k // 16) + 512
         else:
             self.pkg = n * k + 972 * self.books
         self.copies = max(1, -(-3 * L2_BYTES // self.pkg))
@@ -568,6 +570,10 @@ class Layer(Workload):
     def describe(self):
         what = (f"Format A {self.n}x{self.k}, G=64, {self.planes} plane(s), "
                 "quantized from bf16 0.02*StudentT(5)" if self.fmt == "A" else
+                f"7-bit alphabet {self.n}x{self.k}, codes uniform over 45 "
+                "seeded words of the 243, 7-bit indices into the used-code "
+                "table, ladder a_k=3^-(k-1), alpha=0.02, no rho"
+                if self.fmt == "B7" else
                 f"Format B {self.n}x{self.k}, codes uniform 0..242, ladder "
                 "a_k=3^-(k-1), alpha=0.02, no rho" if not self.lut_rows else
                 f"Format B {self.n}x{self.k}, codes uniform 0..242, adaptive "
@@ -593,6 +599,21 @@ class Layer(Workload):
             self.keep = [(c0.clone(), s0.clone()) for _ in range(self.copies)]
             self.w = [tq.weights_a(c, s, n, k, 64, self.planes)
                       for c, s in self.keep]
+        elif self.fmt == "B7":
+            lut = tq.tq_build_lut(I.ALPHA, I.ladder_pow3().numpy())
+            self.keep = []
+            for i in range(self.copies):
+                c = torch.from_numpy(self.codes45(n, k, 5 + i)).to(dev)
+                used = torch.empty(128, dtype=torch.uint8, device=dev)
+                cnt = torch.zeros(1, dtype=torch.int32, device=dev)
+                pk = torch.empty(n, 14 * (k // 16), dtype=torch.uint8,
+                                 device=dev)
+                tq.tq_pack7(c, used, cnt, pk)
+                l7 = torch.from_numpy(tq.tq_build_lut7(
+                    lut, used.cpu().numpy())).to(dev)
+                del c
+                self.keep.append((pk, l7))
+            self.w = [tq.weights_b7(pk, l7, n, k) for pk, l7 in self.keep]
         else:
             self.lut_d = torch.from_numpy(self.book_array(tq.tq_build_lut)).to(dev)
             self.keep = [I.codes_uniform(n, k, 5 + i, device=dev)
@@ -602,6 +623,13 @@ class Layer(Workload):
         self.x = {b: I.x_normal(b, k, 60 + b).to(dev) for b in self.BATCHES}
         self.y = {b: torch.zeros(b, n, device=dev) for b in self.BATCHES}
         self.pin_io(list(self.x.values()), list(self.y.values()))
+
+    @staticmethod
+    def codes45(n, k, seed):
+        """Codes uniform over 45 seeded words of the 243."""
+        rng = np.random.default_rng(seed)
+        words = rng.choice(243, 45, replace=False).astype(np.uint8)
+        return words[rng.integers(0, 45, (n, k))]
 
     def book_array(self, build):
         """The layer's code book, or one per block (seeded ladders)."""
@@ -631,6 +659,9 @@ class Layer(Workload):
         if self.fmt == "A":
             Wh = I.bits(I.student_t_bf16(rows, self.k, seed=3))
             self.pkg_h = oref.quantize_pack_A(Wh, 64, self.planes)
+        elif self.fmt == "B7":
+            self.lut_h = oref.build_lut(I.ALPHA, I.ladder_pow3().numpy())
+            self.b7_h = oref.pack7(self.codes45(rows, self.k, 5))
         else:
             self.codes_h = I.codes_uniform(rows, self.k, 5).numpy()
             self.lut_h = self.book_array(oref.build_lut)
@@ -641,7 +672,13 @@ class Layer(Workload):
         rows = max(0, min(rows, 256 - r0))
         jobs = []
         for b in self.BATCHES:
-            if self.fmt == "A":
+            if self.fmt == "B7":
+                used, _, pk = self.b7_h
+                pr = pk[r0:r0 + rows]
+                jobs.append((lambda b=b, pr=pr, used=used: self.oref.linear_B7(
+                    pr, used, len(pr), self.k, self.lut_h, self.xb[b]),
+                    rows * 14 * (self.k // 16)))
+            elif self.fmt == "A":
                 c, s = self.pkg_h
                 c, s = c[:, r0:r0 + rows], s[:, r0:r0 + rows]
                 jobs.append((lambda b=b, c=c, s=s: self.oref.linear_A(
@@ -1151,7 +1188,8 @@ def main():
     ap.add_argument("--batch", type=int, nargs="+", default=None,
                     help="batches of the decode_step and layer workloads "
                          "(default 1 4 16 64 and 1)")
-    ap.add_argument("--fmt", choices=["A", "B", "a", "b"], default="B",
+    ap.add_argument("--fmt", choices=["A", "B", "B7", "a", "b", "b7"],
+                    default="B",
                     help="layer workload: weight format")
     ap.add_argument("--n", type=int, default=8192, help="layer workload: rows")
     ap.add_argument("--k", type=int, default=5376,

@@ -35,6 +35,11 @@
  *                 p * scales_plane_stride elements; 0 = n*(k/G))
  *   B      codes  uint8  [n][k];  lut fp32 [256] (entries 243..255 NaN);
  *          rho    fp16   [ceil(n / rows_per_scale)] or NULL
+ *   B7     codes  uint8  [n][14 k / 16]: 7-bit indices, 16 per 14 bytes,
+ *                 little-endian (index j of a chunk at bits 7j .. 7j + 6);
+ *          lut    fp32   [128]: LUT7[i] = LUT[used[i]] (tq_build_lut7);
+ *          rho as B (alphaneural.io page, section 8.1, the 7-bit truncated
+ *          alphabet: a layer that uses at most 128 of the 243 words)
  *   x      bf16 [batch][ldx];  y fp32 [batch][ldy];  y = x * W_hat^T.
  *
  * Conventions:
@@ -84,7 +89,8 @@ typedef enum {
 
 typedef enum {
   TQ_FMT_A = 1, /* group ternary, 5 trits per byte, fp16 group scales */
-  TQ_FMT_B = 2  /* 243-entry ladder code book, one code per byte */
+  TQ_FMT_B = 2, /* 243-entry ladder code book, one code per byte */
+  TQ_FMT_B7 = 3 /* Format B over a used-code table: 7-bit indices */
 } tq_format;
 
 typedef struct {
@@ -99,7 +105,8 @@ typedef struct {
                               16-byte aligned. B: rho (fp16, 2-byte
                               aligned) or NULL */
   const float *lut;        /* B: device, 256 fp32 (tq_build_lut), 16-byte
-                              aligned. A: ignored */
+                              aligned. B7: device, 128 fp32 (tq_build_lut7),
+                              16-byte aligned. A: ignored */
   int64_t codes_plane_stride;  /* A: bytes between planes; 0 = dense */
   int64_t scales_plane_stride; /* A: elements between planes; 0 = dense */
   int64_t lut_rows;        /* B: 0 = one code book for every row; r > 0 =
@@ -248,6 +255,28 @@ tq_status tq_linear_experts(const tq_experts *w, const int32_t *ids,
                             int64_t n_tokens, const void *x_bf16, int64_t ldx,
                             float *y, int64_t ldy, int32_t *dev_status,
                             void *cuda_stream);
+
+/* 7-bit truncated alphabet (alphaneural.io page, section 8.1): turn Format B
+ * codes [n][k] (k % 16 == 0) into the layer's table of used codes and 7-bit
+ * indices into it.
+ *   codes        device uint8 [n][k], 16-byte aligned.
+ *   used_out     device uint8 [128], 16-byte aligned: the distinct codes in
+ *                ascending order, padded with 121 (the all-zero word); it
+ *                also holds the call's intermediate set of codes present.
+ *   n_used_out   device int32: the number of distinct codes.
+ *   packed_out   device uint8 [n][14 k / 16], 2-byte aligned.
+ *   dev_status   device int32 or NULL: TQ_ERR_RANGE when more than 128
+ *                codes are in use (the packed output is then unspecified).
+ * Three launches; no memory beyond the outputs. */
+tq_status tq_pack7(const uint8_t *codes, int64_t n, int64_t k,
+                   uint8_t *used_out, int32_t *n_used_out, uint8_t *packed_out,
+                   int32_t *dev_status, void *cuda_stream);
+
+/* The code book of a 7-bit layer on the host: lut7_out[i] = lut[used[i]]
+ * (128 entries; lut is the layer's 256-entry Format B book). Host pointers;
+ * no GPU needed. Errors: TQ_ERR_INVALID_ARG for NULL pointers. */
+tq_status tq_build_lut7(const float lut[256], const uint8_t used[128],
+                        float lut7_out[128]);
 
 /* Static description of a status value. */
 const char *tq_status_string(tq_status status);

@@ -56,6 +56,18 @@ tq_status check_weights(const tq_weights *w, tq::WeightsView *v) {
     // scales 16-byte aligned: kernels fetch them in aligned 16-byte chunks
     if (!aligned(w->codes, 16) || !aligned(w->scales, 16))
       return TQ_ERR_ALIGNMENT;
+  } else if (w->format == TQ_FMT_B7) {
+    // 7-bit indices into a used-code table, rows of 14 k / 16 bytes
+    if (w->planes != 1 || w->lut_rows != 0) return TQ_ERR_INVALID_ARG;
+    if (w->lut == nullptr) return TQ_ERR_INVALID_ARG;
+    if (w->rows_per_scale < 0) return TQ_ERR_INVALID_ARG;
+    if (w->rows_per_scale > 0 && w->scales == nullptr)
+      return TQ_ERR_INVALID_ARG;
+    if (w->k_cols % 16 != 0) return TQ_ERR_SHAPE;
+    if (!aligned(w->codes, 2) || !aligned(w->lut, 16)) return TQ_ERR_ALIGNMENT;
+    if (w->scales != nullptr && !aligned(w->scales, 2)) return TQ_ERR_ALIGNMENT;
+    v->group = 0;
+    if (w->rows_per_scale == 0) v->scales = nullptr;
   } else if (w->format == TQ_FMT_B) {
     if (w->planes != 1) return TQ_ERR_INVALID_ARG;
     if (w->lut == nullptr) return TQ_ERR_INVALID_ARG;
@@ -86,6 +98,10 @@ size_t tq_packed_bytes(int32_t format, int64_t n, int64_t k, int32_t group,
     return (size_t)planes * groups * ((size_t)tq::bytes_per_group(group) + 2);
   }
   if (format == TQ_FMT_B) return (size_t)n * (size_t)k + 243u * 4u;
+  if (format == TQ_FMT_B7) {
+    if (k % 16 != 0) return 0;
+    return (size_t)n * (size_t)(14 * (k / 16)) + 128u * 4u;
+  }
   return 0;
 }
 
@@ -182,6 +198,30 @@ tq_status tq_linear(const tq_weights *w, const void *x_bf16, int64_t batch,
   return from_cuda(tq::launch_linear(
       v, static_cast<const __nv_bfloat16 *>(x_bf16), batch, ldx, y, ldy,
       stream));
+}
+
+tq_status tq_pack7(const uint8_t *codes, int64_t n, int64_t k,
+                   uint8_t *used_out, int32_t *n_used_out, uint8_t *packed_out,
+                   int32_t *dev_status, void *cuda_stream) {
+  if (codes == nullptr || used_out == nullptr || n_used_out == nullptr ||
+      packed_out == nullptr || n < 0 || k < 0)
+    return TQ_ERR_INVALID_ARG;
+  if (k % 16 != 0) return TQ_ERR_SHAPE;
+  if (!aligned(codes, 16) || !aligned(used_out, 16) ||
+      !aligned(n_used_out, 4) || !aligned(packed_out, 2))
+    return TQ_ERR_ALIGNMENT;
+  if (dev_status != nullptr && !aligned(dev_status, 4)) return TQ_ERR_ALIGNMENT;
+  return from_cuda(tq::launch_pack7(codes, n, k, used_out, n_used_out,
+                                    packed_out, dev_status,
+                                    static_cast<cudaStream_t>(cuda_stream)));
+}
+
+tq_status tq_build_lut7(const float lut[256], const uint8_t used[128],
+                        float lut7_out[128]) {
+  if (lut == nullptr || used == nullptr || lut7_out == nullptr)
+    return TQ_ERR_INVALID_ARG;
+  for (int i = 0; i < 128; ++i) lut7_out[i] = lut[used[i]];
+  return TQ_OK;
 }
 
 tq_status tq_linear_experts(const tq_experts *w, const int32_t *ids,

@@ -36,6 +36,29 @@ struct WeightsView {
   int64_t lut_rows;             // B: rows per code book (0: one for all)
 };
 
+// 7-bit alphabet: the 16 indices of a 14-byte chunk (7 aligned 2-byte words,
+// index j at bits 7j .. 7j + 6, little-endian).
+__device__ __forceinline__ void unpack7_chunk(const uint16_t *__restrict__ p,
+                                              uint32_t (&idx)[16]) {
+  uint64_t lo = 0, hi = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) lo |= (uint64_t)__ldg(p + i) << (16 * i);
+#pragma unroll
+  for (int i = 0; i < 3; ++i) hi |= (uint64_t)__ldg(p + 4 + i) << (16 * i);
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const int pos = 7 * j;
+    uint64_t v;
+    if (pos + 7 <= 64)
+      v = lo >> pos;
+    else if (pos >= 64)
+      v = hi >> (pos - 64);
+    else
+      v = (lo >> pos) | (hi << (64 - pos));
+    idx[j] = (uint32_t)v & 0x7Fu;
+  }
+}
+
 // Expert-indexed Format A call (tq_linear_experts): token t uses expert
 // ids[t]; ids == nullptr marks a plain call.
 struct ExpertsView {

@@ -11,6 +11,8 @@ cudaError_t launch_linear(const WeightsView &w, const __nv_bfloat16 *x,
   const int force = g_test_force_path.load();
   if ((force == 2 || force == 3) && gemm_tc_supported(w, batch))
     return gemm_tc(w, x, batch, ldx, y, ldy, stream);
+  if (w.format == TQ_FMT_B7)  // 7-bit indices: the one-warp-per-row kernel
+    return linear_simple(w, x, batch, ldx, y, ldy, stream);
   if (w.format == TQ_FMT_B && w.lut_rows > 0) {
     // adaptive alphabet: the tensor-core kernel when every warp's 32 rows
     // share a code book (any batch), else the one-warp-per-row kernel

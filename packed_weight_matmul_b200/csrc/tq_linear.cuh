@@ -36,6 +36,10 @@ cudaError_t gemv_a(const WeightsView &w, const __nv_bfloat16 *x, float *y,
 cudaError_t gemv_a_experts(const WeightsView &w, const ExpertsView &E,
                            int64_t tokens, const __nv_bfloat16 *x, float *y,
                            cudaStream_t stream);
+// 7-bit truncated alphabet: used-code table and packed indices of codes.
+cudaError_t launch_pack7(const uint8_t *codes, int64_t n, int64_t k,
+                         uint8_t *used, int32_t *n_used, uint8_t *packed,
+                         int32_t *status, cudaStream_t stream);
 
 // Batches that are a real contraction: tcgen05 MMAs on decoded bf16 hi/lo
 // operands, accumulator in tensor memory.

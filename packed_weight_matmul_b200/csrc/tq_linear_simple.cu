@@ -75,6 +75,50 @@ __global__ void __launch_bounds__(kWarps * 32)
   }
 }
 
+// 7-bit alphabet: one warp per row, lane chunks of 16 indices (14 bytes);
+// weights LUT7[i] (times rho on the accumulator, as Format B).
+template <int BT>
+__global__ void __launch_bounds__(kWarps * 32)
+    linear_b7_simple(const uint16_t *__restrict__ packed, int64_t n, int64_t k,
+                     const float *__restrict__ lut7,
+                     const uint16_t *__restrict__ rho, int rps,
+                     const __nv_bfloat16 *__restrict__ x, int64_t ldx,
+                     float *__restrict__ y, int64_t ldy) {
+  __shared__ float sL[128];
+  if (threadIdx.x < 128) sL[threadIdx.x] = lut7[threadIdx.x];
+  __syncthreads();
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int64_t row = (int64_t)blockIdx.x * kWarps + warp;
+  if (row >= n) return;
+  float acc[BT];
+#pragma unroll
+  for (int b = 0; b < BT; ++b) acc[b] = 0.0f;
+  const int64_t cpr = k / 16;
+  const uint16_t *pr = packed + row * cpr * 7;
+  for (int64_t ch = lane; ch < cpr; ch += 32) {
+    uint32_t idx[16];
+    unpack7_chunk(pr + 7 * ch, idx);
+    float wv[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) wv[e] = sL[idx[e]];
+#pragma unroll
+    for (int b = 0; b < BT; ++b) {
+      const uint4 *xp = reinterpret_cast<const uint4 *>(x + b * ldx + 16 * ch);
+      float xv[16];
+      bf16x8_to_f32(xp[0], xv);
+      bf16x8_to_f32(xp[1], xv + 8);
+#pragma unroll
+      for (int e = 0; e < 16; ++e) acc[b] = fmaf(wv[e], xv[e], acc[b]);
+    }
+  }
+  const float r = rho ? __half2float(__ushort_as_half(rho[row / rps])) : 1.0f;
+#pragma unroll
+  for (int b = 0; b < BT; ++b) {
+    const float s = warp_sum(acc[b]);
+    if (lane == 0) y[b * ldy + row] = r * s;
+  }
+}
+
 template <int G, int PLANES, int BT>
 __global__ void __launch_bounds__(kWarps * 32)
     linear_a_simple(const uint8_t *__restrict__ codes,
@@ -150,6 +194,13 @@ cudaError_t launch_tile(const WeightsView &w, const __nv_bfloat16 *x,
                         int64_t ldx, float *y, int64_t ldy,
                         cudaStream_t stream) {
   if (w.format == TQ_FMT_B) return launch_b<BT>(w, x, ldx, y, ldy, stream);
+  if (w.format == TQ_FMT_B7) {
+    const unsigned blocks = (unsigned)((w.n + kWarps - 1) / kWarps);
+    linear_b7_simple<BT><<<blocks, kWarps * 32, 0, stream>>>(
+        reinterpret_cast<const uint16_t *>(w.codes), w.n, w.k, w.lut,
+        w.scales, w.rps, x, ldx, y, ldy);
+    return cudaGetLastError();
+  }
   if (w.group == 64)
     return w.planes == 1 ? launch_a<64, 1, BT>(w, x, ldx, y, ldy, stream)
                          : launch_a<64, 2, BT>(w, x, ldx, y, ldy, stream);

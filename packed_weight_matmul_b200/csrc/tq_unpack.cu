@@ -139,6 +139,39 @@ __global__ void __launch_bounds__(256)
   if (bad) report(status, TQ_ERR_BAD_CODE);
 }
 
+// 7-bit alphabet: one thread per 16 indices (14 bytes); index i decodes to
+// LUT7[i] = LUT[used[i]] (times rho), exactly Format B's weight.
+__global__ void __launch_bounds__(256)
+    unpack_b7_kernel(const uint16_t *__restrict__ packed, int64_t chunks,
+                     int64_t chunks_per_row, const float *__restrict__ lut7,
+                     const uint16_t *__restrict__ rho, int rps,
+                     uint16_t *__restrict__ out) {
+  __shared__ float sL[128];
+  if (threadIdx.x < 128) sL[threadIdx.x] = lut7[threadIdx.x];
+  __syncthreads();
+  for (int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c < chunks;
+       c += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = c / chunks_per_row;
+    const float r = rho ? __half2float(__ushort_as_half(rho[row / rps])) : 1.0f;
+    uint32_t idx[16];
+    unpack7_chunk(packed + 7 * c, idx);
+    uint32_t o[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      float v0 = sL[idx[2 * j]], v1 = sL[idx[2 * j + 1]];
+      if (rho) {
+        v0 = __fmul_rn(r, v0);
+        v1 = __fmul_rn(r, v1);
+      }
+      o[j] = __bfloat16_as_ushort(__float2bfloat16_rn(v0)) |
+             ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v1)) << 16);
+    }
+    uint4 *dst = reinterpret_cast<uint4 *>(out) + 2 * c;
+    __stcs(dst, make_uint4(o[0], o[1], o[2], o[3]));
+    __stcs(dst + 1, make_uint4(o[4], o[5], o[6], o[7]));
+  }
+}
+
 template <int G, int PLANES>
 cudaError_t launch_a(const WeightsView &w, uint16_t *out, int32_t *status,
                      cudaStream_t stream) {
@@ -167,6 +200,12 @@ cudaError_t launch_unpack(const WeightsView &w, uint16_t *out,
   const int64_t chunks = w.n * (w.k / 16);
   const int64_t want = (chunks + 255) / 256;
   const int blocks = (int)(want < (int64_t)sms * 8 ? want : (int64_t)sms * 8);
+  if (w.format == TQ_FMT_B7) {
+    unpack_b7_kernel<<<blocks, 256, 0, stream>>>(
+        reinterpret_cast<const uint16_t *>(w.codes), chunks, w.k / 16, w.lut,
+        w.scales, w.rps, out);
+    return cudaGetLastError();
+  }
   unpack_b_kernel<<<blocks, 256, 0, stream>>>(
       w.codes, w.n, w.k, w.lut, w.lut_rows, w.scales, w.rps, out, status);
   return cudaGetLastError();

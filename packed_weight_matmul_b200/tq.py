@@ -19,14 +19,15 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)),
 TQ_OK, TQ_ERR_INVALID_ARG, TQ_ERR_SHAPE, TQ_ERR_ALIGNMENT = 0, 1, 2, 3
 TQ_ERR_UNSUPPORTED, TQ_ERR_BAD_CODE, TQ_ERR_NONFINITE = 4, 5, 6
 TQ_ERR_RANGE, TQ_ERR_TIMEOUT, TQ_ERR_CUDA = 7, 8, 9
-TQ_FMT_A, TQ_FMT_B = 1, 2
+TQ_FMT_A, TQ_FMT_B, TQ_FMT_B7 = 1, 2, 3
 
 # Every entry point declared in include/tq.h.
 ENTRY_POINTS = ("tq_packed_bytes", "tq_build_lut", "tq_quantize_pack",
                 "tq_unpack", "tq_linear", "tq_status_string",
                 "tq_encode_b", "tq_testing_linear_wait_fault",
                 "tq_testing_force_linear_path", "tq_testing_tc_self_check",
-                "tq_testing_tc_trace", "tq_linear_experts")
+                "tq_testing_tc_trace", "tq_linear_experts", "tq_pack7",
+                "tq_build_lut7")
 
 
 class TqError(RuntimeError):
@@ -83,6 +84,10 @@ def _load():
     L.tq_testing_tc_self_check.argtypes = [i32, P, i32]
     L.tq_testing_tc_trace.restype = C.c_int
     L.tq_testing_tc_trace.argtypes = [P]
+    L.tq_pack7.restype = C.c_int
+    L.tq_pack7.argtypes = [P, i64, i64, P, P, P, P, P]
+    L.tq_build_lut7.restype = C.c_int
+    L.tq_build_lut7.argtypes = [P, P, P]
     L.tq_linear_experts.restype = C.c_int
     L.tq_linear_experts.argtypes = [C.POINTER(tq_experts), P, i64, P, i64, P,
                                     i64, P, P]
@@ -133,6 +138,28 @@ def tq_build_lut(alpha: float, ladder) -> np.ndarray:
                              lad.ctypes.data_as(C.c_void_p),
                              out.ctypes.data_as(C.c_void_p)), "tq_build_lut")
     return out
+
+
+def tq_build_lut7(lut, used) -> np.ndarray:
+    """Host: LUT7[i] = lut[used[i]] for a 7-bit layer (128 entries)."""
+    lut = np.ascontiguousarray(np.asarray(lut, np.float32))
+    used = np.ascontiguousarray(np.asarray(used, np.uint8))
+    assert lut.shape == (256,) and used.shape == (128,)
+    out = np.zeros(128, np.float32)
+    _check(_lib.tq_build_lut7(lut.ctypes.data_as(C.c_void_p),
+                              used.ctypes.data_as(C.c_void_p),
+                              out.ctypes.data_as(C.c_void_p)), "tq_build_lut7")
+    return out
+
+
+def tq_pack7(codes, used_out, n_used_out, packed_out, dev_status=None,
+             stream=None, check=True):
+    n, k = codes.shape
+    st = _lib.tq_pack7(_ptr(codes), n, k, _ptr(used_out), _ptr(n_used_out),
+                       _ptr(packed_out), _ptr(dev_status), _stream(stream))
+    if check:
+        _check(st, "tq_pack7")
+    return st
 
 
 def tq_linear_experts(w: "Experts", ids, x, y, n_tokens=None, ldx=None,
@@ -244,6 +271,16 @@ def experts_a(codes, scales, n_experts, n, k, n_hot=0, codes2=None,
                    n_rows=n, k_cols=k, codes=_ptr(codes), scales=_ptr(scales),
                    codes2=_ptr(codes2), scales2=_ptr(scales2))
     return Experts(d, (codes, scales, codes2, scales2))
+
+
+def weights_b7(packed, lut7, n, k, rho=None, rows_per_scale=0) -> Weights:
+    """7-bit layer: packed indices [n][14 k / 16] and LUT7 [128]."""
+    d = tq_weights(format=TQ_FMT_B7, group=0, planes=1,
+                   rows_per_scale=rows_per_scale if rho is not None else 0,
+                   n_rows=n, k_cols=k, codes=_ptr(packed), scales=_ptr(rho),
+                   lut=_ptr(lut7), codes_plane_stride=0, scales_plane_stride=0,
+                   lut_rows=0)
+    return Weights(d, (packed, lut7, rho))
 
 
 def weights_b(codes, lut, rho=None, rows_per_scale=0, n=None, k=None,

@@ -194,3 +194,28 @@ def test_lut_rows_validation(tq):
     assert _linear(tq, _wa(tq, lut_rows=32)) == E.TQ_ERR_INVALID_ARG
     # a zero-row call with per-block books is valid and launches nothing
     assert _linear(tq, _wb(tq, n_rows=0, lut_rows=32), ldy=0) == E.TQ_OK
+
+
+def test_pack7_and_b7_validation(tq):
+    """tq_pack7 and 7-bit weights: bad arguments are rejected on the host
+    (fake addresses, no GPU touched); the host book builder gathers."""
+    E, L = tq, tq.lib()
+    assert L.tq_pack7(None, 4, 32, 0x20000, 0x30000, 0x40000, None,
+                      None) == E.TQ_ERR_INVALID_ARG
+    assert L.tq_pack7(0x10000, 4, 24, 0x20000, 0x30000, 0x40000, None,
+                      None) == E.TQ_ERR_SHAPE
+    assert L.tq_pack7(0x10008, 4, 32, 0x20000, 0x30000, 0x40000, None,
+                      None) == E.TQ_ERR_ALIGNMENT
+    assert L.tq_pack7(0x10000, 4, 32, 0x20004, 0x30000, 0x40000, None,
+                      None) == E.TQ_ERR_ALIGNMENT
+    assert L.tq_pack7(0x10000, 4, 32, 0x20000, 0x30000, 0x40001, None,
+                      None) == E.TQ_ERR_ALIGNMENT
+    b7 = dict(format=tq.TQ_FMT_B7)
+    assert _linear(tq, _wb(tq, **b7, lut_rows=32)) == E.TQ_ERR_INVALID_ARG
+    assert _linear(tq, _wb(tq, **b7, k_cols=24)) == E.TQ_ERR_SHAPE
+    assert _linear(tq, _wb(tq, **b7, codes=0x10001)) == E.TQ_ERR_ALIGNMENT
+    assert _linear(tq, _wb(tq, **b7, lut=0x30008)) == E.TQ_ERR_ALIGNMENT
+    assert tq.tq_packed_bytes(tq.TQ_FMT_B7, 3, 32) == 3 * 28 + 512
+    lut = np.arange(256, dtype=np.float32)
+    used = np.arange(128, dtype=np.uint8)[::-1].copy()
+    assert np.array_equal(tq.tq_build_lut7(lut, used), lut[used])
