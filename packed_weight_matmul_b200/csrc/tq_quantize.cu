@@ -101,54 +101,58 @@ __global__ void __launch_bounds__(kGroupsPerBlock)
     const uint32_t thr1 =
         (s1 & 0x7FFFu) == 0 ? 0xFFFFu : (__float_as_uint(s1f * 0.5f) >> 16);
 
-    // ---- plane 1: trits -> digits -> bytes ----
-#pragma unroll 1
-    for (int m = 0; m < NB; ++m) {
-      uint32_t b = 0;
+    // ---- plane 1: trits -> bytes ----
+    // A byte of digits d = t + 1 is sum d_i 3^i = 121 + sum t_i 3^i: start
+    // from 121 (all trits 0, also the padding) and add +-3^i per non-zero
+    // trit. Every index is a compile-time constant (full unroll).
 #pragma unroll
-      for (int i = 4; i >= 0; --i) {
+    for (int m = 0; m < NB; ++m) {
+      int b = 121;
+#pragma unroll
+      for (int i = 0; i < 5; ++i) {
         const int j = 5 * m + i;
-        uint32_t d = 1;  // padding digit = trit 0
         if (j < G) {
           const uint32_t v = bf16_at<G>(gw, j);
-          d = ((v & 0x7FFFu) > thr1) ? ((v & 0x8000u) ? 0u : 2u) : 1u;
+          constexpr int kP3[5] = {1, 3, 9, 27, 81};
+          if ((v & 0x7FFFu) > thr1) b += (v & 0x8000u) ? -kP3[i] : kP3[i];
         }
-        b = b * 3 + d;
       }
       sC[0][t * NB + m] = (uint8_t)b;
     }
 
     if constexpr (PLANES == 2) {
-      // ---- plane 2: the same rule on R = fp32_RN(W - s1 t1) ----
-      auto residual = [&](int j) -> float {
+      // ---- plane 2: the same rule on R = fp32_RN(W - s1 t1), computed once
+      uint32_t rbits[G];
+#pragma unroll
+      for (int j = 0; j < G; ++j) {
         const uint32_t v = bf16_at<G>(gw, j);
         const float wf = __uint_as_float(v << 16);
-        if ((v & 0x7FFFu) <= thr1) return wf;  // t1 = 0
-        return __fsub_rn(wf, (v & 0x8000u) ? -s1f : s1f);
-      };
+        rbits[j] = (v & 0x7FFFu) <= thr1
+                       ? __float_as_uint(wf)  // t1 = 0
+                       : __float_as_uint(
+                             __fsub_rn(wf, (v & 0x8000u) ? -s1f : s1f));
+      }
       double sum2 = 0.0;
-#pragma unroll 4
+#pragma unroll
       for (int j = 0; j < G; ++j)
-        sum2 += scaled_f64_from_f32_mag(__float_as_uint(residual(j)) &
-                                        0x7FFFFFFFu);
+        sum2 += scaled_f64_from_f32_mag(rbits[j] & 0x7FFFFFFFu);
       const uint16_t s2 = scale_from_sum<G>(sum2, status);
       scales[total_groups + g0 + t] = s2;
       const float s2f = __half2float(__ushort_as_half(s2));
       const uint32_t thr2 =
           (s2 & 0x7FFFu) == 0 ? 0xFFFFFFFFu : __float_as_uint(s2f * 0.5f);
-#pragma unroll 1
-      for (int m = 0; m < NB; ++m) {
-        uint32_t b = 0;
 #pragma unroll
-        for (int i = 4; i >= 0; --i) {
+      for (int m = 0; m < NB; ++m) {
+        int b = 121;
+#pragma unroll
+        for (int i = 0; i < 5; ++i) {
           const int j = 5 * m + i;
-          uint32_t d = 1;
           if (j < G) {
-            const uint32_t r = __float_as_uint(residual(j));
-            d = ((r & 0x7FFFFFFFu) > thr2) ? ((r & 0x80000000u) ? 0u : 2u)
-                                           : 1u;
+            constexpr int kP3[5] = {1, 3, 9, 27, 81};
+            const uint32_t r = rbits[j];
+            if ((r & 0x7FFFFFFFu) > thr2)
+              b += (r & 0x80000000u) ? -kP3[i] : kP3[i];
           }
-          b = b * 3 + d;
         }
         sC[PLANES - 1][t * NB + m] = (uint8_t)b;
       }
