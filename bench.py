@@ -913,7 +913,7 @@ def make_workload(args):
         return DecodeStep(batches=batches or I.DECODE_BATCHES)
     if args.workload == "layer":
         return Layer(args.fmt, args.n, args.k, batches or (1,), args.planes,
-                     args.lut_rows)
+                     getattr(args, "lut_rows", 0))
     return WORKLOADS[args.workload]()
 
 

@@ -96,8 +96,9 @@ constexpr uint32_t kAStage0 = 2 * kAccCols;
 constexpr uint32_t kAStageCols = 128;    // 64 hi + 64 lo columns
 constexpr int kDecWarps = 8;
 constexpr int kWarpCodes = 0, kWarpX = 1, kWarpMma = 2, kWarpEpi = 3,
-              kWarpDec = 7;
-constexpr int kThreads = 32 * (kWarpDec + kDecWarps);  // 480
+              kWarpDec = 7, kWarpWait = kWarpDec + kDecWarps;
+constexpr int kThreads = 32 * (kWarpWait + 1);  // 512
+constexpr int kBarIdStage = 1;  // named barrier: waiter -> MMA issuer
 constexpr int kMaxCodeStages = 8;
 constexpr int kMaxXStages = 4;
 constexpr uint32_t kBRow = 128;          // Format B row: 128 codes, swizzled
@@ -133,6 +134,19 @@ struct TcPlan {
   int grid_ok;  // Format B: the single-operand code-book path may be used
   size_t smem;
 };
+
+// Named-barrier reduction over `count` threads (whole warps): true when the
+// predicate holds in every participating thread. No shared-memory access.
+__device__ __forceinline__ bool bar_red_and(int id, int count, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n"
+      " barrier.red.and.pred q, %2, %3, p;\n selp.u32 %0, 1, 0, q;\n}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
+}
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t s) {
   return __byte_perm(a, b, s);
@@ -672,33 +686,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kWarpMma) {
     // ---- MMA issuer ---------------------------------------------------------
-    if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(kTileM, n_pad);
-      const uint32_t xhalf = (uint32_t)n_pad * 128u;  // k 64..127 of the tile
-      int xs = 0, ux = 0, as = 0, ua = 0;
-      int ca = 0;  // accumulator commits
-      bool ok = true;
-      int i = 0;
-      for (int t = cid; ok && t < P.tiles; t += nclusters, ++i) {
-        const int buf = i & 1;
-        if (i >= 2 && !mbar_wait(B0 + kBarAccEmpty + 8 * buf,
-                                 (uint32_t)((i >> 1) + 1) & 1u, abort_addr,
-                                 lim)) {
-          if constexpr (CK) ck_record(23, (uint64_t)i);
-          ok = false;
-          break;
-        }
-        tc_fence_after_sync();
-        const uint32_t d = tmem + (uint32_t)buf * kAccCols;
-        for (int it = it0; it < it1; ++it) {
-          if (!mbar_wait(B0 + kBarXFull + 8 * xs,
-                         (uint32_t)(ux / P.x_stages) & 1u, abort_addr, lim) ||
-              !mbar_wait(B0 + kBarAFull + 8 * as,
-                         (uint32_t)(ua / kAStages) & 1u, abort_addr, lim)) {
-            if constexpr (CK) ck_record(24, (uint64_t)ux << 32 | (uint32_t)ua);
-            ok = false;
-            break;
-          }
+    // The whole warp follows the stages; lane 0 issues. The issuer touches
+    // no shared memory while stages flow: the first shared-memory access
+    // after a run of tcgen05.mma stalls until those MMAs complete, so the
+    // waits on the input barriers belong to the waiter warp, which hands
+    // each stage over through a named-barrier reduction (its vote says
+    // whether the inputs arrived or a wait gave up).
+    const uint32_t idesc = idesc_bf16_f32(kTileM, n_pad);
+    const uint32_t xhalf = (uint32_t)n_pad * 128u;  // k 64..127 of the tile
+    int xs = 0, ux = 0, as = 0, ua = 0;
+    int ca = 0;  // accumulator commits
+    bool ok = true;
+    int i = 0;
+    for (int t = cid; ok && t < P.tiles; t += nclusters, ++i) {
+      const int buf = i & 1;
+      const uint32_t d = tmem + (uint32_t)buf * kAccCols;
+      for (int it = it0; it < it1; ++it) {
+        ok = bar_red_and(kBarIdStage, 64, true);
+        if (!ok) break;
+        if (lane == 0) {
           tc_fence_after_sync();
           ck_trace<CK>(trace, 2, t, it, 1);
           const uint32_t xb = x_ring + (uint32_t)xs * P.x_stage_bytes;
@@ -720,23 +726,29 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           mma_commit(B0 + kBarXEmpty + 8 * xs);
           mma_commit(B0 + kBarAEmpty + 8 * as);
-          ++ux;
-          xs = xs + 1 == P.x_stages ? 0 : xs + 1;
-          ++ua;
-          as = as + 1 == kAStages ? 0 : as + 1;
         }
-        if (!ok) break;
+        __syncwarp();
+        ++ux;
+        xs = xs + 1 == P.x_stages ? 0 : xs + 1;
+        ++ua;
+        as = as + 1 == kAStages ? 0 : as + 1;
+      }
+      if (!ok) break;
+      if (lane == 0) {
         ck_trace<CK>(trace, 2, t, 0, 2);
         mma_commit(B0 + kBarAccFull + 8 * buf);
-        ++ca;
         ck_trace<CK>(trace, 2, t, 0, 3);
       }
-      // The arrives of tcgen05.commit land asynchronously, when the MMAs
-      // finish: before the CTA may leave (and its shared memory go to the
-      // next CTA), every arrive this thread caused must have landed. The
-      // drain commit covers every issued MMA; the last commit to each x and
-      // A stage is then observed on its own barrier (those barriers complete
-      // only through these commits). Bounded waits, also after a time-out.
+      __syncwarp();
+      ++ca;
+    }
+    // The arrives of tcgen05.commit land asynchronously, when the MMAs
+    // finish: before the CTA may leave (and its shared memory go to the
+    // next CTA), every arrive this thread caused must have landed. The
+    // drain commit covers every issued MMA; the last commit to each x and
+    // A stage is then observed on its own barrier (those barriers complete
+    // only through these commits). Bounded waits, also after a time-out.
+    if (lane == 0) {
       mma_commit(B0 + kBarDrain);
       mbar_wait(B0 + kBarDrain, 0u);
       for (int j = ux > P.x_stages ? ux - P.x_stages : 0; j < ux; ++j)
@@ -747,6 +759,41 @@ __global__ void __launch_bounds__(kThreads, 1)
                   (uint32_t)(j / kAStages) & 1u);
       for (int j = ca > 2 ? ca - 2 : 0; j < ca; ++j)
         mbar_wait(B0 + kBarAccFull + 8 * (j & 1), (uint32_t)(j >> 1) & 1u);
+    }
+    __syncwarp();
+  } else if (warp == kWarpWait) {
+    // ---- waiter: the MMA issuer's input barriers ----------------------------
+    // Per stage: the accumulator buffer is free (first stage of a tile, from
+    // the third tile on), the x stage and the A stage are full; then one
+    // named-barrier reduction with the issuer carries the verdict. Both
+    // sides stop at the first failed stage, so they take the same number of
+    // reductions.
+    int xs = 0, ux = 0, as = 0, ua = 0;
+    bool ok = true;
+    int i = 0;
+    for (int t = cid; ok && t < P.tiles; t += nclusters, ++i) {
+      const int buf = i & 1;
+      bool acc_ok = true;
+      if (i >= 2)
+        acc_ok = mbar_wait(B0 + kBarAccEmpty + 8 * buf,
+                           (uint32_t)((i >> 1) + 1) & 1u, abort_addr, lim);
+      if constexpr (CK) if (!acc_ok && lane == 0) ck_record(23, (uint64_t)i);
+      for (int it = it0; it < it1; ++it) {
+        bool got = acc_ok &&
+                   mbar_wait(B0 + kBarXFull + 8 * xs,
+                             (uint32_t)(ux / P.x_stages) & 1u, abort_addr,
+                             lim) &&
+                   mbar_wait(B0 + kBarAFull + 8 * as,
+                             (uint32_t)(ua / kAStages) & 1u, abort_addr, lim);
+        got = __all_sync(0xFFFFFFFFu, got);
+        if constexpr (CK) if (!got && lane == 0) ck_record(24, (uint64_t)ux << 32 | (uint32_t)ua);
+        ok = bar_red_and(kBarIdStage, 64, got);
+        if (!ok) break;
+        ++ux;
+        xs = xs + 1 == P.x_stages ? 0 : xs + 1;
+        ++ua;
+        as = as + 1 == kAStages ? 0 : as + 1;
+      }
     }
   } else if (warp < kWarpDec) {
     // ---- epilogue -----------------------------------------------------------
@@ -820,7 +867,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (c < n_pad) part[c * kTileM + r] = __uint_as_float(v[c]);
       }
     }
-  } else {
+  } else if (warp < kWarpDec + kDecWarps) {
     // ---- decoders -----------------------------------------------------------
     const int q = warp & 3;
     const int kp = (warp - kWarpDec) >> 2;  // which 64-k half of the block
