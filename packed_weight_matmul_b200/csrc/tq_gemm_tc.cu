@@ -4,7 +4,9 @@
 //             (precisit.com page, "Three values and a shared scale"; second
 //             plane per the FUCINA README, "The method")
 //   Format B: y[b][n] = rho[n / rps] * sum_k LUT[code[n][k]] x[b][k]
-//             (alphaneural.io page, sections 3.2, 3.3 and 4.2)
+//             (alphaneural.io page, sections 3.2, 3.3 and 4.2), also with
+//             one code book per block of rows (section 8.3) and with 7-bit
+//             indices into the layer's used words (section 8.1)
 //
 // Warp-specialised, one CTA per SM (it holds the whole tensor memory).
 // Without a split of K the CTAs are persistent and walk the 128-row tiles of
@@ -12,7 +14,7 @@
 // tile, each CTA a slice of K. For each 128-wide k block ("iteration"):
 //   - the code producer warp copies the tile's codes into a shared-memory
 //     ring with tensor copies (TMA): Format B one 128-row x 128-code box
-//     per block; Format A one box of codes and one of fp16 scales per window
+//     per block (7-bit indices: 128 rows x 112 bytes); Format A one box of codes and one of fp16 scales per window
 //     of 4 blocks = 8 groups of 13 bytes, from the 16-byte boundary at or
 //     below the window (when rows start on 16-byte boundaries; otherwise one
 //     1-D bulk copy of each row's aligned run). Code boxes use the 128-byte
@@ -28,11 +30,16 @@
 //     into tensor memory (tcgen05.st): A never passes through shared memory.
 //     Each weight w is split into w_hi = bf16(w) and w_lo = bf16(w - w_hi),
 //     so the two MMAs (hi, lo) carry 16 significant bits of w: exact for
-//     Format A (an fp16 scale has 11), relative error <= 2^-17 for Format B;
-//   - one thread issues the 16 MMAs (M = 128, N, K = 16, A from tensor
-//     memory, B from shared memory) and commits them to the barriers that
-//     free the x stage and the A stage, and after the tile's last block to
-//     the accumulator barrier;
+//     Format A (an fp16 scale has 11), relative error <= 2^-17 for Format B.
+//     A Format B book whose entries all lie on one integer grid takes one
+//     exact operand, bf16(m), instead (see the set-up below);
+//   - a waiter warp takes the waits for the x stage, the A stage and the
+//     free accumulator and hands each ready stage to the MMA warp through a
+//     named-barrier reduction, so the issuing thread only issues;
+//   - one thread issues the 16 (or 8) MMAs (M = 128, N, K = 16, A from
+//     tensor memory, B from shared memory) and commits them to the barriers
+//     that free the x stage and the A stage, and after the tile's last block
+//     to the accumulator barrier;
 //   - 4 epilogue warps read the accumulator (double-buffered in tensor
 //     memory, so the next tile's MMAs proceed meanwhile) and store y, or,
 //     with a split, keep the partial tile in shared memory; after a cluster
@@ -44,7 +51,10 @@
 // lane's base word is the complete lookup address and a warp's lookups hit
 // distinct banks:
 //   Format B: entry c of lane l at tab + 256 c + 4 l holds bf16 hi | lo << 16
-//             of LUT[c];
+//             of LUT[c] (or bf16(m) on the grid); 7-bit indices use entries
+//             0..127, the index moved to bits 8..14 of the lane's base word;
+//             with a book per block of rows, each decoder warp keeps its
+//             rows' book unreplicated (1 KB) instead;
 //   Format A: entry b of lane l at tab + 256 b + 8 l holds, for the 5 trits
 //             of code byte b, "selector bytes" 0x10 + 0x22 d (d = t + 1):
 //             trits 0..3 in the first word, trits 2..4 in the second. Four
@@ -62,6 +72,7 @@
 
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "tq_common.cuh"
 #include "tq_linear.cuh"
@@ -102,6 +113,7 @@ constexpr int kBarIdStage = 1;  // named barrier: waiter -> MMA issuer
 constexpr int kMaxCodeStages = 8;
 constexpr int kMaxXStages = 4;
 constexpr uint32_t kBRow = 128;          // Format B row: 128 codes, swizzled
+constexpr uint32_t kB7Row = 112;         // 7-bit alphabet row: 128 indices
 constexpr int kAWin = 4;                 // Format A window: 4 blocks, 8 groups
 constexpr uint32_t kARowCodes = 128;     // 104 code bytes + <= 15 skew
 constexpr uint32_t kARow = 160;          // per-row copies: + 16 scale bytes
@@ -269,6 +281,52 @@ __device__ __forceinline__ void decode_b_compact(const uint32_t (&cw)[16],
     hi[2 * j + 1] = prmt(v2, v3, 0x5410u);
     lo[2 * j + 1] = prmt(v2, v3, 0x7632u);
   }
+}
+
+// 7-bit alphabet: table address of index J of a run of 64 7-bit indices
+// (little-endian bit string d, index J at bits 7J .. 7J + 6). The index
+// lands at bits 8..14, the entry pitch of the lane-replicated table.
+template <int J>
+__device__ __forceinline__ uint32_t b7_addr(const uint32_t (&d)[14],
+                                            uint32_t lane_tab) {
+  constexpr int bit = 7 * J, wd = bit >> 5, s = bit & 31;
+  uint32_t v;
+  if constexpr (s < 8)
+    v = d[wd] << (8 - s);
+  else if constexpr (s <= 25 || wd + 1 >= 14)
+    v = d[wd] >> (s - 8);
+  else
+    v = __funnelshift_r(d[wd], d[wd + 1], s - 8);
+  return (v & 0x7F00u) | lane_tab;
+}
+
+template <int J, bool LO>
+__device__ __forceinline__ void decode_b7_pair(const uint32_t (&d)[14],
+                                               uint32_t lane_tab,
+                                               uint32_t (&hi)[32],
+                                               uint32_t (&lo)[32]) {
+  const uint32_t v0 = lut32(b7_addr<2 * J>(d, lane_tab));
+  const uint32_t v1 = lut32(b7_addr<2 * J + 1>(d, lane_tab));
+  hi[J] = prmt(v0, v1, 0x5410u);
+  if constexpr (LO) lo[J] = prmt(v0, v1, 0x7632u);
+}
+
+template <bool LO, int... J>
+__device__ __forceinline__ void decode_b7_all(const uint32_t (&d)[14],
+                                              uint32_t lane_tab,
+                                              uint32_t (&hi)[32],
+                                              uint32_t (&lo)[32],
+                                              std::integer_sequence<int, J...>) {
+  (decode_b7_pair<J, LO>(d, lane_tab, hi, lo), ...);
+}
+
+// 7-bit alphabet: 64 indices of one row (56 bytes) -> 32 hi (and lo) bf16
+// pairs through the lane-replicated table of the 128 used words.
+template <bool LO>
+__device__ __forceinline__ void decode_b7(const uint32_t (&d)[14],
+                                          uint32_t lane_tab, uint32_t (&hi)[32],
+                                          uint32_t (&lo)[32]) {
+  decode_b7_all<LO>(d, lane_tab, hi, lo, std::make_integer_sequence<int, 32>{});
 }
 
 // Format A: one group (13 code bytes, realigned into b[0..3]) -> 32 hi and
@@ -495,10 +553,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   // adaptive alphabet: every decoder warp builds its rows' compact book per
   // tile in the table region; no shared table, no single-operand path
   const bool adaptive = FMT == TQ_FMT_B && w.lut_rows > 0;
+  // 7-bit alphabet: 7-bit indices into a book of the 128 used words
+  const bool b7 = FMT == TQ_FMT_B && w.format == TQ_FMT_B7;
+  const int n_words = b7 ? 128 : 243;
   if (FMT == TQ_FMT_B && !adaptive) {
     __syncthreads();  // the unit word is initialised
     float lv = 0.0f;
-    if (threadIdx.x < 243) {
+    if ((int)threadIdx.x < n_words) {
       lv = __ldg(w.lut + threadIdx.x);
       const float a = fabsf(lv);
       if (a > 0.0f && a <= 3.4028235e38f)
@@ -507,7 +568,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     const float u = __int_as_float(ld_volatile_s32(B0 + kUnit));
     bool ok = true;
-    if (threadIdx.x < 243) {
+    if ((int)threadIdx.x < n_words) {
       const float m = rintf(__fdiv_rn(lv, u));
       ok = u <= 3.4028235e38f && fabsf(m) <= 256.0f &&
            fabs((double)lv - (double)u * (double)m) <=
@@ -520,11 +581,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (FMT == TQ_FMT_B && !adaptive) {
     for (int i = threadIdx.x; i < 256 * 8; i += blockDim.x) {
       const int e = i >> 3, j = i & 7;
-      const float v = __ldg(w.lut + e);
+      // entries past the book (7-bit alphabet: 128 words) are never read
+      const float v = !b7 || e < 128 ? __ldg(w.lut + e)
+                                     : __int_as_float(0x7FC00000);
       uint32_t word;
       if (grid) {
-        // bf16(m) in the low half; entries 243..255 stay NaN
-        word = e < 243 ? bf16_bits_rn(rintf(__fdiv_rn(v, unit))) : 0x7FC0u;
+        // bf16(m) in the low half; entries past the words stay NaN
+        word = e < n_words ? bf16_bits_rn(rintf(__fdiv_rn(v, unit))) : 0x7FC0u;
       } else {
         const uint32_t h = bf16_bits_rn(v);
         const uint32_t l = bf16_bits_rn(v - __uint_as_float(h << 16));
@@ -570,12 +633,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if constexpr (FMT == TQ_FMT_B) {
           // one box of 128 rows x 128 codes, 128-byte swizzle (16-byte chunk
           // c of row r lands at chunk c ^ (r & 7)); rows past N and codes
-          // past K read as zero, and the decoders mask them
+          // past K read as zero, and the decoders mask them. 7-bit alphabet:
+          // 128 rows x 112 bytes (128 indices), not swizzled
           if (lane == 0) {
+            const uint32_t bytes = kTileM * (b7 ? kB7Row : kBRow);
             uint32_t d = dst0;
-            if constexpr (CK) d = ck_smem<CK>(W, d, kTileM * kBRow, 2);
-            mbar_arrive_expect_tx(full, kTileM * kBRow);
-            tma_load_2d(d, &tmap_c, ws * kKB, (int)row0, full);
+            if constexpr (CK) d = ck_smem<CK>(W, d, bytes, 2);
+            mbar_arrive_expect_tx(full, bytes);
+            tma_load_2d(d, &tmap_c, ws * (b7 ? kB7Row : kKB), (int)row0, full);
           }
           __syncwarp();
         } else if (P.a_map) {
@@ -910,11 +975,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         // this row's codes (crow) and scales (srow) in the stage; a row
         // written by a tensor copy is swizzled: logical byte o is at o ^ sw
-        const bool swz = FMT == TQ_FMT_B || P.a_map;
+        const bool swz = (FMT == TQ_FMT_B && !b7) || P.a_map;
         const uint32_t sw = swz ? (uint32_t)(r & 7) << 4 : 0u;
         const uint32_t crow =
-            code_stage(cs) + (uint32_t)r * (FMT == TQ_FMT_B ? kBRow
-                                            : swz ? kARowCodes : kARow);
+            code_stage(cs) +
+            (uint32_t)r * (FMT == TQ_FMT_B ? (b7 ? kB7Row : kBRow)
+                           : swz           ? kARowCodes
+                                           : kARow);
         const uint32_t srow = swz ? code_stage(cs) + kAMapScales +
                                         (uint32_t)r * kAMapSRow
                                   : crow + kARowCodes;
@@ -953,23 +1020,36 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0 && q == 0 && kp == 0) ck_trace<CK>(trace, 5, t, it, 1);
           uint32_t hi[32], lo[32];
           if constexpr (FMT == TQ_FMT_B) {
+            // this half's 64 codes: four 16-byte loads. 7-bit alphabet: 56
+            // bytes, loaded from byte 0 (kp 0) or 48 (kp 1, the run starting
+            // 8 bytes in); its row pitch, 112, puts a quarter warp's 8 rows
+            // on 8 distinct 16-byte bank groups
+            const uint32_t hoff = (b7 ? 48u : 64u) * (uint32_t)kp;
             uint32_t cw[16];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              const uint32_t a =
-                  crow + ((64u * (uint32_t)kp + 16u * (uint32_t)j) ^ sw);
+              const uint32_t a = crow + ((hoff + 16u * (uint32_t)j) ^ sw);
               const uint4 v4 = lds128(ck_smem<CK>(W, a, 16u, 16));
               cw[4 * j] = v4.x;
               cw[4 * j + 1] = v4.y;
               cw[4 * j + 2] = v4.z;
               cw[4 * j + 3] = v4.w;
             }
-            if (adaptive)
+            if (b7) {
+              uint32_t d[14];
+#pragma unroll
+              for (int i = 0; i < 14; ++i) d[i] = kp ? cw[i + 2] : cw[i];
+              if (grid)
+                decode_b7<false>(d, lane_tab, hi, lo);
+              else
+                decode_b7<true>(d, lane_tab, hi, lo);
+            } else if (adaptive) {
               decode_b_compact(cw, ctab, hi, lo);
-            else if (grid)
+            } else if (grid) {
               decode_b_hi(cw, lane_tab, hi);
-            else
+            } else {
               decode_b(cw, lane_tab, hi, lo);
+            }
             // k past K (in the last block) and rows past N: zero weights
             // (selects, no branch: the tcgen05.st below is warp-wide)
             const int64_t kv = K - ((int64_t)it * kKB + 64 * kp);
@@ -1243,7 +1323,20 @@ cudaError_t launch_tc_as(const WeightsView &w, const __nv_bfloat16 *x,
   memset(&tmap_c, 0, sizeof(tmap_c));
   memset(&tmap_s, 0, sizeof(tmap_s));
   best.a_map = 0;
-  if (FMT == TQ_FMT_B) {
+  if (FMT == TQ_FMT_B && w.format == TQ_FMT_B7) {
+    // [N][7 K / 8] bytes (K a multiple of 128, so every row starts on a
+    // 16-byte boundary); boxes of 128 rows x 112 bytes, not swizzled
+    const cuuint64_t pitch = (cuuint64_t)(w.k / 128) * kB7Row;
+    const cuuint64_t dims[2] = {pitch, (cuuint64_t)w.n};
+    const cuuint64_t strides[1] = {pitch};
+    const cuuint32_t box[2] = {kB7Row, (cuuint32_t)kTileM};
+    if (encode(&tmap_c, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+               const_cast<uint8_t *>(w.codes), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  } else if (FMT == TQ_FMT_B) {
     // [N][K] bytes; boxes of 128 rows x 128 codes, 128-byte swizzle
     const cuuint64_t dims[2] = {(cuuint64_t)w.k, (cuuint64_t)w.n};
     const cuuint64_t strides[1] = {(cuuint64_t)w.k};
@@ -1329,6 +1422,11 @@ bool gemm_tc_supported(const WeightsView &w, int64_t batch) {
     return false;
   // adaptive alphabet: a decoder warp's 32 rows must share a code book
   if (w.format == TQ_FMT_B) return w.lut_rows % 32 == 0;
+  // 7-bit alphabet: tensor copies of whole 112-byte runs (128 indices) need
+  // K a multiple of 128 and the codes on a 16-byte boundary
+  if (w.format == TQ_FMT_B7)
+    return w.k % 128 == 0 &&
+           (reinterpret_cast<uintptr_t>(w.codes) & 15u) == 0;
   return w.format == TQ_FMT_A && w.group == 64;
 }
 
@@ -1338,7 +1436,7 @@ cudaError_t gemm_tc(const WeightsView &w, const __nv_bfloat16 *x,
   for (int64_t b0 = 0; b0 < batch; b0 += kMaxN) {
     const int64_t nb = batch - b0 < kMaxN ? batch - b0 : kMaxN;
     const cudaError_t e =
-        w.format == TQ_FMT_B
+        w.format == TQ_FMT_B || w.format == TQ_FMT_B7
             ? launch_tc<TQ_FMT_B>(w, x + b0 * ldx, nb, ldx, y + b0 * ldy, ldy,
                                   stream)
             : launch_tc<TQ_FMT_A>(w, x + b0 * ldx, nb, ldx, y + b0 * ldy, ldy,
