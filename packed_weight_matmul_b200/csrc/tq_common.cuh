@@ -2,6 +2,7 @@
 #pragma once
 
 #include <atomic>
+#include <utility>
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -73,6 +74,48 @@ struct ExpertsView {
   int64_t ldx, ldy;
   int32_t *status;
 };
+
+// Programmatic dependent launch. A kernel launched with programmatic stream
+// serialization may start while the kernel before it on the stream is still
+// running (once every CTA of that kernel has called pdl_launch_dependents or
+// exited). Before pdl_wait it may only touch its own shared memory and
+// tensor memory and hint the L2 cache (prefetches do not read into the SM,
+// and L2 is coherent, so a prefetch of bytes the earlier kernel is still
+// writing is harmless); pdl_wait returns once the earlier kernel has
+// completed and its writes are visible, so every read of user memory and
+// every global write comes after it. Without the attribute pdl_wait returns
+// at once.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ void pdl_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// L2 prefetch of `bytes` (a multiple of 16, 16-byte aligned) at `p`.
+__device__ __forceinline__ void prefetch_l2_bulk(const void *p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p),
+               "r"(bytes)
+               : "memory");
+}
+
+// Launch `kern` with programmatic stream serialization (see pdl_wait).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block,
+                       size_t smem, cudaStream_t stream, Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 // Raise a kernel's dynamic shared-memory limit to `bytes` once per device.
 // The attribute is one value per function and context; every caller asks for

@@ -460,8 +460,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   // unless it is not a multiple of 64 KB: then no work is safe, the outputs
   // are NaN, and a CTA of a cluster still takes the cluster's two barriers
   // (its partial tile is NaN, so the rows the others finish are NaN too).
+  // the next kernel on the stream may be scheduled onto SMs this grid frees
+  pdl_launch_dependents();
   const uint32_t delta = base - P.base;
   if ((delta & 0xFFFFu) != 0u) {
+    pdl_wait();
     const float qnan = __int_as_float(0x7FC00000);
     if (ks == 1) {
       for (int t = cid; t < P.tiles; t += nclusters)
@@ -540,6 +543,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (FMT == TQ_FMT_A)
       asm volatile("prefetch.tensormap [%0];" ::"l"(&tmap_s) : "memory");
   }
+  // While the kernel before this one on the stream finishes: warm L2 with
+  // the code boxes of this CTA's first stages (Format B); then wait for that
+  // kernel's completion before reading user memory (the code book first).
+  if constexpr (FMT == TQ_FMT_B) {
+    if (warp == kWarpCodes && lane == 0 && cid < P.tiles) {
+      const bool b7p = w.format == TQ_FMT_B7;
+      const int pre = it1 - it0 < P.code_stages ? it1 - it0 : P.code_stages;
+      for (int i = 0; i < pre; ++i)
+        tma_prefetch_2d(&tmap_c, (it0 + i) * (int)(b7p ? kB7Row : kKB),
+                        cid * kTileM);
+    }
+  }
+  pdl_wait();
   // Format B: when every code-book entry is an integer multiple m of one
   // unit u (|m| <= 256, to 2^-20 of the entry; e.g. the balanced-ternary
   // ladder 3^-(i-1), whose 243 words are the integers -121..121 in units of
@@ -1385,13 +1401,18 @@ cudaError_t launch_tc_as(const WeightsView &w, const __nv_bfloat16 *x,
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = best.smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = (unsigned)best.ks;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  // programmatic dependent launch: the set-up and the first L2 prefetches
+  // overlap the end of the kernel before (the kernel waits for it before
+  // reading user memory)
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   unsigned long long *trace =
       CK ? reinterpret_cast<unsigned long long *>(g_test_trace.load()) : nullptr;
   return cudaLaunchKernelEx(&cfg, kern, w, batch, y, ldy, best, tmap_x, tmap_c,

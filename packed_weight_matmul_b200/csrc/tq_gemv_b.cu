@@ -177,11 +177,14 @@ __global__ void __launch_bounds__(NT, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t row_lo = (int64_t)blockIdx.x * n / gridDim.x;
   const int rows = (int)((int64_t)(blockIdx.x + 1) * n / gridDim.x - row_lo);
+  // the next kernel on the stream may be scheduled onto SMs this grid frees
+  pdl_launch_dependents();
 
   // The layout assumes the dynamic window starts at or below kRingLoAddr
   // (then the request covers the code book, the partial sums and the rings).
   const uint32_t base = (uint32_t)__cvta_generic_to_shared(smem);
   if (base > kRingLoAddr) {
+    pdl_wait();
     for (int i = threadIdx.x; i < rows * B; i += NT) {
       const int r = i / B, b = i - r * B;
       y[(int64_t)b * ldy + row_lo + r] = __int_as_float(0x7FC00000);
@@ -272,6 +275,29 @@ __global__ void __launch_bounds__(NT, 1)
         xw[b][q + 3] = v.w;
       }
   };
+
+  // While the kernel before this one on the stream finishes: warm L2 with
+  // this warp's first units (about 8 KB; lane r < R takes row r of each),
+  // then wait for that kernel's completion before reading user memory.
+  {
+    constexpr int kPre = (8192 / (int)kSlot) > 1 ? 8192 / (int)kSlot : 1;
+    UnitPos pq = ld;
+    const uint8_t *pp = ld_p;
+    for (int i = 0; i < kPre && u_begin + i < u_end; ++i) {
+      const int64_t k0 = (int64_t)pq.c * KC;
+      const uint32_t run = (uint32_t)(k - k0 < KC ? k - k0 : KC);
+      if (lane < R && pq.g * R + lane < rows)
+        prefetch_l2_bulk(pp - lane * KPL + (int64_t)lane * kstride, run);
+      if constexpr (CM) {
+        advance_cm(pq, ng);
+        pp = pq.g == 0 ? crow + (int64_t)pq.c * KC : pp + group_step;
+      } else {
+        advance(pq, nchunks);
+        pp = pq.c == 0 ? crow + (int64_t)pq.g * group_step : pp + KC;
+      }
+    }
+  }
+  pdl_wait();
 
   // Start the first copies, then clear the partial sums and build the code
   // book while they fly.
@@ -432,10 +458,9 @@ cudaError_t launch_cfg(const WeightsView &w, const __nv_bfloat16 *x,
   auto kern = gemv_b_kernel<B, R, D, NT, CM>;
   cudaError_t e = ensure_smem_limit<gemv_b_kernel<B, R, D, NT, CM>>(kSmemMax);
   if (e != cudaSuccess) return e;
-  kern<<<(unsigned)ctas, NT, smem, stream>>>(w.codes, w.n, w.k, w.lut,
-                                              w.scales, w.rps, x, ldx, y, ldy,
-                                              rows_max, hi_ring);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3((unsigned)ctas), dim3(NT), smem, stream,
+                    w.codes, w.n, w.k, w.lut, w.scales, w.rps, x, ldx, y, ldy,
+                    rows_max, hi_ring);
 }
 
 int device_sms() {

@@ -145,6 +145,17 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *tmap,
 
 // ---- thread-block clusters -------------------------------------------------
 
+// L2 prefetch of the box of a 2-D tensor map at (c0, c1) (no shared-memory
+// destination, no barrier).
+__device__ __forceinline__ void tma_prefetch_2d(const void *tmap, int c0,
+                                                int c1) {
+  asm volatile(
+      "cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+          tmap),
+      "r"(c0), "r"(c1)
+      : "memory");
+}
+
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
