@@ -43,6 +43,15 @@ tq_status tq_testing_linear_wait_fault(int32_t withhold_first_arrive,
  * Returns TQ_ERR_INVALID_ARG for other values. */
 tq_status tq_testing_force_linear_path(int32_t path);
 
+/* Plan the tensor-core tq_linear launches issued after this call, in every
+ * thread of the process, with a split of K over clusters of `ks` CTAs
+ * (1..8; 0 = the planner's choice) and at most `max_clusters` clusters
+ * (0 = as many as are resident or as there are row tiles), so that tests
+ * can make each cluster walk several tiles on a small shape. A split the
+ * shape or the device cannot take makes those calls fail
+ * (TQ_ERR_CUDA). Returns TQ_ERR_INVALID_ARG for values out of range. */
+tq_status tq_testing_tc_split(int32_t ks, int32_t max_clusters);
+
 /* Select the self-checking build of the tensor-core kernel for the tq_linear
  * calls issued after this call (enable != 0), or the ordinary one. The
  * self-checking kernel verifies every shared-memory, tensor-memory,

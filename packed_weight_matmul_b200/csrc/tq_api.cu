@@ -294,6 +294,13 @@ tq_status tq_testing_force_linear_path(int32_t path) {
   return TQ_OK;
 }
 
+tq_status tq_testing_tc_split(int32_t ks, int32_t max_clusters) {
+  if (ks < 0 || ks > 8 || max_clusters < 0) return TQ_ERR_INVALID_ARG;
+  tq::g_test_tc_ks.store(ks);
+  tq::g_test_tc_clusters.store(max_clusters);
+  return TQ_OK;
+}
+
 tq_status tq_testing_tc_self_check(int32_t enable, uint64_t record_out[4],
                                    int32_t reset) {
   tq::g_test_self_check.store(enable != 0 ? 1 : 0);

@@ -9,9 +9,9 @@
 //             indices into the layer's used words (section 8.1)
 //
 // Warp-specialised, one CTA per SM (it holds the whole tensor memory).
-// Without a split of K the CTAs are persistent and walk the 128-row tiles of
-// y^T: tile t, t + CTAs, ... With a split, a cluster of `ks` CTAs takes one
-// tile, each CTA a slice of K. For each 128-wide k block ("iteration"):
+// Persistent clusters of `ks` CTAs walk the 128-row tiles of y^T: tile t,
+// t + clusters, ...; with a split of K (ks > 1) each CTA of the cluster
+// takes a slice of K of every tile. For each 128-wide k block ("iteration"):
 //   - the code producer warp copies the tile's codes into a shared-memory
 //     ring with tensor copies (TMA): Format B one 128-row x 128-code box
 //     per block (7-bit indices: 128 rows x 112 bytes); Format A one box of codes and one of fp16 scales per window
@@ -42,10 +42,12 @@
 //     to the accumulator barrier;
 //   - 4 epilogue warps read the accumulator (double-buffered in tensor
 //     memory, so the next tile's MMAs proceed meanwhile) and store y, or,
-//     with a split, keep the partial tile in shared memory; after a cluster
-//     barrier each CTA adds the `ks` partials of the rows it owns in rank
-//     order (distributed shared memory; deterministic), applies rho and
-//     stores y; a second barrier keeps every CTA alive while peers read.
+//     with a split, put the partial tile in shared memory; once every CTA
+//     of the cluster has arrived on its "part full" barrier, each CTA adds
+//     the `ks` partials of the rows it owns in rank order (distributed
+//     shared memory; deterministic), applies rho and stores y, and arrives
+//     on every CTA's "part free" barrier, which releases the buffers for
+//     the next tile. This runs while the next tile's blocks stream in.
 // Decoding uses a 64 KB table in shared memory at a 64 KB-aligned address,
 // replicated once per lane, so that one byte permute of a code word with the
 // lane's base word is the complete lookup address and a warp's lookups hit
@@ -89,6 +91,9 @@ std::atomic<int> g_test_self_check{0};
 // Mapped host buffer of the self-checking kernel's progress trace (or 0):
 // entry [block * 8 + role] holds the last step the role reached.
 std::atomic<unsigned long long> g_test_trace{0};
+// Forced split of K and cluster cap (tq_testing_tc_split; 0 = automatic).
+std::atomic<int> g_test_tc_ks{0};
+std::atomic<int> g_test_tc_clusters{0};
 
 // Record of the self-checking instantiation (test hook): [0] first
 // violation (site << 48 | warp << 40 | block), [1] its value, [2] number of
@@ -110,6 +115,7 @@ constexpr int kWarpCodes = 0, kWarpX = 1, kWarpMma = 2, kWarpEpi = 3,
               kWarpDec = 7, kWarpWait = kWarpDec + kDecWarps;
 constexpr int kThreads = 32 * (kWarpWait + 1);  // 512
 constexpr int kBarIdStage = 1;  // named barrier: waiter -> MMA issuer
+constexpr int kBarIdEpi = 2;    // named barrier: the 4 epilogue warps
 constexpr int kMaxCodeStages = 8;
 constexpr int kMaxXStages = 4;
 constexpr uint32_t kBRow = 128;          // Format B row: 128 codes, swizzled
@@ -127,7 +133,8 @@ constexpr uint32_t kBarCodeFull = 0, kBarCodeEmpty = 64, kBarXFull = 128,
                    kBarXEmpty = 160, kBarAFull = 192, kBarAEmpty = 216,
                    kBarAccFull = 240, kBarAccEmpty = 256, kBarDrain = 296,
                    kTmemSlot = 304, kAbort = 308, kUnit = 312,
-                   kBarBytes = 320;
+                   kBarPartFull = 320, kBarPartFree = 328,
+                   kBarBytes = 336;
 
 struct TcPlan {
   int n_pad, ks, tiles, kblocks, iters;
@@ -458,9 +465,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   // rank (a shared::cta address is a shared::cluster one), so every planned
   // address moves by this CTA's offset. It keeps the table's 64 KB alignment
   // unless it is not a multiple of 64 KB: then no work is safe, the outputs
-  // are NaN, and a CTA of a cluster still takes the cluster's two barriers
-  // (its partial tile is NaN, so the rows the others finish are NaN too).
-  // the next kernel on the stream may be scheduled onto SMs this grid frees
+  // it owns are NaN, and a CTA of a cluster still takes the cluster's two
+  // barriers (its peers wait for its partial tiles in vain, time out and
+  // write NaN too).
+  // The next kernel on the stream may be scheduled onto SMs this grid frees.
   pdl_launch_dependents();
   const uint32_t delta = base - P.base;
   if ((delta & 0xFFFFu) != 0u) {
@@ -475,14 +483,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
       namespace cg = cooperative_groups;
       cg::cluster_group cluster = cg::this_cluster();
-      for (int i = threadIdx.x; i < kTileM * n_pad; i += blockDim.x)
-        part[i] = qnan;
       cluster.sync();
-      for (int i = threadIdx.x; i < (r_hi - r_lo) * nb; i += blockDim.x) {
-        const int64_t row = (int64_t)cid * kTileM + r_lo + i % (r_hi - r_lo);
-        if (cid < P.tiles && row < N)
-          y[(int64_t)(i / (r_hi - r_lo)) * ldy + row] = qnan;
-      }
+      const int own = r_hi - r_lo;
+      for (int t = cid; t < P.tiles; t += nclusters)
+        for (int i = threadIdx.x; i < own * nb; i += blockDim.x) {
+          const int64_t row = (int64_t)t * kTileM + r_lo + i % own;
+          if (row < N) y[(int64_t)(i / own) * ldy + row] = qnan;
+        }
       cluster.sync();
     }
     return;
@@ -529,6 +536,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(B0 + kBarAccEmpty + 8 * b, 4);
     }
     mbar_init(B0 + kBarDrain, 1);
+    if (ks > 1) {
+      mbar_init(B0 + kBarPartFull, (uint32_t)ks);
+      mbar_init(B0 + kBarPartFree, (uint32_t)ks);
+    }
     st_volatile_s32(B0 + kUnit, 0x7F800000);  // +inf
     mbar_init_fence();
   }
@@ -622,6 +633,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   tc_fence_before_sync();
   __syncthreads();
+  // with a split of K, peers arrive on this CTA's partial-tile barriers:
+  // every CTA of the cluster has initialised its barriers after this
+  if (ks > 1) cooperative_groups::this_cluster().sync();
   tc_fence_after_sync();
   uint32_t tmem;
   asm volatile("ld.shared.u32 %0, [%1];" : "=r"(tmem) : "r"(B0 + kTmemSlot)
@@ -937,15 +951,67 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
       } else {
-        // a K slice (one tile per CTA): the partial row goes to this CTA's
-        // shared buffer; the owners add the cluster's partials after the
-        // cluster barrier at the end of the kernel
-        // (batch column c of the tile at part[c * 128 ..]: a warp's stores
-        // and the owners' reads are 32 consecutive words, conflict-free)
+        // a K slice: the partial tile goes to this CTA's shared buffer
+        // (batch column c at part[c * 128 ..]: a warp's stores and the
+        // owners' reads are 32 consecutive words, conflict-free), and the
+        // cluster adds the ks partials through distributed shared memory,
+        // each CTA the rows it owns, in rank order (deterministic). Per
+        // tile, each CTA arrives once on every CTA's "part full" barrier
+        // (its partial is written) and once on every CTA's "part free"
+        // barrier (it has read the partials), so a buffer is overwritten
+        // only after every peer has read it. A CTA whose epilogue stopped
+        // (time-out) arrives no more: its peers' next wait times out, and
+        // the rows of the tiles still open are NaN.
+        const int et = (int)threadIdx.x - 32 * kWarpEpi;  // 0..127
+        if (i >= 1 && !dead) {
+          const bool got = mbar_wait_cluster(B0 + kBarPartFree,
+                                             (uint32_t)(i - 1) & 1u,
+                                             abort_addr, lim);
+          if constexpr (CK) if (!got) ck_record(26, (uint64_t)i);
+          dead = !got;
+        }
         if constexpr (CK) ck_smem<CK>(W, P.red + delta, (uint32_t)(kTileM * n_pad * 4), 14);
 #pragma unroll
         for (int c = 0; c < 64; ++c)
-          if (c < n_pad) part[c * kTileM + r] = __uint_as_float(v[c]);
+          if (c < n_pad)
+            part[c * kTileM + r] = dead ? __int_as_float(0x7FC00000)
+                                        : __uint_as_float(v[c]);
+        asm volatile("fence.acq_rel.cluster;" ::: "memory");
+        dead = !bar_red_and(kBarIdEpi, 128, !dead);
+        if (!dead && et == 0)
+          for (int p = 0; p < ks; ++p)
+            mbar_arrive_cluster(B0 + kBarPartFull, (uint32_t)p);
+        bool full = false;
+        if (!dead) {
+          full = mbar_wait_cluster(B0 + kBarPartFull, (uint32_t)i & 1u,
+                                   abort_addr, lim);
+          if constexpr (CK) if (!full) ck_record(27, (uint64_t)i);
+        }
+        namespace cg = cooperative_groups;
+        cg::cluster_group cluster = cg::this_cluster();
+        const int own = r_hi - r_lo;
+        for (int idx = et; idx < own * nb; idx += 128) {
+          const int orr = idx % own, b = idx / own;
+          float sum = __int_as_float(0x7FC00000);
+          if (full) {
+            sum = 0.0f;
+            for (int p = 0; p < ks; ++p)
+              sum += cluster.map_shared_rank(part, p)[b * kTileM + r_lo + orr];
+          }
+          const int64_t row = row0 + r_lo + orr;
+          if (row < N) {
+            float scale = 1.0f;
+            if constexpr (FMT == TQ_FMT_B) {
+              if (w.scales != nullptr)
+                scale = __half2float(__ushort_as_half(w.scales[row / w.rps]));
+            }
+            y[(int64_t)b * ldy + row] = scale * (unit * sum);
+          }
+        }
+        dead = !bar_red_and(kBarIdEpi, 128, full);
+        if (!dead && et == 0)
+          for (int p = 0; p < ks; ++p)
+            mbar_arrive_cluster(B0 + kBarPartFree, (uint32_t)p);
       }
     }
   } else if (warp < kWarpDec + kDecWarps) {
@@ -1134,36 +1200,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before_sync();
   __syncthreads();
   if (threadIdx.x == 0) ck_trace<CK>(trace, 6, 0xFFFF, 0, 1);
+  // every CTA of a cluster stays until its peers have read its partials and
+  // arrived on its barriers
   if (ks > 1) {
-    // Add the cluster's partial tiles through distributed shared memory in
-    // rank order (deterministic); this CTA finishes the rows it owns. The
-    // second barrier keeps every CTA alive while peers read its partials.
-    namespace cg = cooperative_groups;
-    cg::cluster_group cluster = cg::this_cluster();
     __syncwarp();
-    cluster.sync();
-    if (warp >= kWarpEpi && warp < kWarpDec && cid < P.tiles) {
-      const int et = (int)threadIdx.x - 32 * kWarpEpi;  // 0..127
-      const int64_t row0 = (int64_t)cid * kTileM;
-      const int own = r_hi - r_lo;
-      for (int idx = et; idx < own * nb; idx += 128) {
-        const int orr = idx % own, b = idx / own;
-        float sum = 0.0f;
-        for (int p = 0; p < ks; ++p)
-          sum += cluster.map_shared_rank(part, p)[b * kTileM + r_lo + orr];
-        const int64_t row = row0 + r_lo + orr;
-        if (row < N) {
-          float scale = 1.0f;
-          if constexpr (FMT == TQ_FMT_B) {
-            if (w.scales != nullptr)
-              scale = __half2float(__ushort_as_half(w.scales[row / w.rps]));
-          }
-          y[(int64_t)b * ldy + row] = scale * (unit * sum);
-        }
-      }
-    }
-    __syncwarp();
-    cluster.sync();
+    cooperative_groups::this_cluster().sync();
   }
   if (warp == kWarpMma) {
     __syncwarp();  // converged for the warp-wide free
@@ -1276,13 +1317,15 @@ cudaError_t launch_tc_as(const WeightsView &w, const __nv_bfloat16 *x,
   if (tiles > (1 << 30) || iters < 1) return cudaErrorInvalidValue;
 
   // Cluster size: the K split whose resident clusters finish the tiles with
-  // the fewest iterations per CTA (ceil(tiles / resident clusters) waves of
-  // ceil(iters / ks) blocks, plus a per-tile allowance), preferring no split.
+  // the fewest iterations per CTA (ceil(tiles / resident clusters) tiles of
+  // ceil(iters / ks) blocks, plus a set-up allowance), preferring no split.
   static std::atomic<int> occ_cache[16][2][4][9];  // per instantiation
   TcPlan best{};
   int best_clusters = 0;
   int64_t best_cost = -1;
+  const int force_ks = g_test_tc_ks.load(), max_clusters = g_test_tc_clusters.load();
   for (int ks = 1; ks <= 8 && ks <= iters; ++ks) {
+    if (force_ks > 0 && ks != force_ks) continue;
     TcPlan P{};
     if (!plan_smem(FMT, n_pad, ks, (uint32_t)reserved, &P)) continue;
     std::atomic<int> *slot =
@@ -1294,13 +1337,14 @@ cudaError_t launch_tc_as(const WeightsView &w, const __nv_bfloat16 *x,
       if (slot && c > 0) slot->store(c);
     }
     if (c <= 0) continue;
-    // ks = 1: persistent CTAs walk the tiles; ks > 1: one tile per cluster
-    // (the partials are added at the end of the kernel), each wave paying
-    // the set-up again
-    const int64_t clusters = ks == 1 ? (c < tiles ? c : tiles) : tiles;
-    const int64_t waves = (tiles + c - 1) / c;
+    // persistent clusters walk the tiles (with a split, each tile's partials
+    // are added while the next tile runs); the set-up and the last tile's
+    // epilogue are paid once
+    int64_t clusters = c < tiles ? c : tiles;
+    if (max_clusters > 0 && clusters > max_clusters) clusters = max_clusters;
+    const int64_t waves = (tiles + clusters - 1) / clusters;
     const int64_t cost =
-        waves * (((int64_t)iters + ks - 1) / ks + (ks == 1 ? 2 : 4));
+        waves * (((int64_t)iters + ks - 1) / ks) + (ks == 1 ? 2 : 4);
     if (best_cost < 0 || cost < best_cost) {
       best_cost = cost;
       best = P;

@@ -13,6 +13,9 @@ extern std::atomic<int> g_test_force_path;
 // Self-checking tensor-core kernel (tq_testing_tc_self_check) and its record.
 extern std::atomic<int> g_test_self_check;
 extern std::atomic<unsigned long long> g_test_trace;
+// Split of K and cluster cap forced by tq_testing_tc_split (0 = automatic).
+extern std::atomic<int> g_test_tc_ks;
+extern std::atomic<int> g_test_tc_clusters;
 cudaError_t tc_check_record(uint64_t out[4], bool reset);
 
 // One warp per row; any shape the boundary accepts.

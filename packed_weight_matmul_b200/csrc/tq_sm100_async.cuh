@@ -61,6 +61,48 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with acquire at cluster scope: the writes that other CTAs of the
+// cluster released with their arrivals are visible afterwards.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar,
+                                                      uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n"
+      " mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Arrive, with release at cluster scope, on the barrier at this CTA's shared
+// address `bar` in the cluster's CTA `rank` (the same offset in its window).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar,
+                                                    uint32_t rank) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
+               : "=r"(remote)
+               : "r"(bar), "r"(rank));
+  asm volatile(
+      "mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(
+          remote)
+      : "memory");
+}
+
+// Store `v` to the word at this CTA's shared address `addr` in the cluster's
+// CTA `rank`.
+__device__ __forceinline__ void st_cluster_s32(uint32_t addr, uint32_t rank,
+                                               int v) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
+               : "=r"(remote)
+               : "r"(addr), "r"(rank));
+  asm volatile("st.relaxed.cluster.shared::cluster.u32 [%0], %1;" ::"r"(remote),
+               "r"(v)
+               : "memory");
+}
+
 __device__ __forceinline__ int ld_volatile_s32(uint32_t addr) {
   int v;
   asm volatile("ld.volatile.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr)
@@ -88,6 +130,23 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
   const uint64_t t0 = global_ns();
   for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
+    if (ld_volatile_s32(abort_addr) != 0) return false;
+    if (global_ns() - t0 > limit_ns) {
+      st_volatile_s32(abort_addr, 1);
+      return false;
+    }
+  }
+}
+
+// As mbar_wait, with acquire at cluster scope (see mbar_try_wait_cluster).
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar,
+                                                  uint32_t parity,
+                                                  uint32_t abort_addr,
+                                                  uint64_t limit_ns) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (;;) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
     if (ld_volatile_s32(abort_addr) != 0) return false;
     if (global_ns() - t0 > limit_ns) {
       st_volatile_s32(abort_addr, 1);

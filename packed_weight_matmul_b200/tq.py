@@ -27,7 +27,7 @@ ENTRY_POINTS = ("tq_packed_bytes", "tq_build_lut", "tq_quantize_pack",
                 "tq_encode_b", "tq_testing_linear_wait_fault",
                 "tq_testing_force_linear_path", "tq_testing_tc_self_check",
                 "tq_testing_tc_trace", "tq_linear_experts", "tq_pack7",
-                "tq_build_lut7")
+                "tq_build_lut7", "tq_testing_tc_split")
 
 
 class TqError(RuntimeError):
@@ -80,6 +80,8 @@ def _load():
     L.tq_testing_linear_wait_fault.argtypes = [i32, C.c_uint64]
     L.tq_testing_force_linear_path.restype = C.c_int
     L.tq_testing_force_linear_path.argtypes = [i32]
+    L.tq_testing_tc_split.restype = C.c_int
+    L.tq_testing_tc_split.argtypes = [i32, i32]
     L.tq_testing_tc_self_check.restype = C.c_int
     L.tq_testing_tc_self_check.argtypes = [i32, P, i32]
     L.tq_testing_tc_trace.restype = C.c_int
@@ -193,6 +195,13 @@ def tq_testing_force_linear_path(path: int) -> None:
     code book always split into bf16 hi + lo operands."""
     _check(_lib.tq_testing_force_linear_path(int(path)),
            "tq_testing_force_linear_path")
+
+
+def tq_testing_tc_split(ks: int, max_clusters: int = 0) -> None:
+    """Test hook (include/tq_testing.h): split of K over clusters of ks
+    CTAs (0 = planner's choice) and a cap on the number of clusters."""
+    _check(_lib.tq_testing_tc_split(int(ks), int(max_clusters)),
+           "tq_testing_tc_split")
 
 
 def tq_testing_tc_self_check(enable: bool, read: bool = False,

@@ -219,3 +219,16 @@ def test_pack7_and_b7_validation(tq):
     lut = np.arange(256, dtype=np.float32)
     used = np.arange(128, dtype=np.uint8)[::-1].copy()
     assert np.array_equal(tq.tq_build_lut7(lut, used), lut[used])
+
+
+def test_tc_split_hook_range(tq):
+    # host-only: the hook stores the plan override; out-of-range values are
+    # rejected and (0, 0) restores the planner's choice
+    with pytest.raises(tq.TqError):
+        tq.tq_testing_tc_split(9, 0)
+    with pytest.raises(tq.TqError):
+        tq.tq_testing_tc_split(-1, 0)
+    with pytest.raises(tq.TqError):
+        tq.tq_testing_tc_split(2, -1)
+    tq.tq_testing_tc_split(3, 2)
+    tq.tq_testing_tc_split(0, 0)
