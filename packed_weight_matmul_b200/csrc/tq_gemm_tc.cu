@@ -270,6 +270,41 @@ __device__ __forceinline__ void decode_b_hi(const uint32_t (&cw)[16],
   }
 }
 
+// bf16 pair of two fp32 values, `lo` in the low half.
+__device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Format B, single operand, for a code book whose entry c is u * (c - 121)
+// (the balanced-ternary ladder 3^-(i-1): code byte c = 121 + sum t_i 3^i):
+// 64 codes of one row -> 32 bf16 pairs of c - 121, without table lookups.
+// A byte permute places code c in the low byte of the fp32 pattern of
+// 2^23 + c, a packed fp32 subtraction of 2^23 + 121 leaves c - 121 (exact),
+// and one conversion packs two of them. Returns non-zero iff a code of the
+// run is >= 243 (invalid): per byte, bit 7 of (c & 0x7F) + 0x0D is set iff
+// (c & 0x7F) >= 0x73, which with bit 7 of c set is c >= 0xF3.
+__device__ __forceinline__ uint32_t decode_b_arith(const uint32_t (&cw)[16],
+                                                   uint32_t (&hi)[32]) {
+  const float2 bias = make_float2(-8388729.0f, -8388729.0f);  // -(2^23 + 121)
+  uint32_t bad = 0;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const uint32_t w = cw[j];
+    float2 a = make_float2(__uint_as_float(prmt(w, 0x4B000000u, 0x7540u)),
+                           __uint_as_float(prmt(w, 0x4B000000u, 0x7541u)));
+    float2 b = make_float2(__uint_as_float(prmt(w, 0x4B000000u, 0x7542u)),
+                           __uint_as_float(prmt(w, 0x4B000000u, 0x7543u)));
+    a = __fadd2_rn(a, bias);
+    b = __fadd2_rn(b, bias);
+    hi[2 * j] = bf16x2_rn(a.x, a.y);
+    hi[2 * j + 1] = bf16x2_rn(b.x, b.y);
+    bad |= ((w & 0x7F7F7F7Fu) + 0x0D0D0D0Du) & w;
+  }
+  return bad & 0x80808080u;
+}
+
 // Format B with a code book per block of rows (adaptive alphabet): 64 codes
 // of one row -> 32 hi and 32 lo bf16 pairs through the warp's compact book
 // (256 words bf16 hi | lo << 16 at ctab).
@@ -455,8 +490,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   // this CTA's iterations of every tile
   const int it0 = (int)((int64_t)P.iters * rank / ks);
   const int it1 = (int)((int64_t)P.iters * (rank + 1) / ks);
-  // rows of every tile this CTA owns in the cluster reduction
-  const int r_lo = kTileM * rank / ks, r_hi = kTileM * (rank + 1) / ks;
+  // rows of every tile this CTA owns in the cluster reduction: whole groups
+  // of 4 rows (one 16-byte vector of a partial-tile column)
+  const int r_lo = 4 * (kTileM / 4 * rank / ks),
+            r_hi = 4 * (kTileM / 4 * (rank + 1) / ks);
   // partial tile of a K split (same offset in every CTA of the cluster)
   float *const part = reinterpret_cast<float *>(smem + (P.red - P.base));
 
@@ -575,7 +612,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // 2^-20, is below that of the hi + lo split (2^-17). Otherwise each entry
   // becomes bf16 hi + lo (two MMAs). u is the smallest non-zero |entry|; the
   // test runs in every CTA on the same table, so all CTAs agree.
-  bool grid = false;
+  bool grid = false, ident = false;
   float unit = 1.0f;
   // adaptive alphabet: every decoder warp builds its rows' compact book per
   // tile in the table region; no shared table, no single-operand path
@@ -594,18 +631,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncthreads();
     const float u = __int_as_float(ld_volatile_s32(B0 + kUnit));
-    bool ok = true;
+    bool ok = true, id_ok = true;
     if ((int)threadIdx.x < n_words) {
       const float m = rintf(__fdiv_rn(lv, u));
       ok = u <= 3.4028235e38f && fabsf(m) <= 256.0f &&
            fabs((double)lv - (double)u * (double)m) <=
                ldexp(fabs((double)lv), -20);
+      id_ok = m == (float)((int)threadIdx.x - 121);
     }
     grid = __syncthreads_and(ok) != 0 && P.grid_ok != 0;
+    // m = c - 121 for every word: decode without the table
+    const bool all_id = __syncthreads_and(id_ok) != 0;
+    ident = grid && !b7 && all_id;
     if (grid) unit = u;
   }
   // the lane-replicated table
-  if (FMT == TQ_FMT_B && !adaptive) {
+  if (FMT == TQ_FMT_B && !adaptive && !ident) {
     for (int i = threadIdx.x; i < 256 * 8; i += blockDim.x) {
       const int e = i >> 3, j = i & 7;
       // entries past the book (7-bit alphabet: 128 words) are never read
@@ -987,25 +1028,61 @@ __global__ void __launch_bounds__(kThreads, 1)
                                    abort_addr, lim);
           if constexpr (CK) if (!full) ck_record(27, (uint64_t)i);
         }
+        // this CTA's rows: 16-byte vectors (4 rows of one batch column) from
+        // every CTA's partial tile, two vectors per thread in flight
         namespace cg = cooperative_groups;
         cg::cluster_group cluster = cg::this_cluster();
-        const int own = r_hi - r_lo;
-        for (int idx = et; idx < own * nb; idx += 128) {
-          const int orr = idx % own, b = idx / own;
-          float sum = __int_as_float(0x7FC00000);
-          if (full) {
-            sum = 0.0f;
-            for (int p = 0; p < ks; ++p)
-              sum += cluster.map_shared_rank(part, p)[b * kTileM + r_lo + orr];
+        const int own4 = (r_hi - r_lo) / 4;
+        const int units = own4 * nb;
+        for (int u0 = et; u0 < units; u0 += 256) {
+          float4 acc[2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const float qn = __int_as_float(0x7FC00000);
+            acc[h] = make_float4(qn, qn, qn, qn);
           }
-          const int64_t row = row0 + r_lo + orr;
-          if (row < N) {
-            float scale = 1.0f;
-            if constexpr (FMT == TQ_FMT_B) {
-              if (w.scales != nullptr)
-                scale = __half2float(__ushort_as_half(w.scales[row / w.rps]));
+          if (full) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) acc[h] = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int p = 0; p < ks; ++p) {
+              const float *pp = cluster.map_shared_rank(part, p);
+              float4 v4[2];
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const int u = u0 + 128 * h;
+                const int uu = u < units ? u : u0;
+                const int g = uu % own4, b = uu / own4;
+                v4[h] = *reinterpret_cast<const float4 *>(
+                    pp + b * kTileM + r_lo + 4 * g);
+              }
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                acc[h].x += v4[h].x;
+                acc[h].y += v4[h].y;
+                acc[h].z += v4[h].z;
+                acc[h].w += v4[h].w;
+              }
             }
-            y[(int64_t)b * ldy + row] = scale * (unit * sum);
+          }
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int u = u0 + 128 * h;
+            if (u >= units) continue;
+            const int g = u % own4, b = u / own4;
+            const float sv[4] = {acc[h].x, acc[h].y, acc[h].z, acc[h].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int64_t row = row0 + r_lo + 4 * g + e;
+              if (row < N) {
+                float scale = 1.0f;
+                if constexpr (FMT == TQ_FMT_B) {
+                  if (w.scales != nullptr)
+                    scale =
+                        __half2float(__ushort_as_half(w.scales[row / w.rps]));
+                }
+                y[(int64_t)b * ldy + row] = scale * (unit * sv[e]);
+              }
+            }
           }
         }
         dead = !bar_red_and(kBarIdEpi, 128, full);
@@ -1127,6 +1204,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 decode_b7<true>(d, lane_tab, hi, lo);
             } else if (adaptive) {
               decode_b_compact(cw, ctab, hi, lo);
+            } else if (ident) {
+              // an invalid code poisons its row: NaN operands
+              if (decode_b_arith(cw, hi) != 0u) {
+#pragma unroll
+                for (int m = 0; m < 32; ++m) hi[m] = 0x7FC07FC0u;
+              }
             } else if (grid) {
               decode_b_hi(cw, lane_tab, hi);
             } else {
@@ -1339,12 +1422,16 @@ cudaError_t launch_tc_as(const WeightsView &w, const __nv_bfloat16 *x,
     if (c <= 0) continue;
     // persistent clusters walk the tiles (with a split, each tile's partials
     // are added while the next tile runs); the set-up and the last tile's
-    // epilogue are paid once
+    // epilogue are paid once. Measured on B200: when clusters of 3, 5, 6 or
+    // 7 CTAs walk several tiles, every further tile costs about 4 blocks
+    // more (the per-tile hand-over between the CTAs is exposed; clusters of
+    // 2, 4 and 8 hide it)
     int64_t clusters = c < tiles ? c : tiles;
     if (max_clusters > 0 && clusters > max_clusters) clusters = max_clusters;
     const int64_t waves = (tiles + clusters - 1) / clusters;
-    const int64_t cost =
-        waves * (((int64_t)iters + ks - 1) / ks) + (ks == 1 ? 2 : 4);
+    const bool pow2 = (ks & (ks - 1)) == 0;
+    const int64_t cost = waves * (((int64_t)iters + ks - 1) / ks) +
+                         (ks == 1 ? 2 : 4) + (pow2 ? 0 : 4 * (waves - 1));
     if (best_cost < 0 || cost < best_cost) {
       best_cost = cost;
       best = P;

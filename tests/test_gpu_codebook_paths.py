@@ -8,7 +8,9 @@ tolerance as test_gpu_linear), force the hi + lo path on a code book that
 would take the single path (tq_testing_force_linear_path(3)), and check that
 an entry just off the grid is not forced onto it: with every code of a row
 equal and x all ones, an entry rounded onto the grid would miss by about
-1e-3 * K * |w|, far outside the tolerance."""
+1e-3 * K * |w|, far outside the tolerance. A book with entry c = u * (c - 121)
+(the balanced-ternary ladder, any alpha) is decoded without its table; every
+invalid byte value 243..255 must still make its row NaN on each path."""
 import numpy as np
 import pytest
 import torch
@@ -91,3 +93,26 @@ def test_integer_ladder_and_zero_book():
     for batch in (6, 64):
         y, _ = U.linear(w, I.x_normal(batch, 1040, batch))
         assert np.all(y == 0.0)
+
+
+@pytest.mark.parametrize("ladder,path", [("pow3", 0), ("pow3", 3),
+                                         ("free", 0)])
+def test_every_invalid_code_poisons_its_row(force_path, ladder, path):
+    # one invalid byte (243..255) per row in rows 0..12, at k positions that
+    # fall in both 64-k halves of a block, in different blocks and at the
+    # last k; the balanced-ternary book takes the table-free decode (path 0)
+    # or the hi + lo table (path 3), the free ladder the hi + lo table
+    lad = I.ladder_pow3().numpy() if ladder == "pow3" else LADDER_FREE
+    lut = oref.build_lut(I.ALPHA, lad)
+    n, k = 141, 1024
+    codes = I.codes_uniform(n, k, 31)
+    bad_rows = list(range(13))
+    for i in bad_rows:
+        kk = k - 1 if i == 12 else (77 * i + 64 * (i % 2)) % k
+        codes[i, kk] = 243 + i
+    force_path(path)
+    w = U.weights_b_dev(codes, lut)
+    for batch in (5, 16, 64):
+        y, _ = U.linear(w, I.x_normal(batch, k, batch))
+        assert np.all(np.isnan(y[:, bad_rows])), f"b={batch}"
+        assert np.all(np.isfinite(np.delete(y, bad_rows, axis=1))), f"b={batch}"
