@@ -116,6 +116,12 @@ constexpr int kWarpCodes = 0, kWarpX = 1, kWarpMma = 2, kWarpEpi = 3,
 constexpr int kThreads = 32 * (kWarpWait + 1);  // 512
 constexpr int kBarIdStage = 1;  // named barrier: waiter -> MMA issuer
 constexpr int kBarIdEpi = 2;    // named barrier: the 4 epilogue warps
+// Decode variants of the decoder warps (Format A always takes kDecPair):
+// Format B hi + lo table, single-operand table, table-free (entry c =
+// u * (c - 121)), per-warp books (adaptive alphabet), 7-bit indices with a
+// single-operand or a hi + lo table.
+constexpr int kDecPair = 0, kDecGrid = 1, kDecIdent = 2, kDecAdaptive = 3,
+              kDecB7Grid = 4, kDecB7Pair = 5;
 constexpr int kMaxCodeStages = 8;
 constexpr int kMaxXStages = 4;
 constexpr uint32_t kBRow = 128;          // Format B row: 128 codes, swizzled
@@ -1093,190 +1099,214 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp < kWarpDec + kDecWarps) {
     // ---- decoders -----------------------------------------------------------
-    const int q = warp & 3;
-    const int kp = (warp - kWarpDec) >> 2;  // which 64-k half of the block
-    const int r = 32 * q + lane;
-    const uint32_t lane_tab =
-        tab | (uint32_t)lane << (FMT == TQ_FMT_B ? 2 : 3);
-    const uint32_t t_hi =
-        tmem + ((uint32_t)(32 * q) << 16) + kAStage0 + 32u * (uint32_t)kp;
-    const bool skip_first = P.skip_first_arrive != 0;
-    int cs = 0, uc = 0, as = 0, ua = 0;
-    bool ok = true;
-    // this warp's compact book (adaptive alphabet)
-    const uint32_t ctab = tab + (uint32_t)(warp - kWarpDec) * 1024u;
-    for (int t = cid; ok && t < P.tiles; t += nclusters) {
-      const int64_t row = (int64_t)t * kTileM + r;
-      const bool row_ok = row < N;
-      if (adaptive) {
-        // rows t * 128 + 32 q .. + 31 share one book (lut_rows % 32 == 0);
-        // a warp wholly past N reads book 0 (its weights are masked)
-        const int64_t r0w = (int64_t)t * kTileM + 32 * q;
-        const float *bl = w.lut + ((r0w < N ? r0w : 0) / w.lut_rows) * 256;
-        __syncwarp();  // this warp's lookups of the previous tile are done
-        for (int e = lane; e < 256; e += 32) {
-          const float v = __ldg(bl + e);
-          const uint32_t h = bf16_bits_rn(v);
-          const uint32_t l = bf16_bits_rn(v - __uint_as_float(h << 16));
-          asm volatile("st.shared.u32 [%0], %1;" ::"r"(ctab + 4u * (uint32_t)e),
-                       "r"(h | l << 16)
-                       : "memory");
-        }
-        __syncwarp();
-      }
-      for (int ws = it0; ws < it1;) {
-        const int we = window_end(ws, it1, P.kblocks, kWin);
-        ok = __all_sync(0xFFFFFFFFu,
-                        mbar_wait(B0 + kBarCodeFull + 8 * cs,
-                                  (uint32_t)(uc / P.code_stages) & 1u,
-                                  abort_addr, lim));
-        if constexpr (CK) if (!ok && lane == 0) ck_record(28, (uint64_t)uc);
-        if (!ok) break;
-        // this row's codes (crow) and scales (srow) in the stage; a row
-        // written by a tensor copy is swizzled: logical byte o is at o ^ sw
-        const bool swz = (FMT == TQ_FMT_B && !b7) || P.a_map;
-        const uint32_t sw = swz ? (uint32_t)(r & 7) << 4 : 0u;
-        const uint32_t crow =
-            code_stage(cs) +
-            (uint32_t)r * (FMT == TQ_FMT_B ? (b7 ? kB7Row : kBRow)
-                           : swz           ? kARowCodes
-                                           : kARow);
-        const uint32_t srow = swz ? code_stage(cs) + kAMapScales +
-                                        (uint32_t)r * kAMapSRow
-                                  : crow + kARowCodes;
-        // Format A: byte skews of the window's first group inside the code and
-        // scale rows (the same for every row with tensor copies)
-        uint32_t cskew = 0, sskew = 0;
-        int64_t g0 = 0;
-        if constexpr (FMT == TQ_FMT_A) {
-          const int plane = ws / P.kblocks;
-          g0 = 2 * (int64_t)(ws - plane * P.kblocks);
-          if (swz) {
-            cskew = (uint32_t)(13 * g0) & 15u;
-            sskew = 2u * ((uint32_t)g0 & 7u);
-          } else {
-            const int64_t gi = (row_ok ? row : 0) * gpr + g0;
-            cskew = (uint32_t)((reinterpret_cast<uintptr_t>(w.codes) +
-                                (uintptr_t)(plane * w.codes_plane_stride) +
-                                (uintptr_t)(gi * 13)) &
-                               15);
-            sskew = (uint32_t)((reinterpret_cast<uintptr_t>(w.scales) +
-                                (uintptr_t)(2 * (plane * w.scales_plane_stride +
-                                                 gi))) &
-                               15);
+    // One copy of the loop per decode variant, chosen once after the set-up:
+    // while stages flow, only the running variant's code is fetched (the
+    // variants together overflow the instruction cache).
+    auto decoders = [&](auto dec_tag) {
+      constexpr int DEC = decltype(dec_tag)::value;
+      constexpr bool kB7 = DEC == kDecB7Grid || DEC == kDecB7Pair;
+      constexpr bool kGrid =
+          DEC == kDecGrid || DEC == kDecIdent || DEC == kDecB7Grid;
+      const int q = warp & 3;
+      const int kp = (warp - kWarpDec) >> 2;  // which 64-k half of the block
+      const int r = 32 * q + lane;
+      const uint32_t lane_tab =
+          tab | (uint32_t)lane << (FMT == TQ_FMT_B ? 2 : 3);
+      const uint32_t t_hi =
+          tmem + ((uint32_t)(32 * q) << 16) + kAStage0 + 32u * (uint32_t)kp;
+      const bool skip_first = P.skip_first_arrive != 0;
+      int cs = 0, uc = 0, as = 0, ua = 0;
+      bool ok = true;
+      // this warp's compact book (adaptive alphabet)
+      const uint32_t ctab = tab + (uint32_t)(warp - kWarpDec) * 1024u;
+      for (int t = cid; ok && t < P.tiles; t += nclusters) {
+        const int64_t row = (int64_t)t * kTileM + r;
+        const bool row_ok = row < N;
+        if constexpr (DEC == kDecAdaptive) {
+          // rows t * 128 + 32 q .. + 31 share one book (lut_rows % 32 == 0);
+          // a warp wholly past N reads book 0 (its weights are masked)
+          const int64_t r0w = (int64_t)t * kTileM + 32 * q;
+          const float *bl = w.lut + ((r0w < N ? r0w : 0) / w.lut_rows) * 256;
+          __syncwarp();  // this warp's lookups of the previous tile are done
+          for (int e = lane; e < 256; e += 32) {
+            const float v = __ldg(bl + e);
+            const uint32_t h = bf16_bits_rn(v);
+            const uint32_t l = bf16_bits_rn(v - __uint_as_float(h << 16));
+            asm volatile("st.shared.u32 [%0], %1;" ::"r"(ctab + 4u * (uint32_t)e),
+                         "r"(h | l << 16)
+                         : "memory");
           }
-        }
-        for (int it = ws; it < we; ++it) {
-          if (ua >= kAStages) {
-            ok = __all_sync(0xFFFFFFFFu,
-                            mbar_wait(B0 + kBarAEmpty + 8 * as,
-                                      (uint32_t)((ua / kAStages) + 1) & 1u,
-                                      abort_addr, lim));
-            if constexpr (CK) if (!ok && lane == 0) ck_record(29, (uint64_t)ua);
-            if (!ok) break;
-          }
-          tc_fence_after_sync();
-          if (lane == 0 && q == 0 && kp == 0) ck_trace<CK>(trace, 5, t, it, 1);
-          uint32_t hi[32], lo[32];
-          if constexpr (FMT == TQ_FMT_B) {
-            // this half's 64 codes: four 16-byte loads. 7-bit alphabet: 56
-            // bytes, loaded from byte 0 (kp 0) or 48 (kp 1, the run starting
-            // 8 bytes in); its row pitch, 112, puts a quarter warp's 8 rows
-            // on 8 distinct 16-byte bank groups
-            const uint32_t hoff = (b7 ? 48u : 64u) * (uint32_t)kp;
-            uint32_t cw[16];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const uint32_t a = crow + ((hoff + 16u * (uint32_t)j) ^ sw);
-              const uint4 v4 = lds128(ck_smem<CK>(W, a, 16u, 16));
-              cw[4 * j] = v4.x;
-              cw[4 * j + 1] = v4.y;
-              cw[4 * j + 2] = v4.z;
-              cw[4 * j + 3] = v4.w;
-            }
-            if (b7) {
-              uint32_t d[14];
-#pragma unroll
-              for (int i = 0; i < 14; ++i) d[i] = kp ? cw[i + 2] : cw[i];
-              if (grid)
-                decode_b7<false>(d, lane_tab, hi, lo);
-              else
-                decode_b7<true>(d, lane_tab, hi, lo);
-            } else if (adaptive) {
-              decode_b_compact(cw, ctab, hi, lo);
-            } else if (ident) {
-              // an invalid code poisons its row: NaN operands
-              if (decode_b_arith(cw, hi) != 0u) {
-#pragma unroll
-                for (int m = 0; m < 32; ++m) hi[m] = 0x7FC07FC0u;
-              }
-            } else if (grid) {
-              decode_b_hi(cw, lane_tab, hi);
-            } else {
-              decode_b(cw, lane_tab, hi, lo);
-            }
-            // k past K (in the last block) and rows past N: zero weights
-            // (selects, no branch: the tcgen05.st below is warp-wide)
-            const int64_t kv = K - ((int64_t)it * kKB + 64 * kp);
-            if (__any_sync(0xFFFFFFFFu, kv < 64 || !row_ok)) {
-#pragma unroll
-              for (int m = 0; m < 32; ++m) {
-                const uint32_t keep = (row_ok && 2 * m < kv) ? 0xFFFFFFFFu : 0u;
-                hi[m] &= keep;
-                if (!grid) lo[m] &= keep;
-              }
-            }
-          } else {
-            const int gi = 2 * (it - ws) + kp;  // group inside the window
-            const bool valid = row_ok && g0 + gi < gpr;
-            const uint32_t o = cskew + 13u * (uint32_t)gi;
-            const uint32_t wl = o & ~3u;  // logical offsets wl .. wl + 15
-            const uint32_t sh = 8u * (o & 3u);
-            const uint32_t w0 = lds32(ck_smem<CK>(W, crow + (wl ^ sw), 4u, 17)),
-                           w1 = lds32(ck_smem<CK>(W, crow + ((wl + 4) ^ sw), 4u, 17)),
-                           w2 = lds32(ck_smem<CK>(W, crow + ((wl + 8) ^ sw), 4u, 17)),
-                           w3 = lds32(ck_smem<CK>(W, crow + ((wl + 12) ^ sw), 4u, 17));
-            const uint32_t b[4] = {__funnelshift_r(w0, w1, sh),
-                                   __funnelshift_r(w1, w2, sh),
-                                   __funnelshift_r(w2, w3, sh), w3 >> sh};
-            const uint32_t sa = srow + sskew + 2u * (uint32_t)gi;
-            const uint32_t sbits =
-                (lds32(ck_smem<CK>(W, sa & ~3u, 4u, 18)) >> (8u * (sa & 2u))) & 0xFFFFu;
-            const float sf = __half2float(__ushort_as_half((unsigned short)sbits));
-            const uint32_t h = bf16_bits_rn(sf);
-            const uint32_t l = bf16_bits_rn(sf - __uint_as_float(h << 16));
-            decode_a(b, lane_tab, h ^ 0x8000u, h, l ^ 0x8000u, l, hi, lo);
-            if (__any_sync(0xFFFFFFFFu, !valid)) {
-              const uint32_t keep = valid ? 0xFFFFFFFFu : 0u;
-#pragma unroll
-              for (int m = 0; m < 32; ++m) {
-                hi[m] &= keep;
-                lo[m] &= keep;
-              }
-            }
-          }
-          uint32_t ta = t_hi + (uint32_t)as * kAStageCols;
-          if constexpr (CK) ta = ck_tmem<CK>(ta, 96u, (uint32_t)(32 * q), 19);
-          __syncwarp();  // converged for the warp-wide stores
-          tmem_st32(ta, hi);
-          if (!grid) tmem_st32(ta + 64u, lo);
-          tmem_st_wait();
-          if (lane == 0 && q == 0 && kp == 0) ck_trace<CK>(trace, 5, t, it, 2);
-          tc_fence_before_sync();
           __syncwarp();
-          if (lane == 0 && !(skip_first && ua == 0))
-            mbar_arrive(B0 + kBarAFull + 8 * as);
-          ++ua;
-          as = as + 1 == kAStages ? 0 : as + 1;
         }
-        if (!ok) break;
-        // this warp is done reading the window
-        __syncwarp();
-        if (lane == 0) mbar_arrive(B0 + kBarCodeEmpty + 8 * cs);
-        ws = we;
-        ++uc;
-        cs = cs + 1 == P.code_stages ? 0 : cs + 1;
+        for (int ws = it0; ws < it1;) {
+          const int we = window_end(ws, it1, P.kblocks, kWin);
+          ok = __all_sync(0xFFFFFFFFu,
+                          mbar_wait(B0 + kBarCodeFull + 8 * cs,
+                                    (uint32_t)(uc / P.code_stages) & 1u,
+                                    abort_addr, lim));
+          if constexpr (CK) if (!ok && lane == 0) ck_record(28, (uint64_t)uc);
+          if (!ok) break;
+          // this row's codes (crow) and scales (srow) in the stage; a row
+          // written by a tensor copy is swizzled: logical byte o is at o ^ sw
+          const bool swz = (FMT == TQ_FMT_B && !kB7) || P.a_map;
+          const uint32_t sw = swz ? (uint32_t)(r & 7) << 4 : 0u;
+          const uint32_t crow =
+              code_stage(cs) +
+              (uint32_t)r * (FMT == TQ_FMT_B ? (kB7 ? kB7Row : kBRow)
+                             : swz           ? kARowCodes
+                                             : kARow);
+          const uint32_t srow = swz ? code_stage(cs) + kAMapScales +
+                                          (uint32_t)r * kAMapSRow
+                                    : crow + kARowCodes;
+          // Format A: byte skews of the window's first group inside the code and
+          // scale rows (the same for every row with tensor copies)
+          uint32_t cskew = 0, sskew = 0;
+          int64_t g0 = 0;
+          if constexpr (FMT == TQ_FMT_A) {
+            const int plane = ws / P.kblocks;
+            g0 = 2 * (int64_t)(ws - plane * P.kblocks);
+            if (swz) {
+              cskew = (uint32_t)(13 * g0) & 15u;
+              sskew = 2u * ((uint32_t)g0 & 7u);
+            } else {
+              const int64_t gi = (row_ok ? row : 0) * gpr + g0;
+              cskew = (uint32_t)((reinterpret_cast<uintptr_t>(w.codes) +
+                                  (uintptr_t)(plane * w.codes_plane_stride) +
+                                  (uintptr_t)(gi * 13)) &
+                                 15);
+              sskew = (uint32_t)((reinterpret_cast<uintptr_t>(w.scales) +
+                                  (uintptr_t)(2 * (plane * w.scales_plane_stride +
+                                                   gi))) &
+                                 15);
+            }
+          }
+          for (int it = ws; it < we; ++it) {
+            if (ua >= kAStages) {
+              ok = __all_sync(0xFFFFFFFFu,
+                              mbar_wait(B0 + kBarAEmpty + 8 * as,
+                                        (uint32_t)((ua / kAStages) + 1) & 1u,
+                                        abort_addr, lim));
+              if constexpr (CK) if (!ok && lane == 0) ck_record(29, (uint64_t)ua);
+              if (!ok) break;
+            }
+            tc_fence_after_sync();
+            if (lane == 0 && q == 0 && kp == 0) ck_trace<CK>(trace, 5, t, it, 1);
+            uint32_t hi[32], lo[32];
+            if constexpr (FMT == TQ_FMT_B) {
+              // this half's 64 codes: four 16-byte loads. 7-bit alphabet: 56
+              // bytes, loaded from byte 0 (kp 0) or 48 (kp 1, the run starting
+              // 8 bytes in); its row pitch, 112, puts a quarter warp's 8 rows
+              // on 8 distinct 16-byte bank groups
+              const uint32_t hoff = (kB7 ? 48u : 64u) * (uint32_t)kp;
+              uint32_t cw[16];
+  #pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const uint32_t a = crow + ((hoff + 16u * (uint32_t)j) ^ sw);
+                const uint4 v4 = lds128(ck_smem<CK>(W, a, 16u, 16));
+                cw[4 * j] = v4.x;
+                cw[4 * j + 1] = v4.y;
+                cw[4 * j + 2] = v4.z;
+                cw[4 * j + 3] = v4.w;
+              }
+              if constexpr (kB7) {
+                uint32_t d[14];
+  #pragma unroll
+                for (int i = 0; i < 14; ++i) d[i] = kp ? cw[i + 2] : cw[i];
+                decode_b7<!kGrid>(d, lane_tab, hi, lo);
+              } else if constexpr (DEC == kDecAdaptive) {
+                decode_b_compact(cw, ctab, hi, lo);
+              } else if constexpr (DEC == kDecIdent) {
+                // an invalid code poisons its row: NaN operands
+                if (decode_b_arith(cw, hi) != 0u) {
+  #pragma unroll
+                  for (int m = 0; m < 32; ++m) hi[m] = 0x7FC07FC0u;
+                }
+              } else if constexpr (DEC == kDecGrid) {
+                decode_b_hi(cw, lane_tab, hi);
+              } else {
+                decode_b(cw, lane_tab, hi, lo);
+              }
+              // k past K (in the last block) and rows past N: zero weights
+              // (selects, no branch: the tcgen05.st below is warp-wide)
+              const int64_t kv = K - ((int64_t)it * kKB + 64 * kp);
+              if (__any_sync(0xFFFFFFFFu, kv < 64 || !row_ok)) {
+  #pragma unroll
+                for (int m = 0; m < 32; ++m) {
+                  const uint32_t keep = (row_ok && 2 * m < kv) ? 0xFFFFFFFFu : 0u;
+                  hi[m] &= keep;
+                  if constexpr (!kGrid) lo[m] &= keep;
+                }
+              }
+            } else {
+              const int gi = 2 * (it - ws) + kp;  // group inside the window
+              const bool valid = row_ok && g0 + gi < gpr;
+              const uint32_t o = cskew + 13u * (uint32_t)gi;
+              const uint32_t wl = o & ~3u;  // logical offsets wl .. wl + 15
+              const uint32_t sh = 8u * (o & 3u);
+              const uint32_t w0 = lds32(ck_smem<CK>(W, crow + (wl ^ sw), 4u, 17)),
+                             w1 = lds32(ck_smem<CK>(W, crow + ((wl + 4) ^ sw), 4u, 17)),
+                             w2 = lds32(ck_smem<CK>(W, crow + ((wl + 8) ^ sw), 4u, 17)),
+                             w3 = lds32(ck_smem<CK>(W, crow + ((wl + 12) ^ sw), 4u, 17));
+              const uint32_t b[4] = {__funnelshift_r(w0, w1, sh),
+                                     __funnelshift_r(w1, w2, sh),
+                                     __funnelshift_r(w2, w3, sh), w3 >> sh};
+              const uint32_t sa = srow + sskew + 2u * (uint32_t)gi;
+              const uint32_t sbits =
+                  (lds32(ck_smem<CK>(W, sa & ~3u, 4u, 18)) >> (8u * (sa & 2u))) & 0xFFFFu;
+              const float sf = __half2float(__ushort_as_half((unsigned short)sbits));
+              const uint32_t h = bf16_bits_rn(sf);
+              const uint32_t l = bf16_bits_rn(sf - __uint_as_float(h << 16));
+              decode_a(b, lane_tab, h ^ 0x8000u, h, l ^ 0x8000u, l, hi, lo);
+              if (__any_sync(0xFFFFFFFFu, !valid)) {
+                const uint32_t keep = valid ? 0xFFFFFFFFu : 0u;
+  #pragma unroll
+                for (int m = 0; m < 32; ++m) {
+                  hi[m] &= keep;
+                  lo[m] &= keep;
+                }
+              }
+            }
+            uint32_t ta = t_hi + (uint32_t)as * kAStageCols;
+            if constexpr (CK) ta = ck_tmem<CK>(ta, 96u, (uint32_t)(32 * q), 19);
+            __syncwarp();  // converged for the warp-wide stores
+            tmem_st32(ta, hi);
+            if constexpr (!kGrid) tmem_st32(ta + 64u, lo);
+            tmem_st_wait();
+            if (lane == 0 && q == 0 && kp == 0) ck_trace<CK>(trace, 5, t, it, 2);
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0 && !(skip_first && ua == 0))
+              mbar_arrive(B0 + kBarAFull + 8 * as);
+            ++ua;
+            as = as + 1 == kAStages ? 0 : as + 1;
+          }
+          if (!ok) break;
+          // this warp is done reading the window
+          __syncwarp();
+          if (lane == 0) mbar_arrive(B0 + kBarCodeEmpty + 8 * cs);
+          ws = we;
+          ++uc;
+          cs = cs + 1 == P.code_stages ? 0 : cs + 1;
+        }
       }
+    };
+    if constexpr (FMT == TQ_FMT_B) {
+      if (b7) {
+        if (grid)
+          decoders(std::integral_constant<int, kDecB7Grid>{});
+        else
+          decoders(std::integral_constant<int, kDecB7Pair>{});
+      } else if (adaptive) {
+        decoders(std::integral_constant<int, kDecAdaptive>{});
+      } else if (ident) {
+        decoders(std::integral_constant<int, kDecIdent>{});
+      } else if (grid) {
+        decoders(std::integral_constant<int, kDecGrid>{});
+      } else {
+        decoders(std::integral_constant<int, kDecPair>{});
+      }
+    } else {
+      decoders(std::integral_constant<int, kDecPair>{});
     }
   }
 

@@ -116,3 +116,15 @@ def test_every_invalid_code_poisons_its_row(force_path, ladder, path):
         y, _ = U.linear(w, I.x_normal(batch, k, batch))
         assert np.all(np.isnan(y[:, bad_rows])), f"b={batch}"
         assert np.all(np.isfinite(np.delete(y, bad_rows, axis=1))), f"b={batch}"
+
+
+@pytest.mark.parametrize("path", [0, 3])
+def test_integer_grid_that_is_not_the_ternary_ladder(force_path, path):
+    # ladder 5, 4, 3, 2, 1: every entry is alpha times an integer (|m| <= 15)
+    # but not alpha * (c - 121) / 81: the single-operand table path (path 0)
+    # or the hi + lo pair (path 3)
+    lut = oref.build_lut(I.ALPHA, np.array([5, 4, 3, 2, 1], np.float32))
+    codes = I.codes_uniform(300, 2064, 17)
+    force_path(path)
+    _run(codes, lut, rho=I.rho_uniform(300, 4), rps=1,
+         label=f"ladder 5..1 path {path}")
