@@ -283,20 +283,24 @@ __device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
   return r;
 }
 
-// Format B, single operand, for a code book whose entry c is u * (c - 121)
-// (the balanced-ternary ladder 3^-(i-1): code byte c = 121 + sum t_i 3^i):
-// 64 codes of one row -> 32 bf16 pairs of c - 121, without table lookups.
-// A byte permute places code c in the low byte of the fp32 pattern of
-// 2^23 + c, a packed fp32 subtraction of 2^23 + 121 leaves c - 121 (exact),
-// and one conversion packs two of them. Returns non-zero iff a code of the
-// run is >= 243 (invalid): per byte, bit 7 of (c & 0x7F) + 0x0D is set iff
+// Format B, single operand, for a code book whose entry c is u * (c - 121),
+// i.e. entry c = alpha * sum t_i a_i with code byte c = 121 + sum t_i 3^(i-1)
+// and an ascending ternary ladder a_i = 3^(i-1) * a_1 (the least significant
+// trit on the smallest step; the ladder 3^-(i-1) pairs it with the largest
+// step and takes the table):
+// 16 codes (one 16-byte load) -> 8 bf16 pairs of c - 121, without table
+// lookups. A byte permute places code c in the low byte of the fp32 pattern
+// of 2^23 + c, a packed fp32 subtraction of 2^23 + 121 leaves c - 121
+// (exact), and one conversion packs two of them. Returns non-zero iff a code
+// is >= 243 (invalid): per byte, bit 7 of (c & 0x7F) + 0x0D is set iff
 // (c & 0x7F) >= 0x73, which with bit 7 of c set is c >= 0xF3.
-__device__ __forceinline__ uint32_t decode_b_arith(const uint32_t (&cw)[16],
-                                                   uint32_t (&hi)[32]) {
+__device__ __forceinline__ uint32_t decode_b_arith16(const uint4 v,
+                                                     uint32_t (&hi)[8]) {
   const float2 bias = make_float2(-8388729.0f, -8388729.0f);  // -(2^23 + 121)
+  const uint32_t cw[4] = {v.x, v.y, v.z, v.w};
   uint32_t bad = 0;
 #pragma unroll
-  for (int j = 0; j < 16; ++j) {
+  for (int j = 0; j < 4; ++j) {
     const uint32_t w = cw[j];
     float2 a = make_float2(__uint_as_float(prmt(w, 0x4B000000u, 0x7540u)),
                            __uint_as_float(prmt(w, 0x4B000000u, 0x7541u)));
@@ -646,7 +650,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       id_ok = m == (float)((int)threadIdx.x - 121);
     }
     grid = __syncthreads_and(ok) != 0 && P.grid_ok != 0;
-    // m = c - 121 for every word: decode without the table
+    // m = c - 121 for every word (an ascending ternary ladder): decode
+    // without the table
     const bool all_id = __syncthreads_and(id_ok) != 0;
     ident = grid && !b7 && all_id;
     if (grid) unit = u;
@@ -1192,7 +1197,38 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after_sync();
             if (lane == 0 && q == 0 && kp == 0) ck_trace<CK>(trace, 5, t, it, 1);
             uint32_t hi[32], lo[32];
-            if constexpr (FMT == TQ_FMT_B) {
+            uint32_t ta = t_hi + (uint32_t)as * kAStageCols;
+            if constexpr (CK) ta = ck_tmem<CK>(ta, 96u, (uint32_t)(32 * q), 19);
+            if constexpr (FMT == TQ_FMT_B && DEC == kDecIdent) {
+              // table-free decode in 4 chunks of 16 codes, each stored to
+              // tensor memory (8 columns) at once: a short loop body keeps
+              // the decoder's hot code small. An invalid code poisons its
+              // chunk (NaN operands), which poisons the row's sums; k past
+              // K (in the last block) and rows past N get zero weights.
+              const int64_t kv = K - ((int64_t)it * kKB + 64 * kp);
+              const bool edge = __any_sync(0xFFFFFFFFu, kv < 64 || !row_ok);
+#pragma unroll 1
+              for (int j = 0; j < 4; ++j) {
+                const uint32_t a =
+                    crow + ((64u * (uint32_t)kp + 16u * (uint32_t)j) ^ sw);
+                uint32_t h8[8];
+                if (decode_b_arith16(lds128(ck_smem<CK>(W, a, 16u, 16)), h8) !=
+                    0u) {
+#pragma unroll
+                  for (int m = 0; m < 8; ++m) h8[m] = 0x7FC07FC0u;
+                }
+                if (edge) {
+#pragma unroll
+                  for (int m = 0; m < 8; ++m) {
+                    const uint32_t keep =
+                        (row_ok && 2 * (8 * j + m) < kv) ? 0xFFFFFFFFu : 0u;
+                    h8[m] &= keep;
+                  }
+                }
+                __syncwarp();  // converged for the warp-wide store
+                tmem_st8(ta + 8u * (uint32_t)j, h8);
+              }
+            } else if constexpr (FMT == TQ_FMT_B) {
               // this half's 64 codes: four 16-byte loads. 7-bit alphabet: 56
               // bytes, loaded from byte 0 (kp 0) or 48 (kp 1, the run starting
               // 8 bytes in); its row pitch, 112, puts a quarter warp's 8 rows
@@ -1215,12 +1251,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 decode_b7<!kGrid>(d, lane_tab, hi, lo);
               } else if constexpr (DEC == kDecAdaptive) {
                 decode_b_compact(cw, ctab, hi, lo);
-              } else if constexpr (DEC == kDecIdent) {
-                // an invalid code poisons its row: NaN operands
-                if (decode_b_arith(cw, hi) != 0u) {
-  #pragma unroll
-                  for (int m = 0; m < 32; ++m) hi[m] = 0x7FC07FC0u;
-                }
               } else if constexpr (DEC == kDecGrid) {
                 decode_b_hi(cw, lane_tab, hi);
               } else {
@@ -1266,11 +1296,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
               }
             }
-            uint32_t ta = t_hi + (uint32_t)as * kAStageCols;
-            if constexpr (CK) ta = ck_tmem<CK>(ta, 96u, (uint32_t)(32 * q), 19);
-            __syncwarp();  // converged for the warp-wide stores
-            tmem_st32(ta, hi);
-            if constexpr (!kGrid) tmem_st32(ta + 64u, lo);
+            if constexpr (!(FMT == TQ_FMT_B && DEC == kDecIdent)) {
+              __syncwarp();  // converged for the warp-wide stores
+              tmem_st32(ta, hi);
+              if constexpr (!kGrid) tmem_st32(ta + 64u, lo);
+            }
             tmem_st_wait();
             if (lane == 0 && q == 0 && kp == 0) ck_trace<CK>(trace, 5, t, it, 2);
             tc_fence_before_sync();

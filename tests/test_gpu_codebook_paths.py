@@ -9,8 +9,9 @@ would take the single path (tq_testing_force_linear_path(3)), and check that
 an entry just off the grid is not forced onto it: with every code of a row
 equal and x all ones, an entry rounded onto the grid would miss by about
 1e-3 * K * |w|, far outside the tolerance. A book with entry c = u * (c - 121)
-(the balanced-ternary ladder, any alpha) is decoded without its table; every
-invalid byte value 243..255 must still make its row NaN on each path."""
+(an ascending ternary ladder 1/81 .. 1, any alpha: the least significant trit
+on the smallest step) is decoded without its table; every invalid byte value
+243..255 must still make its row NaN on each path."""
 import numpy as np
 import pytest
 import torch
@@ -24,6 +25,8 @@ pytestmark = pytest.mark.gpu
 BATCHES = (5, 16, 33, 64)
 # a ladder whose 243 sums are not on one grid (the encoder's test ladder)
 LADDER_FREE = np.array([1.0, 0.33, 0.115, 0.037, 0.012], np.float32)
+# an ascending ternary ladder: entry c = alpha * (c - 121) / 81
+LADDER_ASC = np.array([1 / 81, 1 / 27, 1 / 9, 1 / 3, 1], np.float32)
 
 
 @pytest.fixture
@@ -96,13 +99,15 @@ def test_integer_ladder_and_zero_book():
 
 
 @pytest.mark.parametrize("ladder,path", [("pow3", 0), ("pow3", 3),
-                                         ("free", 0)])
+                                         ("free", 0), ("asc", 0), ("asc", 3)])
 def test_every_invalid_code_poisons_its_row(force_path, ladder, path):
     # one invalid byte (243..255) per row in rows 0..12, at k positions that
     # fall in both 64-k halves of a block, in different blocks and at the
-    # last k; the balanced-ternary book takes the table-free decode (path 0)
-    # or the hi + lo table (path 3), the free ladder the hi + lo table
-    lad = I.ladder_pow3().numpy() if ladder == "pow3" else LADDER_FREE
+    # last k; the ascending ternary ladder takes the table-free decode
+    # (path 0), the ladder 3^-(k-1) the single-operand table (path 0) or the
+    # hi + lo table (path 3), the free ladder the hi + lo table
+    lad = {"pow3": I.ladder_pow3().numpy(), "free": LADDER_FREE,
+           "asc": LADDER_ASC}[ladder]
     lut = oref.build_lut(I.ALPHA, lad)
     n, k = 141, 1024
     codes = I.codes_uniform(n, k, 31)
@@ -128,3 +133,18 @@ def test_integer_grid_that_is_not_the_ternary_ladder(force_path, path):
     force_path(path)
     _run(codes, lut, rho=I.rho_uniform(300, 4), rps=1,
          label=f"ladder 5..1 path {path}")
+
+
+@pytest.mark.parametrize("path", [0, 3])
+@pytest.mark.parametrize("n,k,rps", [(300, 2064, 0), (257, 4096, 1),
+                                     (1000, 2048, 128)])
+def test_ascending_ternary_ladder_table_free(force_path, path, n, k, rps):
+    # entry c = alpha * (c - 121) / 81: the table-free decode (path 0) and the
+    # hi + lo table (path 3), ragged rows and blocks, rho per row and per head
+    lut = oref.build_lut(I.ALPHA, LADDER_ASC)
+    m = np.rint(lut[:243] / (I.ALPHA / 81)).astype(np.int64)
+    assert np.array_equal(m, np.arange(243) - 121)  # the book is c - 121
+    codes = I.codes_uniform(n, k, n + 3 * k)
+    rho = I.rho_uniform(I.rho_count(n, rps), 6) if rps else None
+    force_path(path)
+    _run(codes, lut, rho, rps, label=f"ascending ladder path {path} {n}x{k}")
