@@ -696,16 +696,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kWarpCodes) {
     // ---- code producer: each window's codes (and scales) ---------------------
     int s = 0, u = 0;  // ring slot, windows issued so far
+    uint32_t ph = 0;   // (u / code_stages) & 1, kept without a division
     bool ok = true;
     for (int t = cid; ok && t < P.tiles; t += nclusters) {
       const int64_t row0 = (int64_t)t * kTileM;
       const int rows = (int)(N - row0 < kTileM ? N - row0 : kTileM);
       for (int ws = it0; ws < it1;) {
-        const int we = window_end(ws, it1, P.kblocks, kWin);
+        const int we =
+            FMT == TQ_FMT_B ? ws + 1 : window_end(ws, it1, P.kblocks, kWin);
         if (u >= P.code_stages)
-          ok = mbar_wait(B0 + kBarCodeEmpty + 8 * s,
-                         (uint32_t)((u / P.code_stages) + 1) & 1u, abort_addr,
-                         lim);
+          ok = mbar_wait(B0 + kBarCodeEmpty + 8 * s, ph ^ 1u, abort_addr, lim);
         ok = __all_sync(0xFFFFFFFFu, ok);
         if constexpr (CK) if (!ok && lane == 0) ck_record(21, (uint64_t)u);
         if (!ok) break;
@@ -781,7 +781,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) ck_trace<CK>(trace, 0, t, ws, 2);
         ws = we;
         ++u;
-        s = s + 1 == P.code_stages ? 0 : s + 1;
+        if (++s == P.code_stages) {
+          s = 0;
+          ph ^= 1u;
+        }
       }
     }
     if (lane == 0) ck_trace<CK>(trace, 0, 0xFFFF, 0, 3);
@@ -798,21 +801,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     // swizzle: the K-major layout the MMA reads)
     if (lane == 0) {
       int s = 0, u = 0;
+      uint32_t ph = 0;  // (u / x_stages) & 1, kept without a division
       bool ok = true;
       const uint32_t half = (uint32_t)n_pad * 128u;
       for (int t = cid; ok && t < P.tiles; t += nclusters) {
         for (int it = it0; it < it1; ++it) {
           if (u >= P.x_stages &&
-              !mbar_wait(B0 + kBarXEmpty + 8 * s,
-                         (uint32_t)((u / P.x_stages) + 1) & 1u, abort_addr,
-                         lim)) {
+              !mbar_wait(B0 + kBarXEmpty + 8 * s, ph ^ 1u, abort_addr, lim)) {
             if constexpr (CK) ck_record(22, (uint64_t)u);
             ok = false;
             break;
           }
           const uint32_t full = B0 + kBarXFull + 8 * s;
           const uint32_t dst = x_ring + (uint32_t)s * P.x_stage_bytes;
-          const int k0 = (it % P.kblocks) * kKB;
+          const int k0 = (it < P.kblocks ? it : it % P.kblocks) * kKB;
           ck_trace<CK>(trace, 1, t, it, 1);
           mbar_arrive_expect_tx(full, 2u * half);
           for (int h = 0; h < 2; ++h) {
@@ -824,7 +826,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_2d(d, &tmap_x, k0 + 64 * h, 0, full);
           }
           ++u;
-          s = s + 1 == P.x_stages ? 0 : s + 1;
+          if (++s == P.x_stages) {
+            s = 0;
+            ph ^= 1u;
+          }
         }
       }
       for (int j = u > P.x_stages ? u - P.x_stages : 0; j < u; ++j)
@@ -916,6 +921,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // sides stop at the first failed stage, so they take the same number of
     // reductions.
     int xs = 0, ux = 0, as = 0, ua = 0;
+    uint32_t xph = 0, aph = 0;  // phases of the x and A rings
     bool ok = true;
     int i = 0;
     for (int t = cid; ok && t < P.tiles; t += nclusters, ++i) {
@@ -927,19 +933,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       if constexpr (CK) if (!acc_ok && lane == 0) ck_record(23, (uint64_t)i);
       for (int it = it0; it < it1; ++it) {
         bool got = acc_ok &&
-                   mbar_wait(B0 + kBarXFull + 8 * xs,
-                             (uint32_t)(ux / P.x_stages) & 1u, abort_addr,
-                             lim) &&
-                   mbar_wait(B0 + kBarAFull + 8 * as,
-                             (uint32_t)(ua / kAStages) & 1u, abort_addr, lim);
+                   mbar_wait(B0 + kBarXFull + 8 * xs, xph, abort_addr, lim) &&
+                   mbar_wait(B0 + kBarAFull + 8 * as, aph, abort_addr, lim);
         got = __all_sync(0xFFFFFFFFu, got);
         if constexpr (CK) if (!got && lane == 0) ck_record(24, (uint64_t)ux << 32 | (uint32_t)ua);
         ok = bar_red_and(kBarIdStage, 64, got);
         if (!ok) break;
         ++ux;
-        xs = xs + 1 == P.x_stages ? 0 : xs + 1;
+        if (++xs == P.x_stages) {
+          xs = 0;
+          xph ^= 1u;
+        }
         ++ua;
-        as = as + 1 == kAStages ? 0 : as + 1;
+        if (++as == kAStages) {
+          as = 0;
+          aph ^= 1u;
+        }
       }
     }
   } else if (warp < kWarpDec) {
@@ -1121,6 +1130,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem + ((uint32_t)(32 * q) << 16) + kAStage0 + 32u * (uint32_t)kp;
       const bool skip_first = P.skip_first_arrive != 0;
       int cs = 0, uc = 0, as = 0, ua = 0;
+      uint32_t cph = 0, aph = 0;  // phases of the code and A rings
       bool ok = true;
       // this warp's compact book (adaptive alphabet)
       const uint32_t ctab = tab + (uint32_t)(warp - kWarpDec) * 1024u;
@@ -1144,11 +1154,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           __syncwarp();
         }
         for (int ws = it0; ws < it1;) {
-          const int we = window_end(ws, it1, P.kblocks, kWin);
-          ok = __all_sync(0xFFFFFFFFu,
-                          mbar_wait(B0 + kBarCodeFull + 8 * cs,
-                                    (uint32_t)(uc / P.code_stages) & 1u,
-                                    abort_addr, lim));
+          // Format B: one block per window (no division on the hot path)
+          const int we =
+              FMT == TQ_FMT_B ? ws + 1 : window_end(ws, it1, P.kblocks, kWin);
+          ok = __all_sync(0xFFFFFFFFu, mbar_wait(B0 + kBarCodeFull + 8 * cs,
+                                                 cph, abort_addr, lim));
           if constexpr (CK) if (!ok && lane == 0) ck_record(28, (uint64_t)uc);
           if (!ok) break;
           // this row's codes (crow) and scales (srow) in the stage; a row
@@ -1188,8 +1198,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int it = ws; it < we; ++it) {
             if (ua >= kAStages) {
               ok = __all_sync(0xFFFFFFFFu,
-                              mbar_wait(B0 + kBarAEmpty + 8 * as,
-                                        (uint32_t)((ua / kAStages) + 1) & 1u,
+                              mbar_wait(B0 + kBarAEmpty + 8 * as, aph ^ 1u,
                                         abort_addr, lim));
               if constexpr (CK) if (!ok && lane == 0) ck_record(29, (uint64_t)ua);
               if (!ok) break;
@@ -1308,7 +1317,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0 && !(skip_first && ua == 0))
               mbar_arrive(B0 + kBarAFull + 8 * as);
             ++ua;
-            as = as + 1 == kAStages ? 0 : as + 1;
+            if (++as == kAStages) {
+              as = 0;
+              aph ^= 1u;
+            }
           }
           if (!ok) break;
           // this warp is done reading the window
@@ -1316,7 +1328,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) mbar_arrive(B0 + kBarCodeEmpty + 8 * cs);
           ws = we;
           ++uc;
-          cs = cs + 1 == P.code_stages ? 0 : cs + 1;
+          if (++cs == P.code_stages) {
+            cs = 0;
+            cph ^= 1u;
+          }
         }
       }
     };
