@@ -90,19 +90,6 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar,
       : "memory");
 }
 
-// Store `v` to the word at this CTA's shared address `addr` in the cluster's
-// CTA `rank`.
-__device__ __forceinline__ void st_cluster_s32(uint32_t addr, uint32_t rank,
-                                               int v) {
-  uint32_t remote;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
-               : "=r"(remote)
-               : "r"(addr), "r"(rank));
-  asm volatile("st.relaxed.cluster.shared::cluster.u32 [%0], %1;" ::"r"(remote),
-               "r"(v)
-               : "memory");
-}
-
 __device__ __forceinline__ int ld_volatile_s32(uint32_t addr) {
   int v;
   asm volatile("ld.volatile.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr)

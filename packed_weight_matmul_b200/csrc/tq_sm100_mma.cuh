@@ -18,18 +18,6 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
          ((uint32_t)(M >> 4) << 24);
 }
 
-// Shared-memory matrix descriptor for a K-major operand without swizzle:
-// core matrices of 8 rows x 16 bytes (rows 16 bytes apart); the second
-// 16-byte column of a k16 step sits LBO bytes after the first, the next 8
-// rows SBO bytes after these. Address, LBO and SBO are stored >> 4; bits
-// 46-47 hold the descriptor version (1 on sm_100); layout type 0 = none.
-__device__ __forceinline__ uint64_t smem_desc_kmajor(uint32_t addr, uint32_t lbo,
-                                                     uint32_t sbo) {
-  return (uint64_t)((addr >> 4) & 0x3FFFu) |
-         ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
-         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
-}
-
 // Shared-memory matrix descriptor for a K-major operand in the 128-byte
 // swizzle layout (as a tensor copy with the 128-byte swizzle writes it):
 // rows of 64 16-bit elements (128 bytes) 128 bytes apart, 16-byte chunk c of
@@ -69,12 +57,6 @@ __device__ __forceinline__ void tc_fence_after_sync() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// Make this thread's generic-proxy shared-memory writes visible to the async
-// proxy (the tensor cores read operands through it).
-__device__ __forceinline__ void fence_async_shared() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 // D[tmem] (+)= A[tmem] * B[smem desc]^T, one thread issues. A (M = 128 rows
 // on the 128 lanes) sits in tensor memory with K along the columns, two
 // 16-bit elements per 32-bit column, the lower k in the low half.
@@ -111,19 +93,6 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
       : "r"(taddr));
 }
 
-// Warp-wide: store 16 consecutive 32-bit columns of this warp's 32 TMEM
-// lanes (lane i of the warp writes TMEM lane base + i).
-__device__ __forceinline__ void tmem_st16(uint32_t taddr,
-                                          const uint32_t (&v)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
-      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]),
-      "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]),
-      "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
-      : "memory");
-}
-
 // Warp-wide: store 32 consecutive 32-bit columns of this warp's 32 lanes.
 __device__ __forceinline__ void tmem_st32(uint32_t taddr,
                                           const uint32_t (&v)[32]) {
@@ -141,6 +110,7 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr,
       : "memory");
 }
 
+// Warp-wide: store 8 consecutive 32-bit columns of this warp's 32 lanes.
 __device__ __forceinline__ void tmem_st8(uint32_t taddr,
                                          const uint32_t (&v)[8]) {
   asm volatile(
