@@ -63,6 +63,14 @@
  *     the kernel's work early; tq_linear then leaves NaN in every output it
  *     could not finish, which is how a time-out is reported. TQ_ERR_TIMEOUT is
  *     reserved: no entry point returns it.
+ *   - tq_linear's kernels are launched with programmatic dependent launch:
+ *     one may begin its set-up (and hint the L2 cache with its first code
+ *     bytes) while the kernel before it on the stream finishes, but it reads
+ *     no user memory and writes nothing before that kernel has completed, so
+ *     stream order holds as for any launch.
+ *   - tq_linear is deterministic: for the same inputs, shapes and device,
+ *     every output is bit-identical from call to call (partial sums are added
+ *     in a fixed order).
  */
 #ifndef TQ_H
 #define TQ_H
