@@ -1111,6 +1111,9 @@ def run_tq(args, world, rank, local):
     e2e_ms = dist_max(e_start.elapsed_time(e_end), world)
     e2e_value = world * step_bytes * args.steps / (e2e_ms / 1e3) / 1e9
 
+    # read-only streaming reference on this GPU, in the same run
+    read_ref = hbm_read_reference()
+
     if rank != 0:
         return
     pk = peaks()
@@ -1124,6 +1127,10 @@ def run_tq(args, world, rank, local):
         "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic", "config": wl.describe(),
         "pct_hbm_peak": 100.0 * value / world / pk["hbm_gbs"],
+        "pct_hbm_nominal": 100.0 * value / world / HBM_NOMINAL_GBS,
+        "hbm_read_ref": read_ref,
+        "pct_hbm_read_ref": (100.0 * value / world / read_ref["gbs"]
+                             if read_ref.get("gbs") else None),
         "roofline": roofline(s, per[dom], pk, wl),
         "per_graph_ms": {st.name: float(p) for st, p in zip(steps, per)},
         "per_graph_gbs": {st.name: st.bytes / (p / 1e3) / 1e9
@@ -1143,6 +1150,37 @@ def run_tq(args, world, rank, local):
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
     print(json.dumps(line), flush=True)
+
+
+HBM_NOMINAL_GBS = 8000.0  # B200 HBM3e, nominal
+
+
+def hbm_read_reference(nbytes=2 ** 31, reps=5):
+    """Read bandwidth of this GPU measured in the same run: a torch fp32
+    reduction over a 2 GiB buffer (it reads every byte once and writes one
+    value), CUDA events, median of `reps` after two warm-up passes. A
+    measurement reference for the % figures, not part of the library."""
+    try:
+        buf = torch.ones(nbytes // 4, dtype=torch.float32, device="cuda")
+        for _ in range(2):
+            buf.sum()
+        times = []
+        for _ in range(reps):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            buf.sum()
+            b.record()
+            torch.cuda.synchronize()
+            times.append(a.elapsed_time(b))
+        del buf
+        torch.cuda.empty_cache()
+        t_ms = float(np.median(times))
+        return {"gbs": nbytes / (t_ms / 1e3) / 1e9, "bytes": nbytes,
+                "method": "torch.sum over a 2 GiB fp32 buffer (read once), "
+                          "CUDA events, median of 5"}
+    except Exception as e:  # the reference is optional; the line is not
+        return {"gbs": None, "error": str(e)[:200]}
 
 
 def roofline(step, ms, pk, wl):
