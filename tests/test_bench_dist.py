@@ -68,3 +68,29 @@ def test_reference_arm_under_torchrun_world2():
     assert line["value"] > 0 and line["unit"] == "GB/s"
     assert line["cpu_baseline"]["kind"] == "oracle"
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_reference_arm_default_workload_line():
+    # the default workload's reference arm (the oracle as it stands, on host
+    # cores) prints one JSON line with the keys of the bench contract
+    cmd = [sys.executable, "bench.py", "--impl", "reference", "--steps", "1",
+           "--warmup", "1", "--ref-seconds", "2"]
+    r = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True,
+                       timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps",
+                "warmup", "ms_per_step", "higher_is_better", "scaling",
+                "vs_baseline", "dtype", "data", "config", "cpu_baseline",
+                "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["n_gpus"] == 1
+    assert line["config"]["workload"].startswith("decode_step")
+    assert line["higher_is_better"] is True and line["unit"] == "GB/s"
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["sample"]
+    assert cb["value"] == line["value"]
+    assert line["e2e"] == {"value": line["value"], "unit": "GB/s",
+                           "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
